@@ -1,0 +1,385 @@
+"""Prefill, full-depth autoregressive decoding and the pipelined speculative
+state machine -- the oracle's normative step order (test infrastructure only).
+
+Follows "LoopSpec: Pipelined Self-Speculative Decoding for Looped Transformers"
+(liuzhao09.github.io/papers/loopspec.html):
+  * section 1 / 3.1: the baseline is full-depth autoregressive decoding -- each
+    position runs all R loops, then commits;
+  * section 2.2: after prefill the first token is committed at full depth; a
+    branch is a fixed prefix plus its current loop depth; all active branches
+    advance the shared block together; at depth d1 a branch reads q1 = p_d1,
+    draws x1 and at once opens a child for prefix + x1; the parent continues to
+    R and verifies; on acceptance the child is kept, on rejection every
+    descendant of the wrong prefix is pruned and decoding restarts from the
+    correct prefix; Fig. 1 gives the loop-step counts 12 / 9 / 7;
+  * section 2.3: at d2 the gate of Eq. 6 decides whether a second child is
+    opened with x2 ~ q2 = p_d2 (-) q1; the cascade verifies x1, then x2 against
+    rho1; the tree is re-rooted on every verification; tokens with equal text
+    but different prefixes are different branches;
+  * section 2.4: a new branch copies its parent's cache indices (not KV);
+    pruning frees only what no surviving path needs.
+
+Step order (a reading of the pages, fixed here and followed by the CUDA
+engine bit for bit):
+  1. prelude for every branch at depth 0 (ascending uid);
+  2. every branch runs loop iteration depth+1 (ascending uid);
+  3. readouts for branches whose depth is in {d1, d2, R};
+  4. proposals, ascending uid: depth == d1 -> x1 ~ q1 = p_d1, child1 (lowest
+     free slot, next uid); depth == d2 and x1 drawn -> gate; if open
+     x2 ~ q2 = p_d2 (-) q1, child2.  Proposals are always drawn; a child is
+     created only if its own next token is still needed (pos + 1 < P + N).
+     A child's first iteration is in the next step;
+  5. if the root (prefix == committed) reached R: verify (cascade) and commit;
+  6. prune every branch whose prefix does not extend the new committed
+     sequence (its slots are freed after this step's allocations); the kept
+     child becomes the root and its slot is appended to the committed slots;
+     with no kept child a new root (depth 0) is created after the frees
+     (unless that commit was the last one).
+"""
+from __future__ import annotations
+
+import dataclasses
+from typing import Any, Dict, List, Optional, Sequence, Tuple
+
+import numpy as np
+
+from . import sampling as S
+
+
+# ----------------------------------------------------------------------------
+# model adapters
+# ----------------------------------------------------------------------------
+
+
+class OracleRows:
+    """Adapter from the state machine's row calls to the fp64 LoopedModel."""
+
+    def __init__(self, model):
+        self.m = model
+
+    def prelude(self, prefix: Sequence[int], pos: int, slots: Sequence[int]):
+        return self.m.prelude(int(prefix[-1]), pos, slots)
+
+    def iterate(self, h, r: int, prefix, pos: int, slots):
+        return self.m.iterate(h, r, pos, slots)
+
+    def readout(self, h, r: int, prefix, pos: int, slots, head: bool = True):
+        hc = self.m.coda(h, r, pos, slots)
+        return self.m.logits(hc) if head else None
+
+
+# ----------------------------------------------------------------------------
+# results
+# ----------------------------------------------------------------------------
+
+
+@dataclasses.dataclass
+class Stats:
+    steps: int = 0
+    rows_sum: int = 0
+    rows_max: int = 0
+    n_first: int = 0
+    n_second: int = 0
+    n_fallback: int = 0
+    gate_checks: int = 0
+    gate_opens: int = 0
+    branches_created: int = 0
+    resid_fallback: int = 0
+
+    def gamma(self, d1: int, d2: int, R: int) -> float:
+        """Mean acceptance length, Eq. 9 (section 3.2)."""
+        n = self.n_first + self.n_second + self.n_fallback
+        den = self.n_first * d1 + self.n_second * d2 + self.n_fallback * R
+        return n * R / den if den else float("nan")
+
+
+@dataclasses.dataclass
+class DecodeResult:
+    tokens: List[int]  # committed after the prompt: x_1 (prefill) then the decode tokens
+    src: List[int]  # per decode token: 1 first proposal, 2 second, 0 full-depth draw
+    commit_step: List[int]  # per decode token: step index (1-based) of its commit
+    committed_slots: List[int]
+    stats: Stats
+    trace: List[List[Tuple[int, int, int, int]]]  # per step: (uid, slot, pos, depth) sorted by uid
+    logits: Dict[Tuple[int, int], np.ndarray]  # optional readout logits keyed (pos, depth)
+
+
+# ----------------------------------------------------------------------------
+# prefill and first commit (section 2.2)
+# ----------------------------------------------------------------------------
+
+
+def readout_depths(R: int, d1: int, d2: int) -> List[int]:
+    return sorted({r for r in (d1, d2, R) if r > 0})
+
+
+def prefill(rows, prompt: Sequence[int], R: int, tags: Sequence[int],
+            keep_logits: bool = False) -> Dict[Tuple[int, int], np.ndarray]:
+    """Prompt positions 0..P-1 at slots 0..P-1, all depths, readouts (coda caches)
+    at every depth in ``tags``.  Returns logits at (P-1, R), plus every (pos, tag)
+    when ``keep_logits``."""
+    P = len(prompt)
+    out: Dict[Tuple[int, int], np.ndarray] = {}
+    for pos in range(P):
+        slots = list(range(pos + 1))
+        prefix = list(prompt[:pos + 1])
+        h = rows.prelude(prefix, pos, slots)
+        for r in range(1, R + 1):
+            h = rows.iterate(h, r, prefix, pos, slots)
+            if r in tags:
+                head = keep_logits or (pos == P - 1 and r == R)
+                z = rows.readout(h, r, prefix, pos, slots, head=head)
+                if head:
+                    out[(pos, r)] = z
+    return out
+
+
+def first_token(z_R: np.ndarray, P: int, temperature: float, top_p: float, seed: int) -> int:
+    p = S.process(z_R, temperature, top_p)
+    return S.race(p, seed, P, S.AR)
+
+
+# ----------------------------------------------------------------------------
+# full-depth autoregressive decoding (the comparison baseline)
+# ----------------------------------------------------------------------------
+
+
+def decode_ar(rows, prompt: Sequence[int], R: int, max_new: int, temperature: float,
+              top_p: float, seed: int, keep_logits: bool = False) -> DecodeResult:
+    """Each position runs all R loops, reads out at R and commits.  The token
+    at position j is drawn with the stream (j, AR)."""
+    P = len(prompt)
+    zs = prefill(rows, prompt, R, [R], keep_logits)
+    committed = list(prompt) + [first_token(zs[(P - 1, R)], P, temperature, top_p, seed)]
+    cslots = list(range(P + 1))
+    st = Stats()
+    logits = dict(zs) if keep_logits else {}
+    src, cstep = [], []
+    for _ in range(max_new):
+        pos = len(committed) - 1
+        slots = cslots[:pos + 1]
+        h = rows.prelude(committed, pos, slots)
+        for r in range(1, R + 1):
+            h = rows.iterate(h, r, committed, pos, slots)
+            st.steps += 1
+            st.rows_sum += 1
+            st.rows_max = 1
+        z = rows.readout(h, R, committed, pos, slots)
+        if keep_logits:
+            logits[(pos, R)] = z
+        p = S.process(z, temperature, top_p)
+        committed.append(S.race(p, seed, pos + 1, S.AR))
+        cslots.append(pos + 1)
+        src.append(S.SRC_FALLBACK)
+        st.n_fallback += 1
+        cstep.append(st.steps)
+    return DecodeResult(committed[P:], src, cstep, cslots, st, [], logits)
+
+
+# ----------------------------------------------------------------------------
+# pipelined speculative decoding (sections 2.2-2.4)
+# ----------------------------------------------------------------------------
+
+
+@dataclasses.dataclass
+class Branch:
+    uid: int
+    parent: int
+    slot: int
+    pos: int  # position of the prefix's last token
+    token: int  # that token
+    chain: Dict[int, int]  # pos -> slot for uncommitted positions of the prefix
+    depth: int = 0
+    state: Any = None
+    p: Optional[np.ndarray] = None  # this step's processed readout
+    x1: int = -1
+    q1: Optional[np.ndarray] = None
+    gate: bool = False
+    x2: int = -1
+    q2: Optional[np.ndarray] = None
+    child1: int = -1
+    child2: int = -1
+
+
+class SpecDecoder:
+    """The pipelined self-speculative decoder.  ``second``: "gated" (the method),
+    "ungated" (residual second proposal always opened) or "masked" (ablation,
+    section 3.4).  ``d2 = 0``: single proposal."""
+
+    def __init__(self, rows, prompt: Sequence[int], R: int, d1: int, d2: int, max_new: int,
+                 temperature: float, top_p: float, seed: int, n_slots: int,
+                 second: str = "gated", keep_trace: bool = True, keep_logits: bool = False,
+                 skip_prefill: bool = False, first: Optional[int] = None):
+        assert 1 <= d1 < R and (d2 == 0 or d1 < d2 < R)
+        self.rows, self.R, self.d1, self.d2 = rows, R, d1, d2
+        self.T, self.top_p, self.seed = temperature, top_p, seed
+        self.second = second
+        self.keep_trace, self.keep_logits = keep_trace, keep_logits
+        P = len(prompt)
+        self.P, self.max_new = P, max_new
+        self.pos_limit = P + max_new  # children only for positions < pos_limit
+        self.tags = readout_depths(R, d1, d2)
+        self.logits: Dict[Tuple[int, int], np.ndarray] = {}
+        if skip_prefill:
+            x1 = first
+        else:
+            zs = prefill(rows, prompt, R, self.tags, keep_logits)
+            if keep_logits:
+                self.logits.update(zs)
+            x1 = first_token(zs[(P - 1, R)], P, temperature, top_p, seed)
+        self.committed = list(prompt) + [x1]
+        self.cslots = list(range(P))
+        self.free = set(range(P, n_slots))
+        self.branches: Dict[int, Branch] = {}
+        self.next_uid = 0
+        self.stats = Stats()
+        self.src: List[int] = []
+        self.cstep: List[int] = []
+        self.trace: List[List[Tuple[int, int, int, int]]] = []
+        root = self._new_branch(-1, P, x1, {})
+        self.cslots.append(root.slot)
+
+    # -- bookkeeping -----------------------------------------------------------
+    def _alloc(self) -> int:
+        if not self.free:
+            raise RuntimeError("slot pool exhausted")
+        s = min(self.free)
+        self.free.remove(s)
+        return s
+
+    def _new_branch(self, parent: int, pos: int, token: int, chain: Dict[int, int]) -> Branch:
+        b = Branch(self.next_uid, parent, self._alloc(), pos, token, dict(chain))
+        b.chain[pos] = b.slot  # index copy of the parent's list + own slot (section 2.4)
+        self.next_uid += 1
+        self.branches[b.uid] = b
+        self.stats.branches_created += 1
+        return b
+
+    def slots_of(self, b: Branch) -> List[int]:
+        L = len(self.committed)
+        return [self.cslots[j] if j < L else b.chain[j] for j in range(b.pos + 1)]
+
+    def prefix_of(self, b: Branch) -> List[int]:
+        toks = {}
+        x = b
+        while x is not None:
+            toks[x.pos] = x.token
+            x = self.branches.get(x.parent)
+        L = len(self.committed)
+        return [self.committed[j] if j < L else toks[j] for j in range(b.pos + 1)]
+
+    def root(self) -> Branch:
+        L = len(self.committed)
+        roots = [b for b in self.branches.values() if b.pos == L - 1]
+        assert len(roots) == 1
+        return roots[0]
+
+    # -- one batched step ----------------------------------------------------------
+    def step(self) -> None:
+        st = self.stats
+        st.steps += 1
+        order = sorted(self.branches)
+        rows = self.rows
+        # 1. prelude for branches at depth 0
+        for u in order:
+            b = self.branches[u]
+            if b.depth == 0:
+                b.state = rows.prelude(self.prefix_of(b), b.pos, self.slots_of(b))
+        # 2. one loop iteration for every branch
+        for u in order:
+            b = self.branches[u]
+            b.state = rows.iterate(b.state, b.depth + 1, self.prefix_of(b), b.pos, self.slots_of(b))
+            b.depth += 1
+        st.rows_sum += len(order)
+        st.rows_max = max(st.rows_max, len(order))
+        if self.keep_trace:
+            self.trace.append([(u, self.branches[u].slot, self.branches[u].pos,
+                                self.branches[u].depth) for u in order])
+        # 3. readouts
+        for u in order:
+            b = self.branches[u]
+            b.p = None
+            if b.depth in self.tags:
+                z = rows.readout(b.state, b.depth, self.prefix_of(b), b.pos, self.slots_of(b))
+                if self.keep_logits:
+                    self.logits[(b.pos, b.depth)] = z
+                b.p = S.process(z, self.T, self.top_p)
+        # 4. proposals
+        for u in order:
+            b = self.branches[u]
+            spawn = b.pos + 1 < self.pos_limit  # is a child at pos+1 still needed?
+            if b.depth == self.d1:
+                b.q1 = b.p
+                b.x1 = S.race(b.q1, self.seed, b.uid, S.PROP1)
+                if spawn:
+                    b.child1 = self._new_branch(b.uid, b.pos + 1, b.x1, b.chain).uid
+            elif self.d2 and b.depth == self.d2 and b.x1 >= 0:
+                st.gate_checks += 1
+                if self.second == "gated":
+                    b.gate = S.gate_open(b.p, b.q1, b.x1)
+                    q2 = S.residual(b.p, b.q1) if b.gate else None
+                elif self.second == "ungated":
+                    q2 = S.residual(b.p, b.q1)
+                else:
+                    q2 = S.masked_second(b.p, b.x1)
+                b.gate = q2 is not None
+                if b.gate:
+                    st.gate_opens += 1
+                    b.q2 = q2
+                    b.x2 = S.race(q2, self.seed, b.uid, S.PROP2)
+                    if spawn:
+                        b.child2 = self._new_branch(b.uid, b.pos + 1, b.x2, b.chain).uid
+        # 5. verify at full depth
+        root = self.root()
+        if root.depth < self.R:
+            return
+        x, src, fb = S.verify(root.p, root.x1, root.q1, root.gate, root.x2, root.q2,
+                              self.seed, root.uid)
+        st.resid_fallback += fb
+        self.committed.append(x)
+        self.src.append(src)
+        self.cstep.append(st.steps)
+        if src == S.SRC_FIRST:
+            st.n_first += 1
+        elif src == S.SRC_SECOND:
+            st.n_second += 1
+        else:
+            st.n_fallback += 1
+        # 6. prune / reroot
+        keep_uid = root.child1 if src == S.SRC_FIRST else root.child2 if src == S.SRC_SECOND else -1
+        keep = set()
+        if keep_uid >= 0:
+            for u in sorted(self.branches):
+                x_ = self.branches[u]
+                while x_ is not None and x_.uid != keep_uid:
+                    x_ = self.branches.get(x_.parent)
+                if x_ is not None:
+                    keep.add(u)
+        for u in sorted(self.branches):
+            if u in keep:
+                continue
+            b = self.branches.pop(u)
+            if u != root.uid:  # the root's slot holds a committed position
+                self.free.add(b.slot)
+        if keep_uid >= 0:
+            self.branches[keep_uid].parent = -1
+            self.cslots.append(self.branches[keep_uid].slot)
+        elif not self.done():
+            L = len(self.committed)
+            nr = self._new_branch(-1, L - 1, x, {})
+            self.cslots.append(nr.slot)
+
+    def done(self) -> bool:
+        return len(self.committed) >= self.P + 1 + self.max_new
+
+    def run(self) -> DecodeResult:
+        while not self.done():
+            self.step()
+        return DecodeResult(self.committed[self.P:], self.src, self.cstep, self.cslots,
+                            self.stats, self.trace, self.logits)
+
+
+def decode_spec(rows, prompt, R, d1, d2, max_new, temperature, top_p, seed, n_slots,
+                **kw) -> DecodeResult:
+    return SpecDecoder(rows, prompt, R, d1, d2, max_new, temperature, top_p, seed, n_slots,
+                       **kw).run()

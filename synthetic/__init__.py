@@ -1,0 +1,267 @@
+"""Seeded synthetic inputs for looped-Transformer decoding.
+
+This module is the ONE place that both the CPU oracle (``oracle/``) and the CUDA
+library (``looped_transformer_self_b200``) take their inputs from.  It holds
+model shapes, random-init weights, token prompts and decode settings, and
+nothing of the method's arithmetic (no norm, attention, readout or sampling).
+
+The model family follows Eq. 1 of "LoopSpec: Pipelined Self-Speculative
+Decoding for Looped Transformers" (page liuzhao09.github.io/papers/loopspec.html,
+section 2.1): a prelude P, one shared block B applied R times, a coda/readout C.
+The pages publish no checkpoints, so every model here is random-init with the
+shapes of the Ouro / Huginn(Raven) families the pages measure (section 3.1),
+and every prompt is synthetic (uniform or Zipf(1.1) token ids) standing in for
+the public task suites the pages evaluate on.
+
+Init recipe (a reading; the pages give none):
+  * linear weights ~ N(0, 1/fan_in), stored in the nn.Linear layout [out, in];
+  * embedding ~ N(0, 1);
+  * RMSNorm gains ~ 1 + 0.1 N(0, 1) (not all ones, so a dropped gain is visible);
+  * LM head ~ N(0, g^2 / d) with the per-config gain g = ``head_gain``;
+  * bf16 models: every value is rounded to bf16 (round-to-nearest-even) and the
+    oracle uses those rounded values.
+Each tensor has its own seed stream (seed, tensor index), so any tensor can be
+regenerated alone.
+"""
+from __future__ import annotations
+
+import dataclasses
+from typing import Dict, Iterator, List, Optional, Tuple
+
+import numpy as np
+
+# ----------------------------------------------------------------------------
+# configurations
+# ----------------------------------------------------------------------------
+
+
+@dataclasses.dataclass(frozen=True)
+class ModelConfig:
+    name: str
+    dtype: str  # "f32" or "bf16": storage/arithmetic type of weights and GEMM operands
+    d_model: int
+    n_heads: int
+    head_dim: int
+    ffn: int
+    vocab: int
+    n_prelude: int  # Transformer layers in P (0: P is the embedding only)
+    n_core: int  # layers of the shared block B
+    n_coda: int  # Transformer layers in C before the final norm + LM head
+    R: int  # full loop depth
+    rms_eps: float = 1e-6
+    rope_theta: float = 10000.0
+    resid_scale: float = 1.0  # s: scales both sublayer outputs of shared-block layers
+    head_gain: float = 3.0  # g: LM head ~ N(0, g^2/d)
+    seed: int = 0
+
+    def replace(self, **kw) -> "ModelConfig":
+        return dataclasses.replace(self, **kw)
+
+    @property
+    def n_layers_total(self) -> int:
+        return self.n_prelude + self.n_core + self.n_coda
+
+    def layer_names(self) -> List[str]:
+        return ([f"pre{i}" for i in range(self.n_prelude)]
+                + [f"core{i}" for i in range(self.n_core)]
+                + [f"coda{i}" for i in range(self.n_coda)])
+
+
+@dataclasses.dataclass(frozen=True)
+class DecodeConfig:
+    d1: int  # first proposal depth (0: no proposals = full-depth AR)
+    d2: int  # second proposal depth (0: single proposal)
+    temperature: float  # 0 = greedy
+    top_p: float
+    seed: int
+    max_new: int  # decode tokens after the first (prefill) token
+
+    def replace(self, **kw) -> "DecodeConfig":
+        return dataclasses.replace(self, **kw)
+
+
+# Residual scales below were tuned (bisection on s, GPU prefill readouts over the
+# config's own prompt) so that the early-vs-full top-1 agreement on the prompt
+# hits the stated target; the achieved value is re-measured and reported by the
+# benchmark on every run.
+MODELS: Dict[str, ModelConfig] = {
+    # Tiny looped LM, fp32: prelude 1, shared 2 layers x R=4, coda 1.
+    "tiny": ModelConfig("tiny", "f32", 128, 4, 32, 384, 512, 1, 2, 1, 4,
+                        resid_scale=1.0, head_gain=3.0),
+    # The same model with a 16-token vocabulary (distribution tests).
+    "tiny16": ModelConfig("tiny16", "f32", 128, 4, 32, 384, 16, 1, 2, 1, 4,
+                          resid_scale=1.0, head_gain=1.5),
+    # Ouro-1.4B-shaped: P = embedding, B = 24 layers x R=4, C = norm + head.
+    "ouro14": ModelConfig("ouro14", "bf16", 2048, 16, 128, 5632, 49152, 0, 24, 0, 4,
+                          resid_scale=0.35, head_gain=3.5),
+    # Huginn/Raven-3.5B-shaped: prelude 2, core 4 x R=32, coda 2.
+    "huginn35": ModelConfig("huginn35", "bf16", 5280, 55, 96, 17920, 65536, 2, 4, 2, 32,
+                            resid_scale=0.12, head_gain=3.5),
+    # Ouro-2.6B-shaped: 48 shared layers x R=4.
+    "ouro26": ModelConfig("ouro26", "bf16", 2048, 16, 128, 5632, 49152, 0, 48, 0, 4,
+                          resid_scale=0.25, head_gain=3.5),
+    # Kernel sweep: one Ouro-shaped 24-layer shared block (no readout).
+    "sweep": ModelConfig("sweep", "bf16", 2048, 16, 128, 5632, 49152, 0, 24, 0, 4,
+                         resid_scale=0.35, head_gain=3.5),
+}
+
+DECODES: Dict[str, DecodeConfig] = {
+    "tiny_greedy": DecodeConfig(2, 3, 0.0, 1.0, 2, 64),
+    "tiny_sample": DecodeConfig(2, 3, 1.0, 0.9, 2, 64),
+    "ouro14_greedy": DecodeConfig(1, 2, 0.0, 1.0, 2, 1024),
+    "ouro14_sample": DecodeConfig(1, 2, 1.0, 0.95, 2, 1024),
+    "huginn35_greedy": DecodeConfig(8, 16, 0.0, 1.0, 2, 512),
+    "ouro26_greedy": DecodeConfig(1, 2, 0.0, 1.0, 2, 2048),
+}
+
+PROMPT_LEN = {"tiny": 32, "tiny16": 32, "ouro14": 512, "huginn35": 256, "ouro26": 4096}
+AGREEMENT_TARGET = {"ouro14": (1, 0.6), "huginn35": (8, 0.7), "ouro26": (1, 0.6)}
+
+
+# ----------------------------------------------------------------------------
+# bf16 rounding (storage format of the bf16 configs)
+# ----------------------------------------------------------------------------
+
+
+def round_to_bf16(x: np.ndarray) -> np.ndarray:
+    """fp32 values rounded to the nearest bf16 (ties to even), returned as fp32."""
+    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
+    r = (u + np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1))) & np.uint32(0xFFFF0000)
+    return r.view(np.float32)
+
+
+def bf16_bits(x: np.ndarray) -> np.ndarray:
+    """Upper 16 bits of fp32 values that are already bf16-representable."""
+    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
+    return (u >> np.uint32(16)).astype(np.uint16)
+
+
+# ----------------------------------------------------------------------------
+# weights
+# ----------------------------------------------------------------------------
+
+LAYER_TENSORS = ("g1", "wqkv", "wo", "g2", "wgu", "wd")
+
+
+def tensor_specs(cfg: ModelConfig) -> List[Tuple[str, Tuple[int, ...], str, float]]:
+    """(name, shape, kind, std) for every tensor, in a fixed order.
+
+    Layouts (row-major, nn.Linear [out, in]):
+      wqkv [3d, d]: rows 0..d-1 = Wq, d..2d-1 = Wk, 2d..3d-1 = Wv; head h owns
+                    rows h*hd..(h+1)*hd-1 of each of Wq/Wk/Wv.
+      wo   [d, d]
+      wgu  [2f, d]: rows 0..f-1 = gate (SiLU input), f..2f-1 = up.
+      wd   [d, f]
+    """
+    d, f, V = cfg.d_model, cfg.ffn, cfg.vocab
+    specs = [("embed", (V, d), "normal", 1.0)]
+    for ln in cfg.layer_names():
+        specs += [
+            (f"{ln}.g1", (d,), "gain", 0.1),
+            (f"{ln}.wqkv", (3 * d, d), "normal", 1.0 / np.sqrt(d)),
+            (f"{ln}.wo", (d, d), "normal", 1.0 / np.sqrt(d)),
+            (f"{ln}.g2", (d,), "gain", 0.1),
+            (f"{ln}.wgu", (2 * f, d), "normal", 1.0 / np.sqrt(d)),
+            (f"{ln}.wd", (d, f), "normal", 1.0 / np.sqrt(f)),
+        ]
+    specs += [("final_norm", (d,), "gain", 0.1),
+              ("head", (V, d), "normal", cfg.head_gain / np.sqrt(d))]
+    return specs
+
+
+def make_tensor(cfg: ModelConfig, index: int) -> Tuple[str, np.ndarray]:
+    name, shape, kind, std = tensor_specs(cfg)[index]
+    rng = np.random.Generator(np.random.PCG64(np.random.SeedSequence([cfg.seed, index])))
+    x = rng.standard_normal(size=shape, dtype=np.float32)
+    if kind == "gain":
+        x = np.float32(1.0) + np.float32(std) * x
+    else:
+        x *= np.float32(std)
+    if cfg.dtype == "bf16":
+        x = round_to_bf16(x)
+    return name, x
+
+
+def iter_weights(cfg: ModelConfig) -> Iterator[Tuple[str, np.ndarray]]:
+    for i in range(len(tensor_specs(cfg))):
+        yield make_tensor(cfg, i)
+
+
+def make_weights(cfg: ModelConfig) -> Dict[str, np.ndarray]:
+    return dict(iter_weights(cfg))
+
+
+# ----------------------------------------------------------------------------
+# prompts and row sets
+# ----------------------------------------------------------------------------
+
+
+def _zipf_probs(V: int, a: float = 1.1) -> np.ndarray:
+    k = np.arange(1, V + 1, dtype=np.float64)
+    w = k ** (-a)
+    return w / w.sum()
+
+
+def uniform_prompt(n: int, vocab: int, seed: int = 1) -> np.ndarray:
+    rng = np.random.default_rng(seed)
+    return rng.integers(0, vocab, size=n).astype(np.int32)
+
+
+def zipf_prompt(n: int, vocab: int, seed: int = 1, a: float = 1.1) -> np.ndarray:
+    """Ids with P(id = k-1) proportional to k^-a, k = 1..vocab."""
+    rng = np.random.default_rng(seed)
+    return rng.choice(vocab, size=n, p=_zipf_probs(vocab, a)).astype(np.int32)
+
+
+def copy_prompt(n: int, vocab: int, seed: int = 1, copy_frac: float = 0.4,
+                span: Tuple[int, int] = (16, 64)) -> Tuple[np.ndarray, float]:
+    """Fresh Zipf(1.1) tokens interleaved with copies of earlier spans.
+
+    Spans of length U{16..64} are copied from a uniform earlier start while the
+    copied fraction is below ``copy_frac``.  Returns (ids, achieved fraction).
+    """
+    rng = np.random.default_rng(seed)
+    p = _zipf_probs(vocab)
+    out: List[int] = []
+    copied = 0
+    while len(out) < n:
+        if len(out) >= span[1] and copied < copy_frac * max(len(out), 1) and rng.random() < 0.5:
+            L = int(rng.integers(span[0], span[1] + 1))
+            L = min(L, n - len(out))
+            s = int(rng.integers(0, len(out) - L + 1))
+            out.extend(out[s:s + L])
+            copied += L
+        else:
+            out.append(int(rng.choice(vocab, p=p)))
+    return np.asarray(out[:n], dtype=np.int32), copied / n
+
+
+def prompt_for(model: str, n: Optional[int] = None, seed: int = 1) -> np.ndarray:
+    cfg = MODELS[model]
+    n = PROMPT_LEN[model] if n is None else n
+    if model in ("tiny", "tiny16"):
+        return uniform_prompt(n, cfg.vocab, seed)
+    if model == "ouro26":
+        return copy_prompt(n, cfg.vocab, seed)[0]
+    return zipf_prompt(n, cfg.vocab, seed)
+
+
+def sweep_rows(M: int, R: int = 4, seed: int = 3, lmin: int = 256,
+               lmax: int = 8192) -> Tuple[np.ndarray, np.ndarray]:
+    """Kernel-sweep rows: depth ~ U{1..R}, attended length ~ U{lmin..lmax}."""
+    rng = np.random.default_rng(seed)
+    depth = rng.integers(1, R + 1, size=M).astype(np.int32)
+    lens = rng.integers(lmin, lmax + 1, size=M).astype(np.int32)
+    return depth, lens
+
+
+def random_hidden(M: int, d: int, seed: int) -> np.ndarray:
+    rng = np.random.default_rng(seed)
+    return rng.standard_normal(size=(M, d), dtype=np.float32)
+
+
+def random_kv(n: int, d: int, seed: int, dtype: str = "bf16") -> np.ndarray:
+    """N(0,1) cache rows, rounded to the storage type."""
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal(size=(n, d), dtype=np.float32)
+    return round_to_bf16(x) if dtype == "bf16" else x
