@@ -1,0 +1,427 @@
+// tcgen05 / TMEM / TMA weight-streaming GEMM (see gemm.cuh for the design).
+#include <stdio.h>
+
+#include <algorithm>
+
+#include "gemm.cuh"
+
+namespace lt {
+
+// ---------------------------------------------------------------------------
+// PTX wrappers
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+constexpr long long WAIT_LIMIT_CYCLES = 2000000000LL;  // ~1 s at 1.9 GHz
+
+// Bounded wait on an mbarrier phase; false when it gave up (or another role did).
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (*abort_flag) return false;
+    if (clock64() - t0 > WAIT_LIMIT_CYCLES) {
+      *abort_flag = 1;
+      return false;
+    }
+  }
+  return true;
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                            uint32_t bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      ".L2::cache_hint [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar), "l"(policy)
+      : "memory");
+}
+__device__ __forceinline__ uint64_t policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ uint64_t policy_evict_last() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   bar)
+               : "memory");
+}
+template <bool TF32>
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                       uint32_t idesc, uint32_t accumulate) {
+  if constexpr (TF32) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+  } else {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+  }
+}
+// 32 lanes x 32 bits, 8 consecutive columns.
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7])
+      : "r"(taddr)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_ld() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, 8-row
+// atoms of 1024 bytes (stride byte offset 1024), sm100 descriptor version 1.
+__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr) {
+  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) |
+         ((uint64_t)(1024 >> 4) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+// Instruction descriptor: D fp32, A/B bf16 (kind::f16) or tf32 (kind::tf32),
+// both K-major, N = ncols, M = 128.
+template <bool TF32, int NC>
+__device__ __forceinline__ constexpr uint32_t instr_desc() {
+  return (1u << 4) | ((TF32 ? 2u : 1u) << 7) | ((TF32 ? 2u : 1u) << 10) |
+         ((uint32_t)(NC >> 3) << 17) | ((uint32_t)(GEMM_BM >> 4) << 24);
+}
+
+template <int NC>
+constexpr int tmem_cols() {
+  return (2 * NC) <= 32 ? 32 : (2 * NC) <= 64 ? 64 : (2 * NC) <= 128 ? 128 : 256;
+}
+
+// ---------------------------------------------------------------------------
+// kernel
+// ---------------------------------------------------------------------------
+template <bool TF32, int NC>
+__global__ void __launch_bounds__(GEMM_THREADS, 1)
+    k_gemm(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
+           float* __restrict__ part, const GemmShape s, const int stages,
+           const int* __restrict__ run_flag, int* __restrict__ err) {
+  constexpr uint32_t A_BYTES = GEMM_BM * GEMM_CHUNK_BYTES;
+  constexpr uint32_t B_BYTES = NC * GEMM_CHUNK_BYTES;
+  constexpr int BKE = TF32 ? 32 : 64;  // elements per k-chunk
+  constexpr int TCOLS = tmem_cols<NC>();
+  constexpr uint32_t IDESC = instr_desc<TF32, NC>();
+
+  pdl_wait();
+  if (run_flag != nullptr && *run_flag == 0) return;
+  const int c = blockIdx.x;
+  const int u0 = sk_u0(c, s.units, s.grid), u1 = sk_u0(c + 1, s.units, s.grid);
+  if (u0 >= u1) return;
+
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (base - raw);
+  const uint32_t a_base = base;
+  const uint32_t b_base = base + stages * A_BYTES;
+  const uint32_t bar_base = b_base + stages * B_BYTES;  // 8-byte aligned
+  // barriers: full[stages], empty[stages], accf[2], acce[2], drain
+  auto full_bar = [&](int i) { return bar_base + 8u * i; };
+  auto empty_bar = [&](int i) { return bar_base + 8u * (stages + i); };
+  auto accf_bar = [&](int i) { return bar_base + 8u * (2 * stages + i); };
+  auto acce_bar = [&](int i) { return bar_base + 8u * (2 * stages + 2 + i); };
+  const uint32_t drain_bar = bar_base + 8u * (2 * stages + 4);
+  uint8_t* misc = gbase + (bar_base - base) + 8u * (2 * stages + 5);
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(misc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < stages; ++i) {
+      mbar_init(full_bar(i), 1);
+      mbar_init(empty_bar(i), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(accf_bar(i), 1);
+      mbar_init(acce_bar(i), 128);
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmW)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmX)) : "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32((const void*)tmem_slot)),
+                 "r"(TCOLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer ----------------
+      const uint64_t pol_w = policy_evict_first(), pol_x = policy_evict_last();
+      int g = 0;
+      for (int u = u0; u < u1 && !*abort_flag;) {
+        const int t = u / s.kch;
+        const int seg_end = min(u1, (t + 1) * s.kch);
+        for (int uu = u; uu < seg_end; ++uu, ++g) {
+          const int st = g % stages, n = g / stages;
+          if (!mbar_wait(empty_bar(st), (n & 1) ^ 1, abort_flag)) break;
+          mbar_expect_tx(full_bar(st), A_BYTES + B_BYTES);
+          const int kx = (uu - t * s.kch) * BKE;
+          tma_load_2d(a_base + st * A_BYTES, &tmW, kx, t * GEMM_BM, full_bar(st), pol_w);
+          tma_load_2d(b_base + st * B_BYTES, &tmX, kx, 0, full_bar(st), pol_x);
+        }
+        u = seg_end;
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------- MMA issuer ----------------
+      int g = 0, seg = 0;
+      bool ok = true;
+      for (int u = u0; u < u1 && ok; ++seg) {
+        const int t = u / s.kch;
+        const int seg_end = min(u1, (t + 1) * s.kch);
+        const int b = seg & 1, use = seg >> 1;
+        if (!mbar_wait(acce_bar(b), (use & 1) ^ 1, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem + (uint32_t)(b * NC);
+        for (int uu = u; uu < seg_end; ++uu, ++g) {
+          const int st = g % stages, n = g / stages;
+          if (!mbar_wait(full_bar(st), n & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = a_base + st * A_BYTES, b0 = b_base + st * B_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < GEMM_CHUNK_BYTES / 32; ++kk) {
+            tc_mma<TF32>(d_tmem, smem_desc(a0 + 32u * kk), smem_desc(b0 + 32u * kk), IDESC,
+                         (uu > u || kk > 0) ? 1u : 0u);
+          }
+          tc_commit(empty_bar(st));
+        }
+        if (!ok) break;
+        tc_commit(accf_bar(b));
+        u = seg_end;
+      }
+      // let every issued MMA finish before TMEM can be released
+      tc_commit(drain_bar);
+      volatile int dummy = 0;
+      mbar_wait(drain_bar, 0, &dummy);
+    }
+  } else {
+    // ---------------- drain: TMEM -> fp32 partials ----------------
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    int seg = 0;
+    for (int u = u0; u < u1; ++seg) {
+      const int t = u / s.kch;
+      const int seg_end = min(u1, (t + 1) * s.kch);
+      const int b = seg & 1, use = seg >> 1;
+      if (!mbar_wait(accf_bar(b), use & 1, abort_flag)) break;
+      tc_fence_after();
+      uint32_t r[NC];
+      const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * NC);
+#pragma unroll
+      for (int j = 0; j < NC / 8; ++j) tmem_ld8(taddr + 8u * j, r + 8 * j);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(acce_bar(b));
+      float* dst = part + ((size_t)(c * s.jmax + seg) * NC) * GEMM_BM + q * 32 + lane;
+#pragma unroll
+      for (int i = 0; i < NC; ++i) dst[(size_t)i * GEMM_BM] = __uint_as_float(r[i]);
+      u = seg_end;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (*abort_flag) {
+    if (threadIdx.x == 0) {
+      set_err(err, DEV_TIMEOUT);
+      // give copies still in flight time to land before the CTA's smem is reused
+      const long long t0 = clock64();
+      while (clock64() - t0 < 4000000LL) {
+      }
+    }
+    __syncthreads();
+  }
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TCOLS)
+                 : "memory");
+  }
+  pdl_trigger();
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+static int stages_for(int ncols) {
+  const int stage = GEMM_BM * GEMM_CHUNK_BYTES + ncols * GEMM_CHUNK_BYTES;
+  int st = (GEMM_SMEM_BUDGET - 1024 - 256) / stage;
+  return std::min(st, 16);
+}
+static size_t smem_bytes(int ncols, int stages) {
+  return 1024 + (size_t)stages * (GEMM_BM + ncols) * GEMM_CHUNK_BYTES + 8 * (2 * stages + 5) + 16;
+}
+
+int gemm_table_ints(int n_out, int k, bool f32, int grid_cap) {
+  GemmShape s;
+  gemm_plan(n_out, k, f32, grid_cap, &s, nullptr, nullptr);
+  return 2 * s.tiles + s.grid;
+}
+
+void gemm_plan(int n_out, int k, bool f32, int grid_cap, GemmShape* s, int* tile_c,
+               int* cta_t0) {
+  const int bke = f32 ? 32 : 64;
+  s->n_out = n_out;
+  s->k = k;
+  s->kch = (k + bke - 1) / bke;
+  s->tiles = (n_out + GEMM_BM - 1) / GEMM_BM;
+  s->units = s->tiles * s->kch;
+  s->grid = std::min(grid_cap, s->units);
+  int jmax = 1;
+  for (int c = 0; c < s->grid; ++c) {
+    const int u0 = sk_u0(c, s->units, s->grid), u1 = sk_u0(c + 1, s->units, s->grid);
+    if (u1 > u0) jmax = std::max(jmax, (u1 - 1) / s->kch - u0 / s->kch + 1);
+    if (cta_t0) cta_t0[c] = u0 / s->kch;
+  }
+  s->jmax = jmax;
+  if (tile_c) {
+    for (int t = 0; t < s->tiles; ++t) {
+      tile_c[2 * t] = sk_cta_of(t * s->kch, s->units, s->grid);
+      tile_c[2 * t + 1] = sk_cta_of(t * s->kch + s->kch - 1, s->units, s->grid);
+    }
+  }
+  s->tile_c = nullptr;
+  s->cta_t0 = nullptr;
+}
+
+size_t gemm_part_bytes(const GemmShape& s, int ncols) {
+  return (size_t)s.grid * s.jmax * ncols * GEMM_BM * sizeof(float);
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn get_encode() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (EncodeTiledFn)p;
+  }
+  return fn;
+}
+
+int make_tmap(CUtensorMap* map, const void* base, bool f32, uint64_t rows, uint64_t k,
+              uint32_t box_rows) {
+  EncodeTiledFn enc = get_encode();
+  if (!enc) return -1;
+  const uint32_t esz = f32 ? 4 : 2;
+  if (((uintptr_t)base & 15) || ((k * esz) & 15) || box_rows == 0 || box_rows > 256) return -2;
+  cuuint64_t dims[2] = {k, rows};
+  cuuint64_t strides[1] = {k * esz};
+  cuuint32_t box[2] = {GEMM_CHUNK_BYTES / esz, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                   const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? 0 : -3;
+}
+
+template <bool TF32, int NC>
+static cudaError_t launch_t(const CUtensorMap& tmW, const CUtensorMap& tmX, float* part,
+                            const GemmShape& s, const int* run_flag, int* err,
+                            cudaStream_t stream, bool pdl) {
+  const int stages = stages_for(NC);
+  const size_t smem = smem_bytes(NC, stages);
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(k_gemm<TF32, NC>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(s.grid);
+  cfg.blockDim = dim3(GEMM_THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, k_gemm<TF32, NC>, tmW, tmX, part, s, stages, run_flag, err);
+}
+
+cudaError_t gemm_launch(const CUtensorMap& tmW, const CUtensorMap& tmX, float* part,
+                        const GemmShape& s, int ncols, bool f32, const int* run_flag, int* err,
+                        cudaStream_t stream, bool pdl) {
+#define LT_GEMM_CASE(N)                                                                    \
+  case N:                                                                                  \
+    return f32 ? launch_t<true, N>(tmW, tmX, part, s, run_flag, err, stream, pdl)           \
+               : launch_t<false, N>(tmW, tmX, part, s, run_flag, err, stream, pdl);
+  switch (ncols) {
+    LT_GEMM_CASE(8)
+    LT_GEMM_CASE(16)
+    LT_GEMM_CASE(32)
+    LT_GEMM_CASE(64)
+    default:
+      return cudaErrorInvalidValue;
+  }
+#undef LT_GEMM_CASE
+}
+
+}  // namespace lt

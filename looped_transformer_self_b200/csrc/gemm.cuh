@@ -1,0 +1,58 @@
+// Weight-streaming GEMM for few rows on sm_100a tensor cores (tcgen05 + TMEM + TMA).
+//
+// Computes partial sums of Y[i][n] = sum_k X[i][k] * W[n][k] for the <= 64
+// active rows i of a decode step and every output feature n of one weight
+// matrix W [n_out x K] (nn.Linear layout, K contiguous).  The shared block's
+// weights are read from HBM once per step however many rows ride along, which
+// is the point of batching every (branch, position, depth) row into one pass
+// ("LoopSpec", liuzhao09.github.io/papers/loopspec.html, sections 1 and 2.2:
+// the current position and the branches opened from shallow proposals call the
+// same shared block and are merged into one batched execution).
+//
+// Design (B200):
+//  * swap-AB: W is the MMA's A operand (M = 128 output features per tile), the
+//    rows are the B operand (N = ncols = table capacity, 8..64).  The MMA always
+//    runs all ncols columns, so a row's result never depends on how many other
+//    rows are active (batch invariance: the speculative and full-depth paths
+//    give bit-identical rows).
+//  * stream-K: the (tile, 128-byte k-chunk) units are split evenly over one CTA
+//    per SM; each CTA streams its contiguous unit range through a TMA ring of
+//    up to ~200 KB of shared memory, issues tcgen05.mma from one thread into
+//    double-buffered TMEM accumulators, and drains each finished tile segment
+//    (tcgen05.ld) as an fp32 partial.  The consumer kernel adds a tile's
+//    partials in CTA order (fixed order: deterministic).  The partition depends
+//    only on (n_out, K, #SMs), never on the active row count.
+//  * bf16 operands: kind::f16 with fp32 accumulate; fp32 operands: kind::tf32.
+//  * K tails and n_out tails are zero-filled by TMA.
+//  * every mbarrier wait is bounded (~1 s); on timeout the kernel records
+//    DEV_TIMEOUT, lets in-flight copies and MMAs land, frees TMEM and returns.
+#pragma once
+
+#include "common.cuh"
+
+namespace lt {
+
+constexpr int GEMM_BM = 128;            // output features per tile (MMA M)
+constexpr int GEMM_CHUNK_BYTES = 128;   // K bytes per stage (one 128B-swizzle row)
+constexpr int GEMM_THREADS = 192;       // warp 0: TMA, warp 1: MMA, warps 2-5: drain
+constexpr int GEMM_SMEM_BUDGET = 200 * 1024;
+
+// Plans the stream-K split of one weight matrix.  `grid_cap`: CTAs (#SMs).
+// Fills the host copies of the reducer tables (tile_c [2*tiles], cta_t0 [grid]).
+void gemm_plan(int n_out, int k, bool f32, int grid_cap, GemmShape* s, int* tile_c_host,
+               int* cta_t0_host);
+int gemm_table_ints(int n_out, int k, bool f32, int grid_cap);  // 2*tiles + grid
+
+// Encodes a K-major 2-D tensor map (rows x k, box box_rows x 128 bytes, 128B swizzle).
+int make_tmap(CUtensorMap* map, const void* base, bool f32, uint64_t rows, uint64_t k,
+              uint32_t box_rows);
+
+// Launches the GEMM.  ncols in {8, 16, 32, 64}.  run_flag (device, may be null):
+// skip when *run_flag == 0.  pdl: launch with programmatic stream serialization.
+cudaError_t gemm_launch(const CUtensorMap& tmW, const CUtensorMap& tmX, float* part,
+                        const GemmShape& s, int ncols, bool f32, const int* run_flag,
+                        int* err, cudaStream_t stream, bool pdl);
+
+size_t gemm_part_bytes(const GemmShape& s, int ncols);
+
+}  // namespace lt
