@@ -1,0 +1,332 @@
+"""Decode benchmark: pipelined self-speculative decoding of a looped LM on B200.
+
+Workload (the pages' single-request decode setting, LoopSpec page section 3.1):
+an Ouro-1.4B-shaped looped LM (bf16, random init with the residual scale tuned
+for depth-1 vs depth-4 top-1 agreement ~0.6; shared stack 24 layers x R = 4,
+d 2048, 16 x 128 heads, SwiGLU 5632, vocab 49152), a 512-token Zipf(1.1)
+prompt, 1024 decoded tokens, proposal readouts at depths 1 and 2.
+
+One bench step = prefill (untimed: the pages time the decode phase only) +
+one greedy pipelined speculative decode of 1024 tokens through the C ABI,
+timed with CUDA events on the decoder's stream.  value = decoded tokens / s
+summed over ranks (replicas: one independent request per GPU, no collective
+on the data path).  The weights (2.47 GB per shared-block pass) exceed the
+126 MB L2, so no flush is needed between steps.
+
+`--impl reference` times the CPU oracle (the plain fp64 implementation the
+GPU path is checked against) on the host cores on a bounded sample of the
+same workload.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+
+def _peaks():
+    try:
+        return json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+    except Exception:
+        return None
+
+
+class Clocks:
+    """nvidia-smi samples of SM clock and throttle reasons during a region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index, self.samples, self.stop = index, [], threading.Event()
+
+    def _run(self):
+        while not self.stop.is_set():
+            try:
+                out = subprocess.run(["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS,
+                                      "--format=csv,noheader,nounits"], capture_output=True,
+                                     text=True, timeout=5).stdout.strip()
+                if out:
+                    self.samples.append([x.strip() for x in out.split(",")])
+            except Exception:
+                pass
+            self.stop.wait(0.2)
+
+    def __enter__(self):
+        self.t = threading.Thread(target=self._run, daemon=True)
+        self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        self.stop.set()
+        self.t.join(timeout=10)
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(s[0]) for s in self.samples if s[0].replace(".", "").isdigit()]
+        mx = [float(s[1]) for s in self.samples if s[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[k] for s in self.samples for k in range(4)
+                          if len(s) > 4 + k and s[4 + k].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(self.samples)}
+
+
+def _dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    if ws <= 1:
+        return 0, 0, 1
+    import datetime
+    import torch.distributed as dist
+    rank, local = int(os.environ["RANK"]), int(os.environ.get("LOCAL_RANK", "0"))
+    backend = "nccl" if os.environ.get("BENCH_BACKEND", "nccl") == "nccl" else "gloo"
+    dist.init_process_group(backend, timeout=datetime.timedelta(seconds=600))
+    return rank, local, ws
+
+
+def _max_over_ranks(x, ws, device):
+    if ws <= 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def _barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle baseline (also the --impl reference arm)
+# ---------------------------------------------------------------------------
+
+def oracle_sample(cfg, dec, prompt, weights, n_prompt=8, n_tokens=4):
+    """Oracle decode tokens/s on a bounded sample: the first n_prompt prompt
+    tokens, then n_tokens greedy pipelined speculative decode tokens (decode
+    phase timed, like the metric)."""
+    from oracle import decode as D
+    from oracle.model import LoopedModel
+    t0 = time.perf_counter()
+    rows = D.OracleRows(LoopedModel(cfg, weights, n_prompt + n_tokens + 16))
+    sd = D.SpecDecoder(rows, list(prompt[:n_prompt]), cfg.R, dec.d1, dec.d2, n_tokens,
+                       dec.temperature, dec.top_p, dec.seed, n_prompt + n_tokens + 16,
+                       keep_trace=False)
+    t1 = time.perf_counter()
+    sd.run()
+    t2 = time.perf_counter()
+    return {"value": n_tokens / (t2 - t1), "unit": "tokens/s", "cores": os.cpu_count(),
+            "kind": "oracle",
+            "sample": f"{cfg.name}: prompt truncated to {n_prompt} tokens, {n_tokens} greedy "
+                      f"speculative decode tokens (d1={dec.d1}, d2={dec.d2}); prefill "
+                      f"{t1 - t0:.1f}s untimed, decode {t2 - t1:.1f}s timed, fp64 on "
+                      f"{os.cpu_count()} host threads"}
+
+
+def run_reference(args):
+    import synthetic as syn
+    rank, _, ws = int(os.environ.get("RANK", "0")), 0, int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return
+    cfg = syn.MODELS[args.model]
+    dec = syn.DECODES[f"{args.model}_greedy"]
+    prompt = syn.prompt_for(args.model)
+    w = syn.make_weights(cfg)
+    for _ in range(args.warmup if args.warmup < 1 else 0):
+        pass
+    vals, last = [], None
+    for _ in range(max(1, args.steps)):
+        last = oracle_sample(cfg, dec, prompt, w, n_tokens=2)
+        vals.append(last["value"])
+    v = sum(vals) / len(vals)
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 2000.0 / v, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "l2": "weights larger than L2"},
+            "cpu_baseline": dict(last, value=v),
+            "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+
+
+METRIC = "decoded tokens/s at batch 1 (greedy, T=1) + step HBM GB/s vs 8 TB/s"
+WORKLOAD = ("ouro14: Ouro-1.4B-shaped looped LM (bf16, 24 shared layers x R=4, d2048, 16x128, "
+            "ffn5632, V49152), 512-token Zipf(1.1) prompt, 1024 decode tokens, proposals at "
+            "depths 1 and 2, batch 1")
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+
+def run_ours(args):
+    import torch
+    import synthetic as syn
+    from looped_transformer_self_b200.binding import Decoder, lib, ProfileC, InfoC
+    import ctypes
+
+    rank, local, ws = _dist()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    cfg = syn.MODELS[args.model]
+    n_new = args.n_new
+    dec_g = syn.DECODES[f"{args.model}_greedy"].replace(max_new=n_new, seed=2 + rank)
+    prompt = syn.prompt_for(args.model, seed=1 + rank)
+    P = len(prompt)
+    t_w = time.time()
+    weights = syn.make_weights(cfg)
+    g = Decoder(cfg, dec_g, weights, max_branches=16, max_ctx=P + 1 + n_new + 8,
+                trace_steps=0, device=dev)
+    t_w = time.time() - t_w
+
+    # agreement of the depth-d1 readout with full depth over the prompt
+    _, am, _ = g.prefill(prompt, argmax=True)
+    tags = sorted({r for r in (dec_g.d1, dec_g.d2, cfg.R) if r > 0})
+    agree = float(np.mean(am[:, tags.index(dec_g.d1)] == am[:, tags.index(cfg.R)]))
+
+    def one_generate(ar=False):
+        g.prefill(prompt)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(g.stream)
+        toks, st = g.generate(n_new, ar=ar)
+        e1.record(g.stream)
+        e1.synchronize()
+        return e0.elapsed_time(e1), toks, st
+
+    for _ in range(args.warmup):
+        one_generate()
+    _barrier(ws)
+    torch.cuda.synchronize()
+    times, stats = [], None
+    with Clocks(local) as clk:
+        for _ in range(args.steps):
+            ms, toks, stats = one_generate()
+            times.append(ms)
+    torch.cuda.synchronize()
+    _barrier(ws)
+    total_ms = _max_over_ranks(sum(times), ws, dev)
+    value = ws * n_new * args.steps / (total_ms / 1000.0)
+
+    # full-depth AR baseline and sampled decoding (same kernels), one run each
+    ar_ms, ar_toks, ar_st = one_generate(ar=True)
+    spec_equal_ar = ar_toks == toks
+    g_s = Decoder(cfg, syn.DECODES[f"{args.model}_sample"].replace(max_new=n_new, seed=2 + rank),
+                  None, max_branches=16, max_ctx=P + 1 + n_new + 8, device=dev)
+    g_s.weights = g.weights
+    g_s.bind_weights()
+    g_s.prefill(prompt)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(g_s.stream)
+    _, st_s = g_s.generate(n_new)
+    e1.record(g_s.stream)
+    e1.synchronize()
+    sample_ms = e0.elapsed_time(e1)
+
+    # live roofline of the dominant kernel: CUDA events around every GEMM of
+    # 64 un-graphed decode steps (on the decoder's stream)
+    g.prefill(prompt)
+    prof = g.profile(64)
+    info = g.info()
+
+    # end to end through the public API: host prompt in, host tokens out
+    t0 = time.perf_counter()
+    first, _, _ = g.prefill(prompt)
+    toks_e2e, _ = g.generate(n_new)
+    torch.cuda.synchronize()
+    e2e_s = time.perf_counter() - t0
+
+    peaks = _peaks()
+    hbm = peaks["hbm_gbs"] if peaks else 6650.0
+    gemm_gbs = prof["gemm_core_bytes"] / (prof["gemm_core_ms"] / 1e3) / 1e9
+    step_bytes = prof["weight_bytes_core"] * prof["steps"] + prof["kv_bytes"]
+    step_gbs = step_bytes / (prof["step_ms"] / 1e3) / 1e9
+    traffic = None
+    tf = os.path.join(ROOT, "profiles", "gemm_traffic.json")
+    if os.path.exists(tf):
+        traffic = json.load(open(tf)).get("traffic_per_launch")
+
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu:
+        cpu = oracle_sample(cfg, dec_g, prompt, weights)
+
+    if rank == 0:
+        n_steps = stats["steps"]
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "parallelism": f"replicas x{ws}",
+                       "l2": "no flush: 2.47 GB of weights per pass exceed the 126 MB L2",
+                       "resid_scale": cfg.resid_scale, "agreement_d1_vs_R": agree,
+                       "max_branches": 16},
+            "speedup_vs_full_depth_ar": (ar_ms / times[-1]),
+            "ar_tokens_per_s": n_new / (ar_ms / 1e3),
+            "sampled_tokens_per_s": n_new / (sample_ms / 1e3),
+            "spec_greedy_equals_ar_greedy": bool(spec_equal_ar),
+            "gamma": _gamma(stats, dec_g.d1, dec_g.d2, cfg.R),
+            "gamma_sampled": _gamma(st_s, dec_g.d1, dec_g.d2, cfg.R),
+            "decode_stats": stats, "sampled_stats": st_s,
+            "step_hbm": {"gbs": step_gbs, "frac_of_measured_hbm": step_gbs / hbm,
+                         "bytes_per_step": step_bytes / max(prof["steps"], 1),
+                         "ms_per_step_profiled": prof["step_ms"] / max(prof["steps"], 1),
+                         "ms_per_step_graphed": times[-1] / n_steps},
+            "roofline": {"kernel": "k_gemm (tcgen05 weight-streaming GEMM)", "bound": "hbm",
+                         "achieved": gemm_gbs, "peak": hbm, "unit": "GB/s",
+                         "frac": gemm_gbs / hbm, "traffic": traffic,
+                         "peak_source": "measured" if peaks else "fallback",
+                         "launches_profiled": prof["gemm_core_launches"]},
+            "cpu_baseline": cpu,
+            "e2e": {"value": n_new / e2e_s, "unit": "tokens/s",
+                    "h2d_bytes_per_step": 4 * P, "d2h_bytes_per_step": 4 * (n_new + 1),
+                    "includes": "lt_prefill + lt_generate wall time, host buffers"},
+            "gpu_launches": info["kernels_per_step"] * n_steps * args.steps,
+            "clocks": clk.summary(),
+            "profile": prof,
+            "weights_gen_s": t_w,
+        }
+        print(json.dumps(line))
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def _gamma(st, d1, d2, R):
+    den = st["n_first"] * d1 + st["n_second"] * d2 + st["n_fallback"] * R
+    n = st["n_first"] + st["n_second"] + st["n_fallback"]
+    return n * R / den if den else None
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--model", default="ouro14")
+    ap.add_argument("--n-new", type=int, default=1024)
+    ap.add_argument("--no-cpu", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -43,6 +43,146 @@ enum {
   LT_ERR_STATE = -6         /* call out of order (e.g. decode before prefill) */
 };
 
+/* Model shape (section 2.1, Eq. 1; section 3.1 for the Ouro / Raven families).
+ * The layer reading: pre-norm RMSNorm (rms_eps), QKV, RoPE (rope_theta,
+ * rotate-half, absolute positions), causal softmax attention, O projection,
+ * RMSNorm, SwiGLU MLP; resid_scale s multiplies both sublayer outputs of the
+ * shared-block layers (prelude and coda layers use 1). */
+typedef struct {
+  int dtype;      /* LT_F32 (tf32 tensor-core operands) or LT_BF16 */
+  int d_model, n_heads, head_dim, ffn, vocab;
+  int n_prelude;  /* Transformer layers of P (0: P is the embedding) */
+  int n_core;     /* layers of the shared block B */
+  int n_coda;     /* Transformer layers of C before the final norm + LM head */
+  int R;          /* full loop depth, 1..32 */
+  float rms_eps, rope_theta, resid_scale;
+} lt_model_config;
+
+/* Decoding settings (sections 2.2-2.3). */
+typedef struct {
+  int d1;              /* first proposal depth, 1 <= d1 < R (0: full-depth AR only) */
+  int d2;              /* second proposal depth, d1 < d2 < R, or 0 (single proposal) */
+  float temperature;   /* 0 = greedy */
+  float top_p;         /* (0, 1]; applied at every readout depth */
+  uint64_t seed;       /* Philox-4x32-10 key */
+  int max_branches;    /* branch-table capacity = GEMM columns: 8, 16, 32 or 64 */
+  int max_ctx;         /* max committed length (prompt + 1 + generated) */
+  int max_new;         /* default token budget of lt_decode_step */
+  int second_mode;     /* 0: gated residual (the method); 1: residual, no gate;
+                          2: p_d2 with x1 masked, no gate (ablations, section 3.4) */
+  int trace_steps;     /* steps whose branch rows are logged (0: none) */
+} lt_decode_config;
+
+/* Per-generate statistics (section 3.2 Eq. 9 counts, Fig. 5, Table 6, Fig. 6). */
+typedef struct {
+  int steps;            /* batched shared-block passes */
+  int rows_sum, rows_max;  /* active branches per pass: sum and peak */
+  int n_first, n_second, n_fallback;  /* commit sources */
+  int gate_checks, gate_opens;
+  int branches_created;
+  int resid_fallback;   /* residuals with zero mass (expected 0) */
+  int committed_len;    /* committed length after the call */
+} lt_stats;
+
+typedef struct lt_handle lt_handle;
+
+/*
+ * Workspace: every device buffer of a handle (branch table, row arrays, KV
+ * pool [planes][slots][K|V][d_model], activations, GEMM partials, readout
+ * vectors, RoPE table).  Caller allocates >= lt_workspace_bytes() bytes of
+ * device memory and keeps it alive until lt_destroy.  Errors: LT_ERR_SHAPE
+ * for unsupported sizes (head_dim not in {32,64,96,128}, max_branches not in
+ * {8,16,32,64}, R > 32, rows not 16-byte multiples, ...).
+ */
+int lt_workspace_bytes(const lt_model_config* m, const lt_decode_config* dc, size_t* bytes);
+/* Creates a handle on `stream` (a cudaStream_t, not the legacy default stream:
+ * decode steps are captured in a CUDA graph). */
+int lt_create(const lt_model_config* m, const lt_decode_config* dc, void* d_workspace,
+              size_t bytes, void* stream, lt_handle** out);
+/*
+ * Weights (device, caller-owned, dtype of the model, row-major nn.Linear
+ * layout [out][in], 16-byte aligned): embedding [vocab][d], final norm [d],
+ * LM head [vocab][d]; d_layers holds 6 pointers per layer in the order
+ * prelude layers, shared-block layers, coda layers:
+ *   g1 [d], wqkv [3d][d] (q rows, then k, then v), wo [d][d], g2 [d],
+ *   wgu [2 ffn][d] (gate rows, then up rows), wd [d][ffn].
+ */
+int lt_load_weights(lt_handle* h, const void* d_embed, const void* d_final_norm,
+                    const void* d_head, const void* const* d_layers);
+/*
+ * Prefill (section 2.2): the prompt runs through P and all R depths of B,
+ * filling the per-depth caches, and through C at every readout depth
+ * {d1, d2, R} (coda caches); the first token is committed from the full-depth
+ * readout of the last position (drawn with the stream (n, AR)).  Resets the
+ * decoding state.  h_first: the committed token.  Optional: h_argmax
+ * [n][n_tags] argmax of every readout; d_logits [n][n_tags][vocab] (device)
+ * logits of every readout; n_tags = |{d1, d2, R} minus 0|, ascending depth.
+ */
+int lt_prefill(lt_handle* h, const int32_t* h_tokens, int n, int32_t* h_first,
+               int32_t* h_argmax, float* d_logits);
+/*
+ * Decode n tokens from the current state.  ar_mode 0: pipelined speculative
+ * decoding (sections 2.2-2.3: proposals at d1 / d2, gate, cascade verify at R,
+ * prune / re-root, all on the device); ar_mode 1: full-depth autoregressive
+ * decoding with the same kernels (the comparison baseline; section 3.1).
+ * h_out: the n committed tokens.  st: statistics of this call (may be NULL).
+ * Greedy speculative output equals greedy AR output bit for bit.
+ */
+int lt_generate(lt_handle* h, int ar_mode, int n, int32_t* h_out, lt_stats* st);
+/* One batched pass.  *n_committed = 1 and *h_tok = the token when this pass
+ * committed one, else 0. */
+int lt_decode_step(lt_handle* h, int ar_mode, int32_t* h_tok, int* n_committed);
+/* Commit log of the last generate / decode calls: token, source (1 first
+ * proposal, 2 second, 0 drawn at full depth) and 1-based step of each commit. */
+int lt_read_log(lt_handle* h, int32_t* h_tok, int32_t* h_src, int32_t* h_step, int n);
+/* Branch rows logged per step, [n_steps][max_branches][4] = (uid, slot, pos,
+ * depth) sorted by uid, unused entries -1. */
+int lt_read_trace(lt_handle* h, int32_t* h_trace, int n_steps);
+/* Committed tokens and their KV slots (arrays of max_ctx ints). */
+int lt_read_committed(lt_handle* h, int32_t* h_tokens, int32_t* h_slots, int* h_len);
+/* Branch table, [12][max_branches]: alive, uid, parent uid, slot, pos, token,
+ * depth, x1, x2, gate, child1 uid, child2 uid. */
+int lt_read_branch_table(lt_handle* h, int32_t* h_table);
+/* Last pass's readout rows: logits and processed probabilities [max_branches]
+ * [vocab], argmax [max_branches].  Any pointer may be NULL; h_rows unused. */
+int lt_read_readouts(lt_handle* h, float* h_logits, float* h_probs, int32_t* h_arg,
+                     int32_t* h_rows);
+/* Per-step timing of the next n_steps passes of the current decode (starting
+ * one like lt_decode_step if needed), run without the CUDA graph and without
+ * programmatic dependent launch, with CUDA events around every GEMM and
+ * attention launch on the handle's stream.  Bytes are algorithmic: weights,
+ * activation rows and results for GEMMs; (pos+2) K and V rows per row and
+ * shared-block layer for the KV. */
+typedef struct {
+  int steps;
+  int rows;                 /* active rows summed over the steps */
+  double step_ms;           /* summed step times */
+  double gemm_core_ms, gemm_core_bytes;  /* shared-block layer GEMMs */
+  int gemm_core_launches;
+  double gemm_other_ms;     /* prelude / coda / LM-head GEMMs */
+  int gemm_other_launches;
+  double attn_ms;           /* attention + split combine */
+  int attn_launches;
+  double kv_bytes;          /* KV read + written by the shared-block layers */
+  double weight_bytes_core; /* one pass of the shared block's GEMM weights */
+} lt_profile;
+int lt_profile_steps(lt_handle* h, int ar_mode, int n_steps, lt_profile* out);
+
+/* Static facts of a handle (captures the step graph if not done yet). */
+typedef struct {
+  int kernels_per_step;     /* kernel launches in one decode step (graph nodes) */
+  int gemm_grid;            /* CTAs of the shared-block GEMMs (one per SM) */
+  int n_tags;               /* readout depths */
+  int kv_slots;
+  double workspace_bytes;
+  double weight_bytes_core, weight_bytes_prelude_coda, weight_bytes_head;
+} lt_info;
+int lt_get_info(lt_handle* h, lt_info* out);
+
+int lt_reset(lt_handle* h);
+const char* lt_last_error(const lt_handle* h);
+void lt_destroy(lt_handle* h);
+
 /*
  * Stand-alone weight-streaming GEMM of the shared block (tcgen05 + TMEM + TMA):
  *   d_y[i][n] = sum_k d_x[i][k] * d_w[n][k],  i < ncols, n < n_out.

@@ -41,11 +41,76 @@ def lib() -> ctypes.CDLL:
 _vp, _sz, _i = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int
 
 
+class ModelConfigC(ctypes.Structure):
+    _fields_ = [("dtype", _i), ("d_model", _i), ("n_heads", _i), ("head_dim", _i), ("ffn", _i),
+                ("vocab", _i), ("n_prelude", _i), ("n_core", _i), ("n_coda", _i), ("R", _i),
+                ("rms_eps", ctypes.c_float), ("rope_theta", ctypes.c_float),
+                ("resid_scale", ctypes.c_float)]
+
+
+class DecodeConfigC(ctypes.Structure):
+    _fields_ = [("d1", _i), ("d2", _i), ("temperature", ctypes.c_float),
+                ("top_p", ctypes.c_float), ("seed", ctypes.c_uint64), ("max_branches", _i),
+                ("max_ctx", _i), ("max_new", _i), ("second_mode", _i), ("trace_steps", _i)]
+
+
+class StatsC(ctypes.Structure):
+    _fields_ = [(n, _i) for n in ("steps", "rows_sum", "rows_max", "n_first", "n_second",
+                                   "n_fallback", "gate_checks", "gate_opens", "branches_created",
+                                   "resid_fallback", "committed_len")]
+
+    def as_dict(self):
+        return {n: getattr(self, n) for n, _ in self._fields_}
+
+
+class ProfileC(ctypes.Structure):
+    _fields_ = [("steps", _i), ("rows", _i), ("step_ms", ctypes.c_double),
+                ("gemm_core_ms", ctypes.c_double), ("gemm_core_bytes", ctypes.c_double),
+                ("gemm_core_launches", _i), ("gemm_other_ms", ctypes.c_double),
+                ("gemm_other_launches", _i), ("attn_ms", ctypes.c_double),
+                ("attn_launches", _i), ("kv_bytes", ctypes.c_double),
+                ("weight_bytes_core", ctypes.c_double)]
+
+    def as_dict(self):
+        return {n: getattr(self, n) for n, _ in self._fields_}
+
+
+class InfoC(ctypes.Structure):
+    _fields_ = [("kernels_per_step", _i), ("gemm_grid", _i), ("n_tags", _i), ("kv_slots", _i),
+                ("workspace_bytes", ctypes.c_double), ("weight_bytes_core", ctypes.c_double),
+                ("weight_bytes_prelude_coda", ctypes.c_double),
+                ("weight_bytes_head", ctypes.c_double)]
+
+    def as_dict(self):
+        return {n: getattr(self, n) for n, _ in self._fields_}
+
+
+_ip = ctypes.POINTER(ctypes.c_int32)
+
+
 def _declare(L):
     L.lt_gemm_scratch_bytes.argtypes = [_i, _i, _i, _i, ctypes.POINTER(_sz)]
     L.lt_gemm_rows.argtypes = [_i, _vp, _vp, _vp, _i, _i, _i, _vp, _sz, _vp]
-    for name in dir(L):
-        pass
+    L.lt_workspace_bytes.argtypes = [ctypes.POINTER(ModelConfigC), ctypes.POINTER(DecodeConfigC),
+                                     ctypes.POINTER(_sz)]
+    L.lt_create.argtypes = [ctypes.POINTER(ModelConfigC), ctypes.POINTER(DecodeConfigC), _vp, _sz,
+                            _vp, ctypes.POINTER(_vp)]
+    L.lt_load_weights.argtypes = [_vp, _vp, _vp, _vp, ctypes.POINTER(_vp)]
+    L.lt_prefill.argtypes = [_vp, _ip, _i, _ip, _ip, _vp]
+    L.lt_generate.argtypes = [_vp, _i, _i, _ip, ctypes.POINTER(StatsC)]
+    L.lt_decode_step.argtypes = [_vp, _i, _ip, ctypes.POINTER(_i)]
+    L.lt_read_log.argtypes = [_vp, _ip, _ip, _ip, _i]
+    L.lt_read_trace.argtypes = [_vp, _ip, _i]
+    L.lt_read_committed.argtypes = [_vp, _ip, _ip, ctypes.POINTER(_i)]
+    L.lt_read_branch_table.argtypes = [_vp, _ip]
+    L.lt_read_readouts.argtypes = [_vp, _vp, _vp, _ip, _ip]
+    L.lt_profile_steps.argtypes = [_vp, _i, _i, ctypes.POINTER(ProfileC)]
+    L.lt_get_info.argtypes = [_vp, ctypes.POINTER(InfoC)]
+    L.lt_reset.argtypes = [_vp]
+    L.lt_last_error.argtypes = [_vp]
+    L.lt_last_error.restype = ctypes.c_char_p
+    L.lt_destroy.argtypes = [_vp]
+    L.lt_destroy.restype = None
 
 
 def check(code: int, what: str = "") -> None:
@@ -77,3 +142,165 @@ def gemm_rows(w: torch.Tensor, x: torch.Tensor, scratch: torch.Tensor = None,
     check(lib().lt_gemm_rows(dtype, _ptr(w), _ptr(x), _ptr(y), n_out, k, ncols, _ptr(scratch),
                              scratch.numel(), _stream(stream)), "lt_gemm_rows")
     return y
+
+
+# ---------------------------------------------------------------------------
+# decoder handle
+# ---------------------------------------------------------------------------
+
+def _i32p(a):
+    return a.ctypes.data_as(_ip)
+
+
+def model_config_c(cfg) -> ModelConfigC:
+    return ModelConfigC(LT_F32 if cfg.dtype == "f32" else LT_BF16, cfg.d_model, cfg.n_heads,
+                        cfg.head_dim, cfg.ffn, cfg.vocab, cfg.n_prelude, cfg.n_core, cfg.n_coda,
+                        cfg.R, cfg.rms_eps, cfg.rope_theta, cfg.resid_scale)
+
+
+class Decoder:
+    """One lt_handle: caller-side device memory (weights, workspace) and a
+    non-default CUDA stream, owned by this object."""
+
+    def __init__(self, cfg, dec, weights=None, max_branches=16, max_ctx=None, trace_steps=0,
+                 second_mode=0, device="cuda"):
+        import numpy as np
+        self.np = np
+        self.cfg, self.dec = cfg, dec
+        self.device = torch.device(device)
+        self.stream = torch.cuda.Stream(device=self.device)
+        self.mc = model_config_c(cfg)
+        self.dc = DecodeConfigC(dec.d1, dec.d2, dec.temperature, dec.top_p, dec.seed,
+                                max_branches, max_ctx or 4096, dec.max_new, second_mode,
+                                trace_steps)
+        need = _sz()
+        check(lib().lt_workspace_bytes(ctypes.byref(self.mc), ctypes.byref(self.dc),
+                                       ctypes.byref(need)), "lt_workspace_bytes")
+        self.workspace = torch.empty(need.value, dtype=torch.uint8, device=self.device)
+        h = _vp()
+        check(lib().lt_create(ctypes.byref(self.mc), ctypes.byref(self.dc),
+                              self.workspace.data_ptr(), need.value, self.stream.cuda_stream,
+                              ctypes.byref(h)), "lt_create")
+        self.h = h
+        self.n_tags = len({r for r in (dec.d1, dec.d2, cfg.R) if r > 0})
+        self.weights = {}
+        if weights is not None:
+            self.load(weights)
+
+    def _err(self):
+        return lib().lt_last_error(self.h).decode()
+
+    def _check(self, code, what):
+        if code != 0:
+            raise LoopedSpecError(code, f"{what}: {self._err()}")
+
+    def load(self, weights) -> None:
+        """weights: iterable of (name, numpy fp32 array) as produced by
+        synthetic.iter_weights / make_weights (bf16 models hold bf16 values)."""
+        dt = torch.float32 if self.cfg.dtype == "f32" else torch.bfloat16
+        items = weights.items() if isinstance(weights, dict) else weights
+        with torch.cuda.stream(self.stream):
+            for name, a in items:
+                self.weights[name] = torch.from_numpy(a).to(device=self.device, dtype=dt,
+                                                            non_blocking=False)
+        self.stream.synchronize()
+        self.bind_weights()
+
+    def bind_weights(self) -> None:
+        """Hands the device tensors in self.weights to the library."""
+        w = self.weights
+        ptrs = []
+        for ln in self.cfg.layer_names():
+            for t in ("g1", "wqkv", "wo", "g2", "wgu", "wd"):
+                ptrs.append(w[f"{ln}.{t}"].data_ptr())
+        arr = (_vp * len(ptrs))(*ptrs)
+        self._check(lib().lt_load_weights(self.h, w["embed"].data_ptr(),
+                                          w["final_norm"].data_ptr(), w["head"].data_ptr(), arr),
+                    "lt_load_weights")
+
+    def prefill(self, tokens, argmax=False, logits=False):
+        np = self.np
+        tok = np.ascontiguousarray(tokens, dtype=np.int32)
+        first = np.zeros(1, dtype=np.int32)
+        am = np.zeros((len(tok), self.n_tags), dtype=np.int32) if argmax else None
+        lg = (torch.empty(len(tok), self.n_tags, self.cfg.vocab, dtype=torch.float32,
+                          device=self.device) if logits else None)
+        self._check(lib().lt_prefill(self.h, _i32p(tok), len(tok), _i32p(first),
+                                     _i32p(am) if am is not None else None,
+                                     lg.data_ptr() if lg is not None else None), "lt_prefill")
+        return int(first[0]), am, lg
+
+    def generate(self, n, ar=False):
+        np = self.np
+        out = np.zeros(max(n, 1), dtype=np.int32)
+        st = StatsC()
+        self._check(lib().lt_generate(self.h, 1 if ar else 0, n, _i32p(out), ctypes.byref(st)),
+                    "lt_generate")
+        return out[:n].tolist(), st.as_dict()
+
+    def step(self, ar=False):
+        tok = self.np.zeros(1, dtype=self.np.int32)
+        n = _i()
+        self._check(lib().lt_decode_step(self.h, 1 if ar else 0, _i32p(tok), ctypes.byref(n)),
+                    "lt_decode_step")
+        return int(tok[0]) if n.value else None
+
+    def read_log(self, n):
+        np = self.np
+        t, s, k = (np.zeros(max(n, 1), dtype=np.int32) for _ in range(3))
+        self._check(lib().lt_read_log(self.h, _i32p(t), _i32p(s), _i32p(k), n), "lt_read_log")
+        return t[:n].tolist(), s[:n].tolist(), k[:n].tolist()
+
+    def read_trace(self, n_steps):
+        np = self.np
+        tr = np.zeros((max(n_steps, 1), self.dc.max_branches, 4), dtype=np.int32)
+        self._check(lib().lt_read_trace(self.h, _i32p(tr), n_steps), "lt_read_trace")
+        return [[tuple(int(v) for v in row) for row in step if row[0] >= 0]
+                for step in tr[:n_steps]]
+
+    def read_committed(self):
+        np = self.np
+        t = np.zeros(self.dc.max_ctx, dtype=np.int32)
+        s = np.zeros(self.dc.max_ctx, dtype=np.int32)
+        L = _i()
+        self._check(lib().lt_read_committed(self.h, _i32p(t), _i32p(s), ctypes.byref(L)),
+                    "lt_read_committed")
+        return t[:L.value].tolist(), s[:L.value].tolist()
+
+    def read_table(self):
+        np = self.np
+        t = np.zeros((12, self.dc.max_branches), dtype=np.int32)
+        self._check(lib().lt_read_branch_table(self.h, _i32p(t)), "lt_read_branch_table")
+        return t
+
+    def read_readouts(self):
+        np = self.np
+        C, V = self.dc.max_branches, self.cfg.vocab
+        lg = np.zeros((C, V), dtype=np.float32)
+        pr = np.zeros((C, V), dtype=np.float32)
+        am = np.zeros(C, dtype=np.int32)
+        self._check(lib().lt_read_readouts(self.h, lg.ctypes.data, pr.ctypes.data, _i32p(am), None),
+                    "lt_read_readouts")
+        return lg, pr, am
+
+    def profile(self, n_steps, ar=False):
+        p = ProfileC()
+        self._check(lib().lt_profile_steps(self.h, 1 if ar else 0, n_steps, ctypes.byref(p)),
+                    "lt_profile_steps")
+        return p.as_dict()
+
+    def info(self):
+        i = InfoC()
+        self._check(lib().lt_get_info(self.h, ctypes.byref(i)), "lt_get_info")
+        return i.as_dict()
+
+    def close(self):
+        if getattr(self, "h", None):
+            lib().lt_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

@@ -32,7 +32,8 @@ extern "C" int lt_gemm_scratch_bytes(int dtype, int n_out, int k, int ncols, siz
   if (!bytes || n_out <= 0 || k <= 0) return LT_ERR_ARG;
   GemmShape s;
   gemm_plan(n_out, k, dtype == LT_F32, sm_count(), &s, nullptr, nullptr);
-  *bytes = align256((size_t)(2 * s.tiles + s.grid) * sizeof(int)) + gemm_part_bytes(s, ncols);
+  *bytes = align256((size_t)(2 * s.tiles + s.grid) * sizeof(int)) + align256(gemm_part_bytes(s, ncols));
+  if (dtype == LT_F32) *bytes += 2 * align256((size_t)n_out * k * 4) + 2 * align256((size_t)ncols * k * 4);
   return LT_OK;
 }
 
@@ -50,18 +51,44 @@ extern "C" int lt_gemm_rows(int dtype, const void* d_w, const void* d_x, float* 
   gemm_plan(n_out, k, f32, sm_count(), &s, nullptr, nullptr);
   std::vector<int> tab(2 * s.tiles + s.grid);
   gemm_plan(n_out, k, f32, sm_count(), &s, tab.data(), tab.data() + 2 * s.tiles);
-  int* d_tab = (int*)d_scratch;
-  float* part = (float*)((char*)d_scratch + align256(tab.size() * sizeof(int)));
+  char* cur = (char*)d_scratch;
+  int* d_tab = (int*)cur;
+  cur += align256(tab.size() * sizeof(int));
+  float* part = (float*)cur;
+  cur += align256(gemm_part_bytes(s, ncols));
   cudaStream_t st = (cudaStream_t)stream;
   if (cudaMemcpyAsync(d_tab, tab.data(), tab.size() * sizeof(int), cudaMemcpyHostToDevice, st) !=
       cudaSuccess)
     return LT_ERR_CUDA;
   s.tile_c = d_tab;
   s.cta_t0 = d_tab + 2 * s.tiles;
-  CUtensorMap tw, tx;
-  if (make_tmap(&tw, d_w, f32, n_out, k, GEMM_BM) != 0) return LT_ERR_SHAPE;
-  if (make_tmap(&tx, d_x, f32, ncols, k, ncols) != 0) return LT_ERR_SHAPE;
-  if (gemm_launch(tw, tx, part, s, ncols, f32, nullptr, nullptr, st, false) != cudaSuccess)
+  CUtensorMap tw, tx, twl, txl;
+  const void* w_hi = d_w;
+  const void* x_hi = d_x;
+  if (f32) {  // fp32 operands run as split tf32 (hi + lo pairs)
+    float* wh = (float*)cur;
+    cur += align256((size_t)n_out * k * 4);
+    float* wl = (float*)cur;
+    cur += align256((size_t)n_out * k * 4);
+    float* xh = (float*)cur;
+    cur += align256((size_t)ncols * k * 4);
+    float* xl = (float*)cur;
+    if (split_tf32((const float*)d_w, wh, wl, (size_t)n_out * k, st) != cudaSuccess ||
+        split_tf32((const float*)d_x, xh, xl, (size_t)ncols * k, st) != cudaSuccess)
+      return LT_ERR_CUDA;
+    w_hi = wh;
+    x_hi = xh;
+    if (make_tmap(&twl, wl, true, n_out, k, GEMM_BM) != 0) return LT_ERR_SHAPE;
+    if (make_tmap(&txl, xl, true, ncols, k, ncols) != 0) return LT_ERR_SHAPE;
+  }
+  if (make_tmap(&tw, w_hi, f32, n_out, k, GEMM_BM) != 0) return LT_ERR_SHAPE;
+  if (make_tmap(&tx, x_hi, f32, ncols, k, ncols) != 0) return LT_ERR_SHAPE;
+  if (!f32) {
+    twl = tw;
+    txl = tx;
+  }
+  if (gemm_launch(tw, twl, tx, txl, part, s, ncols, f32 ? 2 : 0, nullptr, nullptr, st, false) !=
+      cudaSuccess)
     return LT_ERR_CUDA;
   dim3 grid((n_out + 255) / 256, ncols);
   k_reduce_rows<<<grid, 256, 0, st>>>(part, s, ncols, d_y);

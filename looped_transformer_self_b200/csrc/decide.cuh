@@ -1,0 +1,721 @@
+// Readout processing, proposal / accept / resample decisions and on-device
+// branch + KV-slot bookkeeping of the pipelined speculative decoder.
+//
+// Follows "LoopSpec: Pipelined Self-Speculative Decoding for Looped
+// Transformers" (liuzhao09.github.io/papers/loopspec.html):
+//  * section 2.1: the readout C = final norm, LM head, temperature, optional
+//    top-p truncation, normalisation -- applied at every readout depth;
+//  * section 2.2, Eqs. 2-4: residual operator, accept min(1, p/q), resample
+//    from p (-) q; a branch opens a child at its depth-d1 proposal and is
+//    verified at depth R; a rejection prunes every descendant of the wrong
+//    prefix; the tree is re-rooted on every verification;
+//  * section 2.3, Eqs. 5-6: gated residual second proposal and the cascade;
+//  * section 2.4: a child copies its parent's cache indices; pruning frees
+//    only slots no surviving path needs.
+// Readings where the pages are silent (shared with the test oracle, which is
+// written separately): greedy readouts are one-hot argmax (lowest index on
+// ties); top-p keeps every token with p >= theta*, theta* the largest
+// probability value whose upper set holds >= top_p of the mass; draws use the
+// exponential race over Philox-4x32-10 words keyed (seed, uid|position,
+// purpose); the accept test is u * q(x) < p(x) with 24-bit u; the per-step
+// order is: prelude, iterate, readouts, proposals (ascending uid), verify,
+// prune / re-root (frees after this step's allocations).
+#pragma once
+
+#include "common.cuh"
+
+namespace lt {
+
+constexpr int CMAX = 64;        // branch-table capacity limit (= max GEMM columns)
+constexpr int WIN = 32;         // chain window: uncommitted positions a branch may span
+constexpr int MAX_SLOT_WORDS = 2048;  // slot bitmap words held in shared memory (65536 slots)
+
+struct Ctl {
+  int L;              // committed length (prompt + generated)
+  int target_len;     // generation stops when L reaches it
+  int pos_limit;      // a child is created only for pos + 1 < pos_limit
+  int next_uid;
+  int finished;
+  int ar_mode;        // 1: full-depth autoregressive (no proposals)
+  int prepared;       // table depths hold the next iteration's depths
+  int flag_run, flag_new, flag_ro;  // work present in the prepared step
+  int rows_cur;
+  int commit_pending, commit_tok, commit_src;
+  int n_commit;       // commits logged since the log was reset
+  int err;
+  // statistics (Eq. 9's counts, Fig. 5 rows, Table 6 gate rate)
+  int steps, rows_sum, rows_max, n_first, n_second, n_fallback;
+  int gate_checks, gate_opens, branches_created, resid_fallback;
+};
+
+struct Dev {
+  int d, V, R, C, S, d1, d2, greedy, second_mode, trace_cap, max_ctx;
+  float T, top_p;
+  unsigned long long seed;
+  int tag_of_depth[33];
+  Ctl* ctl;
+  // branch table
+  int *b_alive, *b_uid, *b_parent, *b_slot, *b_pos, *b_tok, *b_depth, *b_x1, *b_x2, *b_gate,
+      *b_c1, *b_c2, *b_chain;
+  // rows of the prepared pass
+  int *r_tok, *r_pos, *r_slot, *r_depth, *r_ro, *r_blen, *r_boff, *m_alive, *m_new, *m_ro;
+  int* lists;      // committed slots
+  int* committed;  // committed tokens
+  unsigned int* slot_bits;
+  int *log_tok, *log_src, *log_step;
+  int* trace;      // [trace_cap][C][4]
+  int* ro_arg;
+  float *logits, *P, *q1, *q2, *rho, *rho2;
+};
+
+// ---------------------------------------------------------------------------
+// block helpers
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ bool better_min(float k, int i, float bk, int bi) {
+  return k < bk || (k == bk && i < bi);
+}
+__device__ __forceinline__ bool better_max(float k, int i, float bk, int bi) {
+  return k > bk || (k == bk && i < bi);
+}
+
+// Block-wide arg-min (MIN=true) or arg-max of (key, index), lowest index on ties.
+template <bool MIN>
+__device__ __forceinline__ int block_arg(float k, int idx, float* sk, int* si) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float k2 = __shfl_xor_sync(0xffffffffu, k, o);
+    const int i2 = __shfl_xor_sync(0xffffffffu, idx, o);
+    if (MIN ? better_min(k2, i2, k, idx) : better_max(k2, i2, k, idx)) {
+      k = k2;
+      idx = i2;
+    }
+  }
+  __syncthreads();
+  if (lane == 0) {
+    sk[w] = k;
+    si[w] = idx;
+  }
+  __syncthreads();
+  if (w == 0) {
+    k = lane < nw ? sk[lane] : (MIN ? INFINITY : -INFINITY);
+    idx = lane < nw ? si[lane] : 0x7fffffff;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float k2 = __shfl_xor_sync(0xffffffffu, k, o);
+      const int i2 = __shfl_xor_sync(0xffffffffu, idx, o);
+      if (MIN ? better_min(k2, i2, k, idx) : better_max(k2, i2, k, idx)) {
+        k = k2;
+        idx = i2;
+      }
+    }
+    if (lane == 0) si[32] = idx;
+  }
+  __syncthreads();
+  return si[32];
+}
+
+// Exponential race over weights w[0..V) (w_j <= 0 never chosen).
+__device__ __forceinline__ int block_race(const float* __restrict__ w, int V,
+                                          unsigned long long seed, uint32_t stream,
+                                          uint32_t purpose, float* sk, int* si) {
+  float best = INFINITY;
+  int bi = 0x7fffffff;
+  for (int j = threadIdx.x; j < V; j += blockDim.x) {
+    const float wj = w[j];
+    if (wj > 0.f) {
+      const float k = race_key(seed, stream, purpose, (uint32_t)j, wj);
+      if (better_min(k, j, best, bi)) {
+        best = k;
+        bi = j;
+      }
+    }
+  }
+  return block_arg<true>(best, bi, sk, si);
+}
+
+// Inclusive suffix sums of 1024 u64 bins held one per thread (blockDim 1024).
+__device__ __forceinline__ unsigned long long suffix_scan_1024(unsigned long long v,
+                                                              unsigned long long* wsum) {
+  // prefix scan over reversed order: thread t holds bin 1023 - t
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned long long t = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += t;
+  }
+  __syncthreads();
+  if (lane == 31) wsum[w] = v;
+  __syncthreads();
+  if (w == 0) {
+    unsigned long long s = wsum[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const unsigned long long t = __shfl_up_sync(0xffffffffu, s, o);
+      if (lane >= o) s += t;
+    }
+    wsum[lane] = s;
+  }
+  __syncthreads();
+  return v + (w > 0 ? wsum[w - 1] : 0ull);
+}
+
+// ---------------------------------------------------------------------------
+// K4: readout processing of LM-head partials (one block of 1024 per readout row)
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(1024)
+    k_readout(const float* __restrict__ part, const GemmShape s, int C,
+              const int* __restrict__ mask, int V, int greedy, float T, float top_p,
+              float* __restrict__ logits, float* __restrict__ P, int* __restrict__ arg) {
+  __shared__ float sk[33];
+  __shared__ int si[33];
+  __shared__ float red[33];
+  __shared__ unsigned long long hist[1024];
+  __shared__ unsigned long long wsum[32];
+  __shared__ int sel[2];
+  __shared__ unsigned long long sel_above[1];
+  pdl_wait();
+  pdl_trigger();
+  const int i = blockIdx.x;
+  if (!mask[i]) return;
+  float* z = logits + (size_t)i * V;
+  float* p = P + (size_t)i * V;
+  float best = -INFINITY;
+  int bi = 0x7fffffff;
+  for (int j = threadIdx.x; j < V; j += blockDim.x) {
+    const float v = sk_reduce(part, s, C, i, j);
+    z[j] = v;
+    if (better_max(v, j, best, bi)) {
+      best = v;
+      bi = j;
+    }
+  }
+  const int a = block_arg<false>(best, bi, sk, si);
+  if (threadIdx.x == 0) arg[i] = a;
+  if (greedy) return;
+  // softmax(z / T)
+  const float zmax = z[a];  // same thread may not have written it: reread after the barrier
+  const float invT = 1.f / T;
+  float ssum = 0.f;
+  for (int j = threadIdx.x; j < V; j += blockDim.x) {
+    const float e = expf((z[j] - zmax) * invT);
+    p[j] = e;
+    ssum += e;
+  }
+  const float Z = block_sum(ssum, red);
+  const float invZ = 1.f / Z;
+  if (!(top_p < 1.f)) {
+    for (int j = threadIdx.x; j < V; j += blockDim.x) p[j] *= invZ;
+    return;
+  }
+  // exact top-p threshold: 3-level radix select over the float bits of p with
+  // integer (2^-40) mass, so the sums do not depend on thread order
+  const double SCALE = 1099511627776.0;  // 2^40
+  const unsigned long long target = (unsigned long long)((double)top_p * SCALE + 0.5);
+  unsigned long long above = 0ull;
+  uint32_t prefix = 0u;
+  const int shifts[3] = {20, 10, 0};
+  bool all = false;
+  for (int lvl = 0; lvl < 3; ++lvl) {
+    hist[threadIdx.x] = 0ull;
+    __syncthreads();
+    const int sh = shifts[lvl];
+    for (int j = threadIdx.x; j < V; j += blockDim.x) {
+      const float pj = (lvl == 0) ? p[j] * invZ : p[j];
+      if (lvl == 0) p[j] = pj;
+      const uint32_t b = __float_as_uint(pj);
+      if (lvl == 0 || (b >> (sh + 10)) == prefix) {
+        const unsigned long long m = (unsigned long long)((double)pj * SCALE + 0.5);
+        atomicAdd(&hist[(b >> sh) & 1023u], m);
+      }
+    }
+    __syncthreads();
+    const int bin = 1023 - threadIdx.x;
+    const unsigned long long hv = hist[bin];
+    const unsigned long long cum = suffix_scan_1024(hv, wsum);  // mass of bins >= bin
+    if (threadIdx.x == 0) sel[0] = -1;
+    __syncthreads();
+    if (above + cum >= target && above + cum - hv < target) {
+      sel[0] = bin;
+      sel_above[0] = above + cum - hv;
+    }
+    __syncthreads();
+    if (sel[0] < 0) {
+      all = true;
+      break;
+    }
+    above = sel_above[0];
+    prefix = (prefix << 10) | (uint32_t)sel[0];
+    __syncthreads();
+  }
+  const uint32_t theta = all ? 0u : prefix;
+  float ks = 0.f;
+  for (int j = threadIdx.x; j < V; j += blockDim.x) {
+    const float pj = p[j];
+    if (__float_as_uint(pj) >= theta) ks += pj;
+  }
+  const float Z2 = block_sum(ks, red);
+  const float inv2 = 1.f / Z2;
+  for (int j = threadIdx.x; j < V; j += blockDim.x) {
+    const float pj = p[j];
+    p[j] = __float_as_uint(pj) >= theta ? pj * inv2 : 0.f;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// K5: proposals at d1 / d2 and the verification cascade at R (one block per
+// readout row).  The table entry's x1 / gate / x2 and the q1 / q2 vectors are
+// stored for the verification at R (D5 of the branch state).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float residual_into(const float* __restrict__ mu,
+                                               const float* __restrict__ nu, int V,
+                                               float* __restrict__ out, float* red) {
+  float zs = 0.f;
+  for (int j = threadIdx.x; j < V; j += blockDim.x) {
+    const float w = fmaxf(mu[j] - nu[j], 0.f);
+    out[j] = w;
+    zs += w;
+  }
+  const float Z = block_sum(zs, red);
+  if (Z > 0.f) {
+    const float inv = 1.f / Z;
+    for (int j = threadIdx.x; j < V; j += blockDim.x) out[j] *= inv;
+  }
+  __syncthreads();
+  return Z;
+}
+
+__global__ void __launch_bounds__(1024) k_decide(Dev D) {
+  __shared__ float sk[33];
+  __shared__ int si[33];
+  __shared__ float red[33];
+  pdl_wait();
+  pdl_trigger();
+  Ctl* c = D.ctl;
+  const int i = blockIdx.x;
+  if (c->finished || !D.m_ro[i]) return;
+  const int r = D.r_depth[i];
+  const int uid = D.b_uid[i];
+  const bool ar = c->ar_mode != 0;
+  const int V = D.V;
+  const bool t0 = threadIdx.x == 0;
+  const bool prop1 = !ar && r == D.d1;
+  const bool prop2 = !ar && D.d2 > 0 && r == D.d2 && D.b_x1[i] >= 0;
+  if (r == D.R && D.r_pos[i] != c->L - 1) {
+    if (t0) set_err(&c->err, DEV_STATE);
+    return;
+  }
+  if (D.greedy) {
+    if (!t0) return;
+    const int a = D.ro_arg[i];
+    if (prop1) D.b_x1[i] = a;
+    if (prop2) {
+      const int g = a != D.b_x1[i];
+      D.b_gate[i] = g;
+      D.b_x2[i] = g ? a : -1;
+      atomicAdd(&c->gate_checks, 1);
+      atomicAdd(&c->gate_opens, g);
+    }
+    if (r == D.R) {
+      int src = 0;
+      if (!ar) {
+        if (D.b_x1[i] >= 0 && a == D.b_x1[i]) src = 1;
+        else if (D.b_gate[i] && a == D.b_x2[i]) src = 2;
+      }
+      c->commit_tok = a;
+      c->commit_src = src;
+      c->commit_pending = 1;
+    }
+    return;
+  }
+  const float* p = D.P + (size_t)i * V;
+  float* q1 = D.q1 + (size_t)i * V;
+  float* q2 = D.q2 + (size_t)i * V;
+  if (prop1) {
+    for (int j = threadIdx.x; j < V; j += blockDim.x) q1[j] = p[j];
+    const int x1 = block_race(p, V, D.seed, (uint32_t)uid, P_PROP1, sk, si);
+    if (t0) D.b_x1[i] = x1;
+  }
+  if (prop2) {
+    const int x1 = D.b_x1[i];
+    int open = 0;
+    if (D.second_mode == 0) {  // gated residual (Eqs. 5-6)
+      if (p[x1] < q1[x1]) open = residual_into(p, q1, V, q2, red) > 0.f;
+    } else if (D.second_mode == 1) {  // residual, no gate (ablation)
+      open = residual_into(p, q1, V, q2, red) > 0.f;
+    } else {  // non-residual ablation (section 3.4): p_d2 with x1 removed, renormalised
+      float zs = 0.f;
+      for (int j = threadIdx.x; j < V; j += blockDim.x) {
+        const float w = j == x1 ? 0.f : p[j];
+        q2[j] = w;
+        zs += w;
+      }
+      const float Z = block_sum(zs, red);
+      if (Z > 0.f) {
+        for (int j = threadIdx.x; j < V; j += blockDim.x) q2[j] /= Z;
+        open = 1;
+      }
+      __syncthreads();
+    }
+    int x2 = -1;
+    if (open) x2 = block_race(q2, V, D.seed, (uint32_t)uid, P_PROP2, sk, si);
+    if (t0) {
+      D.b_gate[i] = open;
+      D.b_x2[i] = x2;
+      atomicAdd(&c->gate_checks, 1);
+      atomicAdd(&c->gate_opens, open);
+    }
+  }
+  if (r != D.R) return;
+  // verification at full depth
+  int x, src = 0, fb = 0;
+  if (ar) {
+    x = block_race(p, V, D.seed, (uint32_t)(D.r_pos[i] + 1), P_AR, sk, si);
+  } else if (D.b_x1[i] < 0) {
+    x = block_race(p, V, D.seed, (uint32_t)uid, P_RES, sk, si);
+  } else {
+    const int x1 = D.b_x1[i];
+    const float u1 = uniform01(D.seed, (uint32_t)uid, P_ACC1);
+    if (u1 * q1[x1] < p[x1]) {
+      x = x1;
+      src = 1;
+    } else {
+      const float* rho1 = D.rho;
+      if (!(residual_into(p, q1, V, D.rho, red) > 0.f)) {
+        rho1 = p;  // unreachable in exact arithmetic
+        fb = 1;
+      }
+      const int x2 = D.b_x2[i];
+      if (D.b_gate[i] && x2 >= 0) {
+        const float u2 = uniform01(D.seed, (uint32_t)uid, P_ACC2);
+        if (u2 * q2[x2] < rho1[x2]) {
+          x = x2;
+          src = 2;
+        } else {
+          const float* r2 = D.rho2;
+          if (!(residual_into(rho1, q2, V, D.rho2, red) > 0.f)) {
+            r2 = rho1;
+            fb += 1;
+          }
+          x = block_race(r2, V, D.seed, (uint32_t)uid, P_RES, sk, si);
+        }
+      } else {
+        x = block_race(rho1, V, D.seed, (uint32_t)uid, P_RES, sk, si);
+      }
+    }
+  }
+  if (t0) {
+    c->commit_tok = x;
+    c->commit_src = src;
+    c->commit_pending = 1;
+    if (fb) atomicAdd(&c->resid_fallback, fb);
+  }
+}
+
+// First token after prefill: full-depth readout of the last prompt position,
+// drawn with the stream (position P, AR) like every autoregressive draw.
+__global__ void __launch_bounds__(1024) k_first_token(Dev D, int row, int P_len) {
+  __shared__ float sk[33];
+  __shared__ int si[33];
+  pdl_wait();
+  pdl_trigger();
+  int x;
+  if (D.greedy) x = D.ro_arg[row];
+  else x = block_race(D.P + (size_t)row * D.V, D.V, D.seed, (uint32_t)P_len, P_AR, sk, si);
+  if (threadIdx.x == 0) {
+    D.committed[P_len] = x;
+    D.ctl->L = P_len + 1;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// K6: branch / KV-slot bookkeeping (one block; the tree logic runs on one
+// thread over shared-memory copies of the table, which is <= 64 entries).
+// mode 0: apply this step's proposals and commit, prune / re-root, prepare the
+// next step.  mode 1: make sure a root exists and the next step is prepared.
+// ---------------------------------------------------------------------------
+struct BookSmem {
+  int alive[CMAX], uid[CMAX], parent[CMAX], slot[CMAX], pos[CMAX], tok[CMAX], depth[CMAX],
+      x1[CMAX], x2[CMAX], gate[CMAX], c1[CMAX], c2[CMAX];
+  int chain[CMAX * WIN];
+  unsigned int bits[MAX_SLOT_WORDS];
+  int order[CMAX];
+};
+
+__device__ int bk_alloc_slot(BookSmem& b, int S, int* err) {
+  const int words = (S + 31) >> 5;
+  for (int w = 0; w < words; ++w) {
+    const unsigned int v = b.bits[w];
+    if (v != 0xffffffffu) {
+      const int bit = __ffs(~v) - 1;
+      const int s = w * 32 + bit;
+      if (s >= S) break;
+      b.bits[w] = v | (1u << bit);
+      return s;
+    }
+  }
+  set_err(err, DEV_SLOTS_FULL);
+  return -1;
+}
+__device__ void bk_free_slot(BookSmem& b, int s) { b.bits[s >> 5] &= ~(1u << (s & 31)); }
+
+__device__ int bk_new_entry(BookSmem& b, const Dev& D, Ctl& c, int parent_e, int pos, int tok,
+                            int depth, bool prepared) {
+  int e = -1;
+  for (int k = 0; k < D.C; ++k)
+    if (!b.alive[k]) {
+      e = k;
+      break;
+    }
+  if (e < 0) {
+    set_err(&c.err, DEV_TABLE_FULL);
+    return -1;
+  }
+  const int s = bk_alloc_slot(b, D.S, &c.err);
+  if (s < 0) return -1;
+  if (pos - (c.L - 1) >= WIN) {
+    set_err(&c.err, DEV_CHAIN);
+    return -1;
+  }
+  b.alive[e] = 1;
+  b.uid[e] = c.next_uid++;
+  b.parent[e] = parent_e >= 0 ? b.uid[parent_e] : -1;
+  b.slot[e] = s;
+  b.pos[e] = pos;
+  b.tok[e] = tok;
+  b.depth[e] = depth;
+  b.x1[e] = b.x2[e] = -1;
+  b.gate[e] = 0;
+  b.c1[e] = b.c2[e] = -1;
+  if (parent_e >= 0)
+    for (int k = 0; k < WIN; ++k) b.chain[e * WIN + k] = b.chain[parent_e * WIN + k];
+  b.chain[e * WIN + (pos % WIN)] = s;
+  c.branches_created++;
+  (void)prepared;
+  return e;
+}
+
+__device__ int bk_find_uid(const BookSmem& b, int C, int uid) {
+  if (uid < 0) return -1;
+  for (int k = 0; k < C; ++k)
+    if (b.alive[k] && b.uid[k] == uid) return k;
+  return -1;
+}
+
+__device__ void bk_logic(BookSmem& b, const Dev& D, Ctl& c, int mode) {
+  const int C = D.C;
+  if (mode == 0 && c.prepared) {
+    c.prepared = 0;
+    c.steps++;
+    c.rows_sum += c.rows_cur;
+    c.rows_max = max(c.rows_max, c.rows_cur);
+    int n = 0;
+    for (int k = 0; k < C; ++k)
+      if (b.alive[k]) b.order[n++] = k;
+    for (int a = 1; a < n; ++a) {  // ascending uid
+      const int v = b.order[a];
+      int j = a - 1;
+      while (j >= 0 && b.uid[b.order[j]] > b.uid[v]) {
+        b.order[j + 1] = b.order[j];
+        --j;
+      }
+      b.order[j + 1] = v;
+    }
+    if (!c.ar_mode) {
+      for (int a = 0; a < n; ++a) {
+        const int e = b.order[a];
+        const bool spawn = b.pos[e] + 1 < c.pos_limit;
+        if (!spawn) continue;
+        if (b.depth[e] == D.d1 && b.x1[e] >= 0) {
+          const int ch = bk_new_entry(b, D, c, e, b.pos[e] + 1, b.x1[e], 0, false);
+          if (ch < 0) return;
+          b.c1[e] = b.uid[ch];
+        } else if (D.d2 > 0 && b.depth[e] == D.d2 && b.gate[e] && b.x2[e] >= 0) {
+          const int ch = bk_new_entry(b, D, c, e, b.pos[e] + 1, b.x2[e], 0, false);
+          if (ch < 0) return;
+          b.c2[e] = b.uid[ch];
+        }
+      }
+    }
+    if (c.commit_pending) {
+      c.commit_pending = 0;
+      const int x = c.commit_tok, src = c.commit_src;
+      int root = -1;
+      for (int k = 0; k < C; ++k)
+        if (b.alive[k] && b.pos[k] == c.L - 1) root = k;
+      if (root < 0 || c.L >= D.max_ctx) {
+        set_err(&c.err, DEV_NO_ROOT);
+        return;
+      }
+      D.committed[c.L] = x;
+      D.log_tok[c.n_commit] = x;
+      D.log_src[c.n_commit] = src;
+      D.log_step[c.n_commit] = c.steps;
+      c.n_commit++;
+      c.L++;
+      if (src == 1) c.n_first++;
+      else if (src == 2) c.n_second++;
+      else c.n_fallback++;
+      const int surv = bk_find_uid(b, C, src == 1 ? b.c1[root] : src == 2 ? b.c2[root] : -1);
+      for (int k = 0; k < C; ++k) {
+        if (!b.alive[k]) continue;
+        bool keep = false;
+        if (surv >= 0)
+          keep = k == surv || (b.pos[k] > b.pos[surv] &&
+                               b.chain[k * WIN + (b.pos[surv] % WIN)] == b.slot[surv]);
+        if (!keep) {
+          b.alive[k] = 0;
+          if (k != root) bk_free_slot(b, b.slot[k]);
+        }
+      }
+      if (surv >= 0) {
+        b.parent[surv] = -1;
+        D.lists[c.L - 1] = b.slot[surv];
+      } else if (c.L < c.target_len) {
+        const int e = bk_new_entry(b, D, c, -1, c.L - 1, x, 0, false);
+        if (e < 0) return;
+        D.lists[c.L - 1] = b.slot[e];
+      }
+      if (c.L >= c.target_len) c.finished = 1;
+    }
+    if (c.finished) return;
+    for (int k = 0; k < C; ++k)
+      if (b.alive[k]) b.depth[k]++;
+    c.prepared = 1;
+  } else if (mode == 1) {
+    if (c.finished) return;
+    int root = -1;
+    for (int k = 0; k < C; ++k)
+      if (b.alive[k] && b.pos[k] == c.L - 1) root = k;
+    if (root < 0) {
+      const int e = bk_new_entry(b, D, c, -1, c.L - 1, D.committed[c.L - 1], c.prepared ? 1 : 0,
+                                 c.prepared);
+      if (e < 0) return;
+      D.lists[c.L - 1] = b.slot[e];
+    }
+    if (!c.prepared) {
+      for (int k = 0; k < C; ++k)
+        if (b.alive[k]) b.depth[k]++;
+      c.prepared = 1;
+    }
+  }
+}
+
+__global__ void __launch_bounds__(256) k_book(Dev D, int mode) {
+  __shared__ BookSmem b;
+  pdl_wait();
+  pdl_trigger();
+  Ctl* cg = D.ctl;
+  const int C = D.C, words = (D.S + 31) >> 5;
+  for (int k = threadIdx.x; k < C; k += blockDim.x) {
+    b.alive[k] = D.b_alive[k];
+    b.uid[k] = D.b_uid[k];
+    b.parent[k] = D.b_parent[k];
+    b.slot[k] = D.b_slot[k];
+    b.pos[k] = D.b_pos[k];
+    b.tok[k] = D.b_tok[k];
+    b.depth[k] = D.b_depth[k];
+    b.x1[k] = D.b_x1[k];
+    b.x2[k] = D.b_x2[k];
+    b.gate[k] = D.b_gate[k];
+    b.c1[k] = D.b_c1[k];
+    b.c2[k] = D.b_c2[k];
+  }
+  for (int k = threadIdx.x; k < C * WIN; k += blockDim.x) b.chain[k] = D.b_chain[k];
+  for (int k = threadIdx.x; k < words; k += blockDim.x) b.bits[k] = D.slot_bits[k];
+  __shared__ Ctl c;
+  if (threadIdx.x == 0) c = *cg;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    if (!c.err) bk_logic(b, D, c, mode);
+    if (c.err) c.finished = 1;
+    // rebuild the rows of the prepared step
+    int rows = 0, any_new = 0, any_ro = 0;
+    const bool on_all = c.prepared && !c.finished;
+    for (int k = 0; k < C; ++k) {
+      const int on = on_all && b.alive[k];
+      const int dep = b.depth[k];
+      int ro = -1;
+      if (on && dep >= 1 && dep <= D.R) ro = c.ar_mode ? (dep == D.R ? D.tag_of_depth[D.R] : -1)
+                                                      : D.tag_of_depth[dep];
+      D.m_alive[k] = on;
+      D.m_new[k] = on && dep == 1;
+      D.m_ro[k] = ro >= 0;
+      D.r_ro[k] = ro;
+      D.r_tok[k] = b.tok[k];
+      D.r_pos[k] = b.pos[k];
+      D.r_slot[k] = b.slot[k];
+      D.r_depth[k] = dep;
+      D.r_blen[k] = c.L;
+      D.r_boff[k] = 0;
+      rows += on;
+      any_new |= on && dep == 1;
+      any_ro |= ro >= 0;
+    }
+    c.rows_cur = rows;
+    c.flag_run = rows > 0;
+    c.flag_new = any_new;
+    c.flag_ro = any_ro;
+    if (on_all && c.steps < D.trace_cap) {
+      int n = 0;
+      for (int k = 0; k < C; ++k)
+        if (b.alive[k]) b.order[n++] = k;
+      for (int a = 1; a < n; ++a) {
+        const int v = b.order[a];
+        int j = a - 1;
+        while (j >= 0 && b.uid[b.order[j]] > b.uid[v]) {
+          b.order[j + 1] = b.order[j];
+          --j;
+        }
+        b.order[j + 1] = v;
+      }
+      int* tr = D.trace + (size_t)c.steps * C * 4;
+      for (int a = 0; a < C; ++a) {
+        const int e = a < n ? b.order[a] : -1;
+        tr[4 * a + 0] = e >= 0 ? b.uid[e] : -1;
+        tr[4 * a + 1] = e >= 0 ? b.slot[e] : -1;
+        tr[4 * a + 2] = e >= 0 ? b.pos[e] : -1;
+        tr[4 * a + 3] = e >= 0 ? b.depth[e] : -1;
+      }
+    }
+    *cg = c;
+  }
+  __syncthreads();
+  for (int k = threadIdx.x; k < C; k += blockDim.x) {
+    D.b_alive[k] = b.alive[k];
+    D.b_uid[k] = b.uid[k];
+    D.b_parent[k] = b.parent[k];
+    D.b_slot[k] = b.slot[k];
+    D.b_pos[k] = b.pos[k];
+    D.b_tok[k] = b.tok[k];
+    D.b_depth[k] = b.depth[k];
+    D.b_x1[k] = b.x1[k];
+    D.b_x2[k] = b.x2[k];
+    D.b_gate[k] = b.gate[k];
+    D.b_c1[k] = b.c1[k];
+    D.b_c2[k] = b.c2[k];
+  }
+  for (int k = threadIdx.x; k < C * WIN; k += blockDim.x) D.b_chain[k] = b.chain[k];
+  for (int k = threadIdx.x; k < words; k += blockDim.x) D.slot_bits[k] = b.bits[k];
+}
+
+// Rows of one prefill chunk: prompt positions c0 .. c0+n-1 (slots = positions).
+__global__ void k_prefill_rows(Dev D, int c0, int n, int P_len, int depth, int ro_tag) {
+  pdl_wait();
+  pdl_trigger();
+  for (int k = threadIdx.x; k < D.C; k += blockDim.x) {
+    const int on = k < n;
+    D.m_alive[k] = on;
+    D.m_new[k] = on && depth == 0;
+    D.r_tok[k] = on ? D.committed[c0 + k] : 0;
+    D.r_pos[k] = on ? c0 + k : 0;
+    D.r_slot[k] = on ? c0 + k : 0;
+    D.r_depth[k] = depth;
+    D.r_ro[k] = on ? ro_tag : -1;
+    D.m_ro[k] = on && ro_tag >= 0;
+    D.r_blen[k] = P_len;
+    D.r_boff[k] = 0;
+  }
+}
+
+}  // namespace lt

@@ -134,13 +134,21 @@ constexpr int tmem_cols() {
 // ---------------------------------------------------------------------------
 // kernel
 // ---------------------------------------------------------------------------
-template <bool TF32, int NC>
+// MODE 0: bf16 operands.  MODE 1: tf32 operands.  MODE 2: fp32 operands as
+// hi + lo tf32 pairs (hi = value with the low 13 mantissa bits cleared, lo =
+// the exact remainder); each k-step issues hi*hi + hi*lo + lo*hi, which keeps
+// the products to ~2^-21 relative error (fp32-grade) on the tensor cores.
+template <int MODE, int NC>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
-    k_gemm(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
+    k_gemm(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmWlo,
+           const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmXlo,
            float* __restrict__ part, const GemmShape s, const int stages,
            const int* __restrict__ run_flag, int* __restrict__ err) {
+  constexpr bool TF32 = MODE != 0;
+  constexpr int NSPLIT = MODE == 2 ? 2 : 1;
   constexpr uint32_t A_BYTES = GEMM_BM * GEMM_CHUNK_BYTES;
   constexpr uint32_t B_BYTES = NC * GEMM_CHUNK_BYTES;
+  constexpr uint32_t SA = NSPLIT * A_BYTES, SB = NSPLIT * B_BYTES;  // per-stage bytes
   constexpr int BKE = TF32 ? 32 : 64;  // elements per k-chunk
   constexpr int TCOLS = tmem_cols<NC>();
   constexpr uint32_t IDESC = instr_desc<TF32, NC>();
@@ -156,8 +164,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* gbase = smem_raw + (base - raw);
   const uint32_t a_base = base;
-  const uint32_t b_base = base + stages * A_BYTES;
-  const uint32_t bar_base = b_base + stages * B_BYTES;  // 8-byte aligned
+  const uint32_t b_base = base + stages * SA;
+  const uint32_t bar_base = b_base + stages * SB;  // 8-byte aligned
   // barriers: full[stages], empty[stages], accf[2], acce[2], drain
   auto full_bar = [&](int i) { return bar_base + 8u * i; };
   auto empty_bar = [&](int i) { return bar_base + 8u * (stages + i); };
@@ -183,6 +191,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmW)) : "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmX)) : "memory");
+    if constexpr (NSPLIT == 2) {
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmWlo)) : "memory");
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmXlo)) : "memory");
+    }
   }
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -207,10 +219,14 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         for (int uu = u; uu < seg_end; ++uu, ++g) {
           const int st = g % stages, n = g / stages;
           if (!mbar_wait(empty_bar(st), (n & 1) ^ 1, abort_flag)) break;
-          mbar_expect_tx(full_bar(st), A_BYTES + B_BYTES);
+          mbar_expect_tx(full_bar(st), SA + SB);
           const int kx = (uu - t * s.kch) * BKE;
-          tma_load_2d(a_base + st * A_BYTES, &tmW, kx, t * GEMM_BM, full_bar(st), pol_w);
-          tma_load_2d(b_base + st * B_BYTES, &tmX, kx, 0, full_bar(st), pol_x);
+          tma_load_2d(a_base + st * SA, &tmW, kx, t * GEMM_BM, full_bar(st), pol_w);
+          tma_load_2d(b_base + st * SB, &tmX, kx, 0, full_bar(st), pol_x);
+          if constexpr (NSPLIT == 2) {
+            tma_load_2d(a_base + st * SA + A_BYTES, &tmWlo, kx, t * GEMM_BM, full_bar(st), pol_w);
+            tma_load_2d(b_base + st * SB + B_BYTES, &tmXlo, kx, 0, full_bar(st), pol_x);
+          }
         }
         u = seg_end;
       }
@@ -237,11 +253,20 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t a0 = a_base + st * A_BYTES, b0 = b_base + st * B_BYTES;
+          const uint32_t a0 = a_base + st * SA, b0 = b_base + st * SB;
 #pragma unroll
           for (int kk = 0; kk < GEMM_CHUNK_BYTES / 32; ++kk) {
-            tc_mma<TF32>(d_tmem, smem_desc(a0 + 32u * kk), smem_desc(b0 + 32u * kk), IDESC,
-                         (uu > u || kk > 0) ? 1u : 0u);
+            const uint32_t acc = (uu > u || kk > 0) ? 1u : 0u;
+            if constexpr (NSPLIT == 2) {
+              // small cross terms first, then the leading product
+              tc_mma<TF32>(d_tmem, smem_desc(a0 + A_BYTES + 32u * kk), smem_desc(b0 + 32u * kk),
+                           IDESC, acc);
+              tc_mma<TF32>(d_tmem, smem_desc(a0 + 32u * kk), smem_desc(b0 + B_BYTES + 32u * kk),
+                           IDESC, 1u);
+              tc_mma<TF32>(d_tmem, smem_desc(a0 + 32u * kk), smem_desc(b0 + 32u * kk), IDESC, 1u);
+            } else {
+              tc_mma<TF32>(d_tmem, smem_desc(a0 + 32u * kk), smem_desc(b0 + 32u * kk), IDESC, acc);
+            }
           }
           tc_commit(empty_bar(st));
         }
@@ -300,13 +325,14 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
-static int stages_for(int ncols) {
-  const int stage = GEMM_BM * GEMM_CHUNK_BYTES + ncols * GEMM_CHUNK_BYTES;
+static int stages_for(int ncols, int nsplit) {
+  const int stage = nsplit * (GEMM_BM * GEMM_CHUNK_BYTES + ncols * GEMM_CHUNK_BYTES);
   int st = (GEMM_SMEM_BUDGET - 1024 - 256) / stage;
   return std::min(st, 16);
 }
-static size_t smem_bytes(int ncols, int stages) {
-  return 1024 + (size_t)stages * (GEMM_BM + ncols) * GEMM_CHUNK_BYTES + 8 * (2 * stages + 5) + 16;
+static size_t smem_bytes(int ncols, int stages, int nsplit) {
+  return 1024 + (size_t)stages * nsplit * (GEMM_BM + ncols) * GEMM_CHUNK_BYTES +
+         8 * (2 * stages + 5) + 16;
 }
 
 int gemm_table_ints(int n_out, int k, bool f32, int grid_cap) {
@@ -380,15 +406,17 @@ int make_tmap(CUtensorMap* map, const void* base, bool f32, uint64_t rows, uint6
   return r == CUDA_SUCCESS ? 0 : -3;
 }
 
-template <bool TF32, int NC>
-static cudaError_t launch_t(const CUtensorMap& tmW, const CUtensorMap& tmX, float* part,
+template <int MODE, int NC>
+static cudaError_t launch_t(const CUtensorMap& tmW, const CUtensorMap& tmWlo,
+                            const CUtensorMap& tmX, const CUtensorMap& tmXlo, float* part,
                             const GemmShape& s, const int* run_flag, int* err,
                             cudaStream_t stream, bool pdl) {
-  const int stages = stages_for(NC);
-  const size_t smem = smem_bytes(NC, stages);
+  const int nsplit = MODE == 2 ? 2 : 1;
+  const int stages = stages_for(NC, nsplit);
+  const size_t smem = smem_bytes(NC, stages, nsplit);
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(k_gemm<TF32, NC>,
+    cudaError_t e = cudaFuncSetAttribute(k_gemm<MODE, NC>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     attr_set = true;
@@ -403,16 +431,18 @@ static cudaError_t launch_t(const CUtensorMap& tmW, const CUtensorMap& tmX, floa
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, k_gemm<TF32, NC>, tmW, tmX, part, s, stages, run_flag, err);
+  return cudaLaunchKernelEx(&cfg, k_gemm<MODE, NC>, tmW, tmWlo, tmX, tmXlo, part, s, stages,
+                            run_flag, err);
 }
 
-cudaError_t gemm_launch(const CUtensorMap& tmW, const CUtensorMap& tmX, float* part,
-                        const GemmShape& s, int ncols, bool f32, const int* run_flag, int* err,
-                        cudaStream_t stream, bool pdl) {
-#define LT_GEMM_CASE(N)                                                                    \
-  case N:                                                                                  \
-    return f32 ? launch_t<true, N>(tmW, tmX, part, s, run_flag, err, stream, pdl)           \
-               : launch_t<false, N>(tmW, tmX, part, s, run_flag, err, stream, pdl);
+cudaError_t gemm_launch(const CUtensorMap& tmW, const CUtensorMap& tmWlo, const CUtensorMap& tmX,
+                        const CUtensorMap& tmXlo, float* part, const GemmShape& s, int ncols,
+                        int mode, const int* run_flag, int* err, cudaStream_t stream, bool pdl) {
+#define LT_GEMM_CASE(N)                                                                      \
+  case N:                                                                                    \
+    return mode == 2   ? launch_t<2, N>(tmW, tmWlo, tmX, tmXlo, part, s, run_flag, err, stream, pdl) \
+           : mode == 1 ? launch_t<1, N>(tmW, tmWlo, tmX, tmXlo, part, s, run_flag, err, stream, pdl) \
+                       : launch_t<0, N>(tmW, tmWlo, tmX, tmXlo, part, s, run_flag, err, stream, pdl);
   switch (ncols) {
     LT_GEMM_CASE(8)
     LT_GEMM_CASE(16)
@@ -422,6 +452,23 @@ cudaError_t gemm_launch(const CUtensorMap& tmW, const CUtensorMap& tmX, float* p
       return cudaErrorInvalidValue;
   }
 #undef LT_GEMM_CASE
+}
+
+__global__ void k_split_tf32(const float* __restrict__ src, float* __restrict__ hi,
+                             float* __restrict__ lo, size_t n) {
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n;
+       i += (size_t)gridDim.x * blockDim.x) {
+    const float v = src[i];
+    const float h = __uint_as_float(__float_as_uint(v) & 0xFFFFE000u);
+    hi[i] = h;
+    lo[i] = v - h;
+  }
+}
+
+cudaError_t split_tf32(const float* src, float* hi, float* lo, size_t n, cudaStream_t stream) {
+  const int blocks = (int)std::min<size_t>((n + 255) / 256, 4096);
+  k_split_tf32<<<blocks, 256, 0, stream>>>(src, hi, lo, n);
+  return cudaGetLastError();
 }
 
 }  // namespace lt

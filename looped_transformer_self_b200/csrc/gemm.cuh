@@ -22,7 +22,8 @@
 //    (tcgen05.ld) as an fp32 partial.  The consumer kernel adds a tile's
 //    partials in CTA order (fixed order: deterministic).  The partition depends
 //    only on (n_out, K, #SMs), never on the active row count.
-//  * bf16 operands: kind::f16 with fp32 accumulate; fp32 operands: kind::tf32.
+//  * bf16 operands: kind::f16 with fp32 accumulate; fp32 operands: kind::tf32,
+//    either one pass or split hi + lo (three MMAs per k-step, fp32-grade).
 //  * K tails and n_out tails are zero-filled by TMA.
 //  * every mbarrier wait is bounded (~1 s); on timeout the kernel records
 //    DEV_TIMEOUT, lets in-flight copies and MMAs land, frees TMEM and returns.
@@ -47,11 +48,16 @@ int gemm_table_ints(int n_out, int k, bool f32, int grid_cap);  // 2*tiles + gri
 int make_tmap(CUtensorMap* map, const void* base, bool f32, uint64_t rows, uint64_t k,
               uint32_t box_rows);
 
-// Launches the GEMM.  ncols in {8, 16, 32, 64}.  run_flag (device, may be null):
-// skip when *run_flag == 0.  pdl: launch with programmatic stream serialization.
-cudaError_t gemm_launch(const CUtensorMap& tmW, const CUtensorMap& tmX, float* part,
-                        const GemmShape& s, int ncols, bool f32, const int* run_flag,
-                        int* err, cudaStream_t stream, bool pdl);
+// Launches the GEMM.  ncols in {8, 16, 32, 64}.  mode: 0 bf16, 1 tf32, 2 fp32 as
+// split tf32 (tmWlo / tmXlo map the low parts; ignored otherwise).  run_flag
+// (device, may be null): skip when *run_flag == 0.  pdl: launch with
+// programmatic stream serialization.
+cudaError_t gemm_launch(const CUtensorMap& tmW, const CUtensorMap& tmWlo, const CUtensorMap& tmX,
+                        const CUtensorMap& tmXlo, float* part, const GemmShape& s, int ncols,
+                        int mode, const int* run_flag, int* err, cudaStream_t stream, bool pdl);
+
+// hi = src with the low 13 mantissa bits cleared (exact in tf32), lo = src - hi.
+cudaError_t split_tf32(const float* src, float* hi, float* lo, size_t n, cudaStream_t stream);
 
 size_t gemm_part_bytes(const GemmShape& s, int ncols);
 

@@ -1,0 +1,380 @@
+// Per-layer kernels of the batched mixed-depth pass (CUDA cores, HBM/L2-bound).
+//
+// One decode step runs every shared-block layer once over all active rows;
+// each row sits at its own loop depth and reads/writes only the KV cache of
+// that depth ("LoopSpec", liuzhao09.github.io/papers/loopspec.html, section
+// 2.1 and Fig. 2: shared weights, but states and KV of different depths are
+// never mixed).  Layer (a reading; the pages give only Eq. 1): pre-norm,
+// RMSNorm -> QKV -> RoPE -> causal attention -> O (+ s * residual) -> RMSNorm ->
+// SwiGLU MLP (+ s * residual).
+//
+// Row bookkeeping arrays (length C = table capacity = GEMM columns):
+//   mask[i]     row takes part in this pass (else its columns are zero and its
+//               hidden state and caches are untouched)
+//   r_pos[i]    position of the row's token; r_slot[i] its KV slot
+//   tag[i]      cache plane of the row within the layer (loop depth - 1 for
+//               shared-block layers, readout index for coda layers, 0 for prelude)
+//   slot of position j < r_pos[i]:  j < r_blen[i] ? lists[r_boff[i] + j]
+//                                   : chain[i * W + j % W]
+// KV pool: kv[((plane * S + slot) * 2 + {0: K, 1: V}) * d + feature].
+#pragma once
+
+#include "common.cuh"
+
+namespace lt {
+
+constexpr int ATT_CH = 256;       // positions per attention split (fixed: batch invariant)
+constexpr int EPI_THREADS = 256;
+
+// Writes a GEMM operand element.  bf16: rounded.  fp32 with lo != 0: the value
+// is stored as a tf32 pair, hi (low 13 mantissa bits cleared) at X[i] and the
+// exact remainder at X[lo + i], for the split-tf32 tensor-core GEMM.
+template <typename T>
+__device__ __forceinline__ void store_act(T* X, size_t i, float v, size_t lo);
+template <>
+__device__ __forceinline__ void store_act<__nv_bfloat16>(__nv_bfloat16* X, size_t i, float v,
+                                                         size_t) {
+  X[i] = __float2bfloat16_rn(v);
+}
+template <>
+__device__ __forceinline__ void store_act<float>(float* X, size_t i, float v, size_t lo) {
+  if (lo) {
+    const float h = __uint_as_float(__float_as_uint(v) & 0xFFFFE000u);
+    X[i] = h;
+    X[lo + i] = v - h;
+  } else {
+    X[i] = v;
+  }
+}
+
+template <typename T>
+__device__ __forceinline__ size_t kv_off(int plane, int slot, int which, int S, int d) {
+  return (((size_t)plane * S + slot) * 2 + which) * (size_t)d;
+}
+
+// ---- embedding: H^(0) of new rows (prelude P starts from the token's embedding)
+template <typename T>
+__global__ void k_embed(const T* __restrict__ E, const int* __restrict__ tok,
+                        const int* __restrict__ mask, int d, int V, float* __restrict__ h,
+                        int* err) {
+  pdl_wait();
+  pdl_trigger();
+  const int i = blockIdx.x;
+  if (!mask[i]) return;
+  const int t = tok[i];
+  if (t < 0 || t >= V) {
+    if (threadIdx.x == 0) set_err(err, DEV_BAD_INDEX);
+    return;
+  }
+  for (int n = threadIdx.x; n < d; n += blockDim.x)
+    h[(size_t)i * d + n] = to_f<T>(E[(size_t)t * d + n]);
+}
+
+// ---- X = RMSNorm(h) * g for masked rows, zeros elsewhere ----------------------
+template <typename T>
+__global__ void k_stage_norm(const float* __restrict__ h, const int* __restrict__ mask,
+                             const T* __restrict__ g, float eps, int d, T* __restrict__ X,
+                             size_t lo) {
+  __shared__ float red[33];
+  pdl_wait();
+  pdl_trigger();
+  const int i = blockIdx.x;
+  const float* hr = h + (size_t)i * d;
+  T* xr = X + (size_t)i * d;
+  if (!mask[i]) {
+    for (int n = threadIdx.x; n < d; n += blockDim.x) store_act<T>(xr, n, 0.f, lo);
+    return;
+  }
+  float ss = 0.f;
+  for (int n = threadIdx.x; n < d; n += blockDim.x) ss += hr[n] * hr[n];
+  ss = block_sum(ss, red);
+  const float inv = rsqrtf(ss / d + eps);
+  for (int n = threadIdx.x; n < d; n += blockDim.x)
+    store_act<T>(xr, n, hr[n] * inv * to_f<T>(g[n]), lo);
+}
+
+template <typename T>
+__global__ void k_copy_rows(const float* __restrict__ src, const int* __restrict__ mask, int d,
+                            float* __restrict__ dst) {
+  pdl_wait();
+  pdl_trigger();
+  const int i = blockIdx.x;
+  if (!mask[i]) return;
+  for (int n = threadIdx.x; n < d; n += blockDim.x) dst[(size_t)i * d + n] = src[(size_t)i * d + n];
+}
+
+// ---- QKV epilogue: reduce partials, RoPE(q, k), scatter K/V to the row's plane --
+template <typename T>
+__global__ void k_qkv_epi(const float* __restrict__ part, const GemmShape s, int C,
+                          const int* __restrict__ mask, const int* __restrict__ r_pos,
+                          const int* __restrict__ r_slot, const int* __restrict__ tagsrc,
+                          int tag_off, int plane_base, int S, int d, int hd,
+                          const float2* __restrict__ rope, T* __restrict__ kv,
+                          float* __restrict__ q, int* err) {
+  pdl_wait();
+  pdl_trigger();
+  const int i = blockIdx.x;
+  if (!mask[i]) return;
+  const int pos = r_pos[i], slot = r_slot[i];
+  const int tag = (tagsrc ? tagsrc[i] : 0) + tag_off;
+  if (slot < 0 || slot >= S) {
+    if (threadIdx.x == 0) set_err(err, DEV_BAD_INDEX);
+    return;
+  }
+  const int plane = plane_base + tag;
+  T* krow = kv + kv_off<T>(plane, slot, 0, S, d);
+  T* vrow = kv + kv_off<T>(plane, slot, 1, S, d);
+  const int half = hd / 2;
+  for (int p = threadIdx.x; p < d / 2; p += blockDim.x) {
+    const int head = p / half, e = p - head * half;
+    const int n1 = head * hd + e, n2 = n1 + half;
+    const float2 cs = rope[(size_t)pos * half + e];
+    const float q1 = sk_reduce(part, s, C, i, n1), q2 = sk_reduce(part, s, C, i, n2);
+    q[(size_t)i * d + n1] = q1 * cs.x - q2 * cs.y;
+    q[(size_t)i * d + n2] = q2 * cs.x + q1 * cs.y;
+    const float k1 = sk_reduce(part, s, C, i, d + n1), k2 = sk_reduce(part, s, C, i, d + n2);
+    krow[n1] = from_f<T>(k1 * cs.x - k2 * cs.y);
+    krow[n2] = from_f<T>(k2 * cs.x + k1 * cs.y);
+  }
+  for (int n = threadIdx.x; n < d; n += blockDim.x)
+    vrow[n] = from_f<T>(sk_reduce(part, s, C, i, 2 * d + n));
+}
+
+// ---- vector loads of EPL consecutive cache elements ------------------------------
+template <typename T, int EPL>
+__device__ __forceinline__ void load_vec(const T* __restrict__ p, float* out) {
+  constexpr int BYTES = EPL * (int)sizeof(T);
+  if constexpr (sizeof(T) == 2) {
+    if constexpr (BYTES % 16 == 0) {
+#pragma unroll
+      for (int c = 0; c < BYTES / 16; ++c) {
+        uint4 u = __ldg(reinterpret_cast<const uint4*>(p) + c);
+        const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          float2 f = __bfloat1622float2(b[j]);
+          out[c * 8 + 2 * j] = f.x;
+          out[c * 8 + 2 * j + 1] = f.y;
+        }
+      }
+    } else {
+#pragma unroll
+      for (int c = 0; c < BYTES / 4; ++c) {
+        uint32_t u = __ldg(reinterpret_cast<const unsigned int*>(p) + c);
+        float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u));
+        out[2 * c] = f.x;
+        out[2 * c + 1] = f.y;
+      }
+    }
+  } else {
+    if constexpr (BYTES % 16 == 0) {
+#pragma unroll
+      for (int c = 0; c < BYTES / 16; ++c) {
+        float4 f = __ldg(reinterpret_cast<const float4*>(p) + c);
+        out[4 * c] = f.x;
+        out[4 * c + 1] = f.y;
+        out[4 * c + 2] = f.z;
+        out[4 * c + 3] = f.w;
+      }
+    } else {
+#pragma unroll
+      for (int c = 0; c < BYTES / 8; ++c) {
+        float2 f = __ldg(reinterpret_cast<const float2*>(p) + c);
+        out[2 * c] = f.x;
+        out[2 * c + 1] = f.y;
+      }
+    }
+  }
+}
+
+// ---- paged, per-depth, branch-aware decode attention ------------------------------
+// Block (row i, head h, split sp) covers positions [sp*CH, min(sp*CH+CH, pos+1)) of
+// the row's own prefix (committed slots, then the ancestors' and its own slot),
+// all read from the row's depth plane.  16 lanes share one cache row (HD/16
+// elements each, vector loads); 8 half-warps work on different positions.
+// Output per split: (running max m, sum l, unnormalised acc[HD]).
+template <typename T, int HD>
+__global__ void __launch_bounds__(128) k_attn(
+    const float* __restrict__ q, const T* __restrict__ kv, int plane_base,
+    const int* __restrict__ tagsrc, int tag_off, int S, int d, int H,
+    const int* __restrict__ mask, const int* __restrict__ r_pos, const int* __restrict__ r_blen,
+    const int* __restrict__ r_boff, const int* __restrict__ lists, const int* __restrict__ chain,
+    int W, int max_splits, float* __restrict__ opart, int* err) {
+  constexpr int EPL = HD / 16;
+  __shared__ float qs[HD];
+  __shared__ float sc[ATT_CH];
+  __shared__ int sl[ATT_CH];
+  __shared__ float red[33];
+  __shared__ float accs[8][HD];
+  pdl_wait();
+  pdl_trigger();
+  const int i = blockIdx.x, h = blockIdx.y, sp = blockIdx.z;
+  if (!mask[i]) return;
+  const int n = r_pos[i] + 1;
+  const int start = sp * ATT_CH;
+  if (start >= n) return;
+  const int cnt = min(ATT_CH, n - start);
+  const int plane = plane_base + (tagsrc ? tagsrc[i] : 0) + tag_off;
+  const float scale = rsqrtf((float)HD);
+  for (int e = threadIdx.x; e < HD; e += blockDim.x) qs[e] = q[(size_t)i * d + h * HD + e] * scale;
+  const int blen = r_blen[i], boff = r_boff[i];
+  for (int t = threadIdx.x; t < cnt; t += blockDim.x) {
+    const int j = start + t;
+    int s = j < blen ? lists[boff + j] : chain[i * W + (j % W)];
+    if (s < 0 || s >= S) {
+      set_err(err, DEV_BAD_INDEX);
+      s = 0;
+    }
+    sl[t] = s;
+  }
+  __syncthreads();
+  const int hw = threadIdx.x >> 4, l16 = threadIdx.x & 15;
+  const size_t head_off = (size_t)h * HD + l16 * EPL;
+  float qv[EPL];
+#pragma unroll
+  for (int e = 0; e < EPL; ++e) qv[e] = qs[l16 * EPL + e];
+  // scores (both half-warps of a warp run the same trip count: the shuffles
+  // below need the whole warp)
+  for (int tb = hw & ~1; tb < cnt; tb += 8) {
+    const int t = tb + (hw & 1);
+    const bool ok = t < cnt;
+    float kvv[EPL];
+    if (ok) {
+      load_vec<T, EPL>(kv + kv_off<T>(plane, sl[t], 0, S, d) + head_off, kvv);
+    } else {
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) kvv[e] = 0.f;
+    }
+    float dot = 0.f;
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) dot += qv[e] * kvv[e];
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+    if (ok && l16 == 0) sc[t] = dot;
+  }
+  __syncthreads();
+  float mx = -INFINITY;
+  for (int t = threadIdx.x; t < cnt; t += blockDim.x) mx = fmaxf(mx, sc[t]);
+  mx = block_max(mx, red);
+  float ls = 0.f;
+  for (int t = threadIdx.x; t < cnt; t += blockDim.x) {
+    const float w = __expf(sc[t] - mx);
+    sc[t] = w;
+    ls += w;
+  }
+  ls = block_sum(ls, red);  // contains __syncthreads: sc[] is complete below
+  float acc[EPL];
+#pragma unroll
+  for (int e = 0; e < EPL; ++e) acc[e] = 0.f;
+  for (int t = hw; t < cnt; t += 8) {
+    float vv[EPL];
+    load_vec<T, EPL>(kv + kv_off<T>(plane, sl[t], 1, S, d) + head_off, vv);
+    const float w = sc[t];
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) acc[e] += w * vv[e];
+  }
+#pragma unroll
+  for (int e = 0; e < EPL; ++e) accs[hw][l16 * EPL + e] = acc[e];
+  __syncthreads();
+  float* out = opart + ((size_t)(i * H + h) * max_splits + sp) * (HD + 2);
+  for (int e = threadIdx.x; e < HD; e += blockDim.x) {
+    float a = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) a += accs[w][e];
+    out[2 + e] = a;
+  }
+  if (threadIdx.x == 0) {
+    out[0] = mx;
+    out[1] = ls;
+  }
+}
+
+// Combine the splits of (row, head) in split order and write the O-GEMM input row.
+template <typename T, int HD>
+__global__ void k_attn_combine(const float* __restrict__ opart, const int* __restrict__ mask,
+                               const int* __restrict__ r_pos, int H, int max_splits, int d,
+                               T* __restrict__ X, size_t lo) {
+  pdl_wait();
+  pdl_trigger();
+  const int i = blockIdx.x, h = blockIdx.y;
+  T* xr = X + (size_t)i * d + h * HD;
+  if (!mask[i]) {
+    for (int e = threadIdx.x; e < HD; e += blockDim.x) store_act<T>(xr, e, 0.f, lo);
+    return;
+  }
+  const int ns = (r_pos[i] + 1 + ATT_CH - 1) / ATT_CH;
+  const float* base = opart + (size_t)(i * H + h) * max_splits * (HD + 2);
+  float M = -INFINITY;
+  for (int s = 0; s < ns; ++s) M = fmaxf(M, base[(size_t)s * (HD + 2)]);
+  float L = 0.f;
+  for (int s = 0; s < ns; ++s) L += base[(size_t)s * (HD + 2) + 1] * __expf(base[(size_t)s * (HD + 2)] - M);
+  for (int e = threadIdx.x; e < HD; e += blockDim.x) {
+    float o = 0.f;
+    for (int s = 0; s < ns; ++s)
+      o += base[(size_t)s * (HD + 2) + 2 + e] * __expf(base[(size_t)s * (HD + 2)] - M);
+    store_act<T>(xr, e, o / L, lo);
+  }
+}
+
+// ---- residual epilogue: h += scale * (X W^T); optional next RMSNorm -> X ----------
+template <typename T>
+__global__ void k_resid_epi(const float* __restrict__ part, const GemmShape s, int C,
+                            const int* __restrict__ mask, float* __restrict__ h, float scale,
+                            const T* __restrict__ g_next, float eps, int d,
+                            T* __restrict__ X, size_t lo) {
+  __shared__ float red[33];
+  pdl_wait();
+  pdl_trigger();
+  const int i = blockIdx.x;
+  T* xr = X + (size_t)i * d;
+  if (!mask[i]) {
+    if (g_next)
+      for (int n = threadIdx.x; n < d; n += blockDim.x) store_act<T>(xr, n, 0.f, lo);
+    return;
+  }
+  float* hr = h + (size_t)i * d;
+  float ss = 0.f;
+  for (int n = threadIdx.x; n < d; n += blockDim.x) {
+    const float v = hr[n] + scale * sk_reduce(part, s, C, i, n);
+    hr[n] = v;
+    ss += v * v;
+  }
+  if (!g_next) return;
+  ss = block_sum(ss, red);
+  const float inv = rsqrtf(ss / d + eps);
+  for (int n = threadIdx.x; n < d; n += blockDim.x)
+    store_act<T>(xr, n, hr[n] * inv * to_f<T>(g_next[n]), lo);
+}
+
+// ---- SwiGLU epilogue: X = SiLU(gate) * up ------------------------------------------
+template <typename T>
+__global__ void k_gu_epi(const float* __restrict__ part, const GemmShape s, int C,
+                         const int* __restrict__ mask, int f, T* __restrict__ X, size_t lo) {
+  pdl_wait();
+  pdl_trigger();
+  const int i = blockIdx.x;
+  T* xr = X + (size_t)i * f;
+  const bool on = mask[i] != 0;
+  for (int n = blockIdx.y * blockDim.x + threadIdx.x; n < f; n += gridDim.y * blockDim.x) {
+    float a = 0.f;
+    if (on) {
+      const float g = sk_reduce(part, s, C, i, n), u = sk_reduce(part, s, C, i, f + n);
+      a = g / (1.f + __expf(-g)) * u;
+    }
+    store_act<T>(xr, n, a, lo);
+  }
+}
+
+// ---- RoPE table: (cos, sin) of pos * theta^(-2e/hd), computed in double ------------
+__global__ void k_rope_table(float2* __restrict__ rope, int max_pos, int hd, double theta) {
+  const int half = hd / 2;
+  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= max_pos * half) return;
+  const int pos = idx / half, e = idx - pos * half;
+  const double inv = pow(theta, -2.0 * e / hd);
+  double sn, cs;
+  sincos((double)pos * inv, &sn, &cs);
+  rope[idx] = make_float2((float)cs, (float)sn);
+}
+
+}  // namespace lt

@@ -85,6 +85,7 @@ class Stats:
     gate_opens: int = 0
     branches_created: int = 0
     resid_fallback: int = 0
+    table_peak: int = 0  # most branches alive at once (children exist before the same step's prune)
 
     def gamma(self, d1: int, d2: int, R: int) -> float:
         """Mean acceptance length, Eq. 9 (section 3.2)."""
@@ -102,6 +103,28 @@ class DecodeResult:
     stats: Stats
     trace: List[List[Tuple[int, int, int, int]]]  # per step: (uid, slot, pos, depth) sorted by uid
     logits: Dict[Tuple[int, int], np.ndarray]  # optional readout logits keyed (pos, depth)
+    step_margin: List[float] = dataclasses.field(default_factory=list)
+    # per step: smallest top-1 minus top-2 probability (softmax at T = 1) over
+    # the readouts whose argmax or draw that step's decisions used
+    step_gap: List[float] = dataclasses.field(default_factory=list)
+    # per step: smallest (z_top1 - z_top2) / max|z| over the same readouts
+
+
+def top2_gap(z: np.ndarray) -> float:
+    """(z_top1 - z_top2) / max|z|: how far a readout's argmax is from a tie,
+    relative to the logits' scale."""
+    z = np.asarray(z, np.float64)
+    a = np.partition(z, -2)[-2:]
+    return float((a[1] - a[0]) / np.max(np.abs(z)))
+
+
+def top2_margin(z: np.ndarray) -> float:
+    """p(top1) - p(top2) of softmax(z) at T = 1 (the greedy-margin reading)."""
+    z = np.asarray(z, np.float64)
+    p = np.exp(z - z.max())
+    p /= p.sum()
+    a = np.partition(p, -2)[-2:]
+    return float(a[1] - a[0])
 
 
 # ----------------------------------------------------------------------------
@@ -236,6 +259,8 @@ class SpecDecoder:
         self.src: List[int] = []
         self.cstep: List[int] = []
         self.trace: List[List[Tuple[int, int, int, int]]] = []
+        self.step_margin: List[float] = []
+        self.step_gap: List[float] = []
         root = self._new_branch(-1, P, x1, {})
         self.cslots.append(root.slot)
 
@@ -253,6 +278,7 @@ class SpecDecoder:
         self.next_uid += 1
         self.branches[b.uid] = b
         self.stats.branches_created += 1
+        self.stats.table_peak = max(self.stats.table_peak, len(self.branches))
         return b
 
     def slots_of(self, b: Branch) -> List[int]:
@@ -296,6 +322,7 @@ class SpecDecoder:
             self.trace.append([(u, self.branches[u].slot, self.branches[u].pos,
                                 self.branches[u].depth) for u in order])
         # 3. readouts
+        margin = gap = float("inf")
         for u in order:
             b = self.branches[u]
             b.p = None
@@ -303,7 +330,11 @@ class SpecDecoder:
                 z = rows.readout(b.state, b.depth, self.prefix_of(b), b.pos, self.slots_of(b))
                 if self.keep_logits:
                     self.logits[(b.pos, b.depth)] = z
+                margin = min(margin, top2_margin(z))
+                gap = min(gap, top2_gap(z))
                 b.p = S.process(z, self.T, self.top_p)
+        self.step_margin.append(margin)
+        self.step_gap.append(gap)
         # 4. proposals
         for u in order:
             b = self.branches[u]
@@ -376,7 +407,8 @@ class SpecDecoder:
         while not self.done():
             self.step()
         return DecodeResult(self.committed[self.P:], self.src, self.cstep, self.cslots,
-                            self.stats, self.trace, self.logits)
+                            self.stats, self.trace, self.logits, self.step_margin,
+                            self.step_gap)
 
 
 def decode_spec(rows, prompt, R, d1, d2, max_new, temperature, top_p, seed, n_slots,

@@ -1,0 +1,178 @@
+"""GPU parity of the decoder (through the C ABI) against the CPU oracle.
+
+Tiny looped LM (fp32 weights; tf32 tensor-core operands): prefill readout
+logits at every position and every readout depth, greedy full-depth AR and
+pipelined speculative decoding (tokens, commit sources and steps, per-step
+branch rows with slots), sampled decoding, and GPU speculative == GPU AR.
+
+Tolerances: logits are compared in relative L-inf (max |z_gpu - z_oracle| /
+max |z_oracle|).  For bf16 models the bound is 2e-2 (bf16 operands).  The
+tiny fp32 model runs its GEMMs as split tf32 on the tensor cores (hi*hi +
+hi*lo + lo*hi, ~2^-21 relative per product) with fp32 everywhere else, so its
+bound is 1e-4 (fp32 arithmetic through ~12 layer applications, with margin).
+
+Integer work (branch rows, slots, commit sources and steps) must be bit-exact
+up to the first step whose decisions rest on a readout whose oracle argmax is
+within the logit error bound of a tie: relative gap (z1 - z2) / max|z| <=
+2 * tolerance.  Beyond that step both choices are correct and the runs may
+legitimately diverge.
+"""
+import numpy as np
+import pytest
+
+import synthetic as syn
+
+pytestmark = pytest.mark.gpu
+
+TOL_F32 = 1e-4
+
+
+def _rel_linf(a, b):
+    return float(np.max(np.abs(np.asarray(a, np.float64) - b)) / np.max(np.abs(b)))
+
+
+@pytest.fixture(scope="module")
+def tiny():
+    cfg = syn.MODELS["tiny"]
+    return cfg, syn.make_weights(cfg), syn.prompt_for("tiny")
+
+
+@pytest.fixture(scope="module")
+def oracle_greedy(tiny):
+    from oracle import decode as D
+    from oracle.model import LoopedModel
+    cfg, w, prompt = tiny
+    dec = syn.DECODES["tiny_greedy"]
+    ar = D.decode_ar(D.OracleRows(LoopedModel(cfg, w, 256)), prompt, cfg.R, dec.max_new, 0.0, 1.0,
+                     dec.seed, keep_logits=True)
+    sp = D.decode_spec(D.OracleRows(LoopedModel(cfg, w, 256)), prompt, cfg.R, dec.d1, dec.d2,
+                       dec.max_new, 0.0, 1.0, dec.seed, 256, keep_logits=True)
+    return ar, sp
+
+
+def _decoder(cfg, dec, w, **kw):
+    from looped_transformer_self_b200.binding import Decoder
+    kw.setdefault("max_branches", 8)
+    kw.setdefault("max_ctx", 160)
+    kw.setdefault("trace_steps", 512)
+    return Decoder(cfg, dec, w, **kw)
+
+
+def test_tiny_prefill_logits_match_oracle(tiny):
+    from oracle import decode as D
+    from oracle.model import LoopedModel
+    cfg, w, prompt = tiny
+    dec = syn.DECODES["tiny_greedy"]
+    g = _decoder(cfg, dec, w)
+    first, am, lg = g.prefill(prompt, argmax=True, logits=True)
+    tags = [2, 3, 4]
+    zs = D.prefill(D.OracleRows(LoopedModel(cfg, w, 64)), prompt, cfg.R, tags, keep_logits=True)
+    lg = lg.cpu().numpy()
+    worst = 0.0
+    for pos in range(len(prompt)):
+        for t, r in enumerate(tags):
+            worst = max(worst, _rel_linf(lg[pos, t], zs[(pos, r)]))
+            assert am[pos, t] == int(np.argmax(lg[pos, t]))
+    assert worst < TOL_F32, worst
+    assert first == int(np.argmax(zs[(len(prompt) - 1, 4)]))
+
+
+def _margin(z):
+    p = np.exp(z - z.max())
+    p /= p.sum()
+    s = np.sort(p)[::-1]
+    return s[0] - s[1]
+
+
+def test_tiny_greedy_ar_matches_oracle(tiny, oracle_greedy):
+    cfg, w, prompt = tiny
+    dec = syn.DECODES["tiny_greedy"]
+    ar, _ = oracle_greedy
+    g = _decoder(cfg, dec, w)
+    first, _, _ = g.prefill(prompt)
+    toks, st = g.generate(dec.max_new, ar=True)
+    gpu = [first] + toks
+    assert st["steps"] == dec.max_new * cfg.R
+    for k, (a, b) in enumerate(zip(gpu, ar.tokens)):
+        if a != b:  # allowed only where the oracle's top-1 / top-2 margin is tiny
+            pos = len(prompt) - 1 + k
+            assert _margin(ar.logits[(pos, cfg.R)]) <= 0.05, (k, a, b)
+            break
+
+
+def test_tiny_greedy_spec_equals_gpu_ar_and_oracle(tiny, oracle_greedy):
+    cfg, w, prompt = tiny
+    dec = syn.DECODES["tiny_greedy"]
+    ar_o, sp_o = oracle_greedy
+    g = _decoder(cfg, dec, w)
+    first, _, _ = g.prefill(prompt)
+    ar_toks, _ = g.generate(dec.max_new, ar=True)
+    first2, _, _ = g.prefill(prompt)
+    sp_toks, st = g.generate(dec.max_new, ar=False)
+    assert first2 == first
+    assert sp_toks == ar_toks  # bit-identical greedy: speculative == full-depth AR
+    n = dec.max_new
+    tok, src, step = g.read_log(n)
+    seq = [first] + sp_toks
+    k = next((i for i, (a, b) in enumerate(zip(seq, sp_o.tokens)) if a != b), None)
+    if k is not None:  # a committed token may differ only at a low full-depth margin
+        pos = len(prompt) - 1 + k
+        assert _margin(sp_o.logits[(pos, cfg.R)]) <= 0.05
+    check_integer_work(g, sp_o, st, src, step)
+
+
+def check_integer_work(g, sp_o, st, src, step):
+    """Branch rows, slots, commit sources and steps are bit-exact up to the
+    first step whose decisions rest on a near-tie readout (see the module
+    docstring); returns that step (None: the whole run was checked)."""
+    low = next((s for s, g_ in enumerate(sp_o.step_gap) if g_ <= 2 * TOL_F32), None)
+    upto = len(sp_o.step_margin) if low is None else low + 1  # steps 1..upto decided alike
+    tr = g.read_trace(min(st["steps"], upto))
+    assert tr == sp_o.trace[:len(tr)]
+    assert len(tr) == min(st["steps"], upto)
+    for k, (s_o, c_o) in enumerate(zip(sp_o.src, sp_o.commit_step)):
+        if c_o > upto:
+            break
+        assert (src[k], step[k]) == (s_o, c_o), k
+    if low is None:
+        assert st["steps"] == sp_o.stats.steps
+        assert st["rows_max"] == sp_o.stats.rows_max
+        assert st["gate_opens"] == sp_o.stats.gate_opens
+        assert g.read_committed()[1] == sp_o.committed_slots
+    return low
+
+
+@pytest.mark.parametrize("d1,d2", [(1, 2), (1, 0), (2, 0), (1, 3)])
+def test_tiny_greedy_spec_other_depths(tiny, d1, d2):
+    cfg, w, prompt = tiny
+    dec = syn.DECODES["tiny_greedy"].replace(d1=d1, d2=d2, max_new=40)
+    # the table must hold the transient peak: (1, 2, 4) forks up to 12 branches
+    g = _decoder(cfg, dec, w, max_branches=16 if (d1, d2) == (1, 2) else 8)
+    g.prefill(prompt)
+    ar_toks, _ = g.generate(dec.max_new, ar=True)
+    g.prefill(prompt)
+    sp_toks, st = g.generate(dec.max_new, ar=False)
+    assert sp_toks == ar_toks
+    assert st["n_first"] + st["n_second"] + st["n_fallback"] == dec.max_new
+
+
+def test_tiny_sampled_spec_matches_oracle(tiny):
+    from oracle import decode as D
+    from oracle.model import LoopedModel
+    cfg, w, prompt = tiny
+    dec = syn.DECODES["tiny_sample"]
+    n = 32
+    sp_o = D.decode_spec(D.OracleRows(LoopedModel(cfg, w, 256)), prompt, cfg.R, dec.d1, dec.d2, n,
+                         dec.temperature, dec.top_p, dec.seed, 256)
+    g = _decoder(cfg, dec, w)
+    first, _, _ = g.prefill(prompt)
+    toks, st = g.generate(n)
+    gpu = [first] + toks
+    same = next((i for i, (a, b) in enumerate(zip(gpu, sp_o.tokens)) if a != b), None)
+    # draws near a decision boundary may differ (fp32 vs fp64 probabilities);
+    # with these seeds none is expected
+    assert same is None, (same, gpu, sp_o.tokens)
+    _, src, step = g.read_log(n)
+    assert src == sp_o.src and step == sp_o.commit_step
+    assert g.read_trace(st["steps"]) == sp_o.trace
+    assert st["gate_opens"] == sp_o.stats.gate_opens

@@ -2,8 +2,9 @@
 
 Reference: the same bf16 (or fp32) operand values multiplied in fp64 on the
 CPU.  bf16 operands are exact in both, so the only difference is the fp32
-accumulation order: |err| <= ~K * 2^-24 * sum|x_k w_k|.  tf32 operands keep 10
-mantissa bits: |err| <= ~2^-10 * sum|x_k w_k| per product term.
+accumulation order: |err| <= ~K * 2^-24 * sum|x_k w_k|.  fp32 operands run as
+split tf32 (hi*hi + hi*lo + lo*hi): each product is within ~2^-21 relative,
+so |err| <= ~(2^-20 + K * 2^-24) * sum|x_k w_k|.
 """
 import pytest
 import torch
@@ -38,14 +39,14 @@ def test_gemm_bf16_matches_fp64(n_out, k, ncols):
 
 
 @pytest.mark.parametrize("n_out,k", [(384, 128), (1152, 128), (512, 128), (128, 384), (300, 200)])
-def test_gemm_tf32_matches_fp64(n_out, k):
+def test_gemm_f32_split_tf32_matches_fp64(n_out, k):
     from looped_transformer_self_b200.binding import gemm_rows
     g = torch.Generator().manual_seed(n_out + k)
     w = (torch.randn(n_out, k, generator=g) / k ** 0.5).cuda()
     x = torch.randn(8, k, generator=g).cuda()
     y = gemm_rows(w, x).double().cpu()
     err = (y - _ref(w, x)).abs()
-    assert torch.all(err <= _bound(w, x, 2.0 ** -9)), float(err.max())
+    assert torch.all(err <= _bound(w, x, 2.0 ** -20 + 4 * k * 2.0 ** -24)), float(err.max())
 
 
 def test_gemm_rows_are_independent_and_deterministic():

@@ -53,6 +53,7 @@ def test_max_branches_with_unconditional_forking():
                             4096, keep_trace=False)
         assert res.stats.rows_max == mx
         assert res.stats.n_first == 60 + 0 and res.stats.gate_opens > 0
+        assert res.stats.table_peak >= mx
 
 
 @pytest.mark.parametrize("d1,d2", [(1, 0), (2, 0), (1, 2), (2, 3)])
