@@ -20,6 +20,10 @@ __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
                : "memory");
 }
+// Adds expected transaction bytes to the current phase without arriving.
+__device__ __forceinline__ void mbar_expect_tx_only(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.expect_tx.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
@@ -153,11 +157,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   constexpr int TCOLS = tmem_cols<NC>();
   constexpr uint32_t IDESC = instr_desc<TF32, NC>();
 
-  pdl_wait();
-  if (run_flag != nullptr && *run_flag == 0) return;
   const int c = blockIdx.x;
   const int u0 = sk_u0(c, s.units, s.grid), u1 = sk_u0(c + 1, s.units, s.grid);
-  if (u0 >= u1) return;
+  if (u0 >= u1) {
+    pdl_wait();
+    return;
+  }
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -208,28 +213,63 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0) {
+  // Weights do not depend on earlier kernels: the first `npre` stages of
+  // weight tiles are requested before waiting on the preceding grid, so with
+  // programmatic dependent launch this CTA's prologue and pipeline fill overlap
+  // the kernels in front of it.  Their barriers get the weight bytes now
+  // (expect_tx without arrival) and the activation bytes plus the arrival once
+  // the activations may be read.
+  const int npre = min(stages, u1 - u0);
+  const uint64_t pol_w = policy_evict_first(), pol_x = policy_evict_last();
+  if (warp == 0 && lane == 0) {
+    for (int g = 0; g < npre; ++g) {
+      const int uu = u0 + g, t = uu / s.kch;
+      const int kx = (uu - t * s.kch) * BKE;
+      mbar_expect_tx_only(full_bar(g), SA);
+      tma_load_2d(a_base + g * SA, &tmW, kx, t * GEMM_BM, full_bar(g), pol_w);
+      if constexpr (NSPLIT == 2)
+        tma_load_2d(a_base + g * SA + A_BYTES, &tmWlo, kx, t * GEMM_BM, full_bar(g), pol_w);
+    }
+  }
+  pdl_wait();
+  const bool skip = run_flag != nullptr && *run_flag == 0;
+  if (skip) {
+    if (warp == 0 && lane == 0) {
+      // let the prefetched weight tiles land before the CTA goes away
+      volatile int dummy = 0;
+      for (int g = 0; g < npre; ++g) {
+        mbar_arrive(full_bar(g));
+        mbar_wait(full_bar(g), 0, &dummy);
+      }
+    }
+  } else if (warp == 0) {
     if (lane == 0) {
       // ---------------- TMA producer ----------------
-      const uint64_t pol_w = policy_evict_first(), pol_x = policy_evict_last();
       int g = 0;
       for (int u = u0; u < u1 && !*abort_flag;) {
         const int t = u / s.kch;
         const int seg_end = min(u1, (t + 1) * s.kch);
         for (int uu = u; uu < seg_end; ++uu, ++g) {
           const int st = g % stages, n = g / stages;
-          if (!mbar_wait(empty_bar(st), (n & 1) ^ 1, abort_flag)) break;
-          mbar_expect_tx(full_bar(st), SA + SB);
           const int kx = (uu - t * s.kch) * BKE;
-          tma_load_2d(a_base + st * SA, &tmW, kx, t * GEMM_BM, full_bar(st), pol_w);
-          tma_load_2d(b_base + st * SB, &tmX, kx, 0, full_bar(st), pol_x);
-          if constexpr (NSPLIT == 2) {
-            tma_load_2d(a_base + st * SA + A_BYTES, &tmWlo, kx, t * GEMM_BM, full_bar(st), pol_w);
-            tma_load_2d(b_base + st * SB + B_BYTES, &tmXlo, kx, 0, full_bar(st), pol_x);
+          if (g < npre) {  // weights already requested
+            mbar_expect_tx(full_bar(st), SB);
+          } else {
+            if (!mbar_wait(empty_bar(st), (n & 1) ^ 1, abort_flag)) break;
+            mbar_expect_tx(full_bar(st), SA + SB);
+            tma_load_2d(a_base + st * SA, &tmW, kx, t * GEMM_BM, full_bar(st), pol_w);
+            if constexpr (NSPLIT == 2)
+              tma_load_2d(a_base + st * SA + A_BYTES, &tmWlo, kx, t * GEMM_BM, full_bar(st),
+                          pol_w);
           }
+          tma_load_2d(b_base + st * SB, &tmX, kx, 0, full_bar(st), pol_x);
+          if constexpr (NSPLIT == 2)
+            tma_load_2d(b_base + st * SB + B_BYTES, &tmXlo, kx, 0, full_bar(st), pol_x);
         }
         u = seg_end;
       }
+      // on abort: arrive on prefetched stages never reached so their loads can land
+      for (int gg = g; gg < npre; ++gg) mbar_arrive(full_bar(gg));
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -279,7 +319,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       volatile int dummy = 0;
       mbar_wait(drain_bar, 0, &dummy);
     }
-  } else {
+  } else if (warp >= 2) {
     // ---------------- drain: TMEM -> fp32 partials ----------------
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     int seg = 0;

@@ -36,7 +36,10 @@ namespace lt {
 constexpr int GEMM_BM = 128;            // output features per tile (MMA M)
 constexpr int GEMM_CHUNK_BYTES = 128;   // K bytes per stage (one 128B-swizzle row)
 constexpr int GEMM_THREADS = 192;       // warp 0: TMA, warp 1: MMA, warps 2-5: drain
-constexpr int GEMM_SMEM_BUDGET = 200 * 1024;
+// Shared memory per CTA for the TMA ring: ~100 KB keeps >= 4 stages (>= 64 KB of
+// weight tiles in flight per SM, well above what HBM latency x bandwidth needs)
+// and lets the next GEMM's CTA become resident, and prefetch, while this one drains.
+constexpr int GEMM_SMEM_BUDGET = 104 * 1024;
 
 // Plans the stream-K split of one weight matrix.  `grid_cap`: CTAs (#SMs).
 // Fills the host copies of the reducer tables (tile_c [2*tiles], cta_t0 [grid]).
