@@ -202,6 +202,29 @@ int lt_gemm_scratch_bytes(int dtype, int n_out, int k, int ncols, size_t* bytes)
 int lt_gemm_rows(int dtype, const void* d_w, const void* d_x, float* d_y, int n_out, int k,
                  int ncols, void* d_scratch, size_t scratch_bytes, void* stream);
 
+/*
+ * Allocation-free variant of lt_gemm_rows, for callers that cannot allocate
+ * device memory (a graph or memory pool owns every allocation, a plug-in gets
+ * a stream but no allocator, or another framework has reserved the device).
+ * The paper has no counterpart: this is a deployment convenience.
+ *   - bf16 only (dtype must be LT_BF16; LT_F32 returns LT_ERR_ARG);
+ *   - its scratch (reduction tables + fp32 partials) is one static device
+ *     array of LT_NOALLOC_SCRATCH_BYTES inside the library, present on every
+ *     device that loads the library until the process exits; sizes whose
+ *     scratch would exceed it return LT_ERR_CAPACITY (e.g. n_out 49152 with
+ *     ncols 64);
+ *   - the first call on a device resolves the array's device address, so make
+ *     that first call before any stream capture;
+ *   - every call shares the array: calls that overlap on the GPU (other
+ *     streams, other threads) race; serialise them.  Nothing in the array needs
+ *     clearing between calls;
+ *   - it calls no cudaMalloc / cudaFree and no allocating library routine.
+ * Arguments and result as lt_gemm_rows; synchronises `stream` before return.
+ */
+#define LT_NOALLOC_SCRATCH_BYTES (8u << 20)
+int lt_gemm_rows_noalloc(int dtype, const void* d_w, const void* d_x, float* d_y, int n_out,
+                         int k, int ncols, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

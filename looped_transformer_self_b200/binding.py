@@ -91,6 +91,7 @@ _ip = ctypes.POINTER(ctypes.c_int32)
 def _declare(L):
     L.lt_gemm_scratch_bytes.argtypes = [_i, _i, _i, _i, ctypes.POINTER(_sz)]
     L.lt_gemm_rows.argtypes = [_i, _vp, _vp, _vp, _i, _i, _i, _vp, _sz, _vp]
+    L.lt_gemm_rows_noalloc.argtypes = [_i, _vp, _vp, _vp, _i, _i, _i, _vp]
     L.lt_workspace_bytes.argtypes = [ctypes.POINTER(ModelConfigC), ctypes.POINTER(DecodeConfigC),
                                      ctypes.POINTER(_sz)]
     L.lt_create.argtypes = [ctypes.POINTER(ModelConfigC), ctypes.POINTER(DecodeConfigC), _vp, _sz,
@@ -141,6 +142,18 @@ def gemm_rows(w: torch.Tensor, x: torch.Tensor, scratch: torch.Tensor = None,
     y = torch.empty(ncols, n_out, dtype=torch.float32, device=w.device)
     check(lib().lt_gemm_rows(dtype, _ptr(w), _ptr(x), _ptr(y), n_out, k, ncols, _ptr(scratch),
                              scratch.numel(), _stream(stream)), "lt_gemm_rows")
+    return y
+
+
+def gemm_rows_noalloc(w: torch.Tensor, x: torch.Tensor, stream=None) -> torch.Tensor:
+    """Y[i][n] = sum_k x[i][k] w[n][k] through lt_gemm_rows_noalloc: bf16 only,
+    scratch in the library's static device array (no allocation by the call)."""
+    assert w.is_cuda and x.is_cuda and w.dtype == x.dtype == torch.bfloat16
+    n_out, k = w.shape
+    ncols = x.shape[0]
+    y = torch.empty(ncols, n_out, dtype=torch.float32, device=w.device)
+    check(lib().lt_gemm_rows_noalloc(LT_BF16, _ptr(w), _ptr(x), _ptr(y), n_out, k, ncols,
+                                     _stream(stream)), "lt_gemm_rows_noalloc")
     return y
 
 
