@@ -262,7 +262,7 @@ def run_ours(args):
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu:
-        cpu = oracle_sample(cfg, dec_g, prompt, weights)
+        cpu = oracle_sample(cfg, dec_g, prompt, weights, n_prompt=8, n_tokens=24)
 
     if rank == 0:
         n_steps = stats["steps"]

@@ -132,6 +132,23 @@ int lt_generate(lt_handle* h, int ar_mode, int n, int32_t* h_out, lt_stats* st);
 /* One batched pass.  *n_committed = 1 and *h_tok = the token when this pass
  * committed one, else 0. */
 int lt_decode_step(lt_handle* h, int ar_mode, int32_t* h_tok, int* n_committed);
+/*
+ * Explicit edits of the branch tree between two decode steps (after
+ * lt_decode_step; the next step sees the edited tree).  The pages' own
+ * commits and rollbacks happen inside each step on the device (section 2.2:
+ * accept keeps the child's subtree, reject prunes every descendant of the
+ * wrong prefix); these calls expose the same two operations to callers that
+ * decide acceptance themselves (e.g. externally proposed continuations).
+ *   lt_rollback_branch: prune branch `uid` (not the root) and its descendants,
+ *     freeing their KV slots; its parent forgets the child.
+ *   lt_commit_branch: commit the token of `uid`, which must be a child of the
+ *     root, WITHOUT full-depth verification (logged with source 3); every
+ *     branch outside its subtree is pruned and it becomes the root.
+ * Errors: LT_ERR_ARG for an unknown uid, the root, or (commit) a non-child;
+ * LT_ERR_STATE when no decode is in progress.
+ */
+int lt_rollback_branch(lt_handle* h, int32_t uid);
+int lt_commit_branch(lt_handle* h, int32_t uid);
 /* Commit log of the last generate / decode calls: token, source (1 first
  * proposal, 2 second, 0 drawn at full depth) and 1-based step of each commit. */
 int lt_read_log(lt_handle* h, int32_t* h_tok, int32_t* h_src, int32_t* h_step, int n);

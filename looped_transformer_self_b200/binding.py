@@ -105,6 +105,8 @@ def _declare(L):
     L.lt_read_committed.argtypes = [_vp, _ip, _ip, ctypes.POINTER(_i)]
     L.lt_read_branch_table.argtypes = [_vp, _ip]
     L.lt_read_readouts.argtypes = [_vp, _vp, _vp, _ip, _ip]
+    L.lt_rollback_branch.argtypes = [_vp, ctypes.c_int32]
+    L.lt_commit_branch.argtypes = [_vp, ctypes.c_int32]
     L.lt_profile_steps.argtypes = [_vp, _i, _i, ctypes.POINTER(ProfileC)]
     L.lt_get_info.argtypes = [_vp, ctypes.POINTER(InfoC)]
     L.lt_reset.argtypes = [_vp]
@@ -257,6 +259,12 @@ class Decoder:
         self._check(lib().lt_decode_step(self.h, 1 if ar else 0, _i32p(tok), ctypes.byref(n)),
                     "lt_decode_step")
         return int(tok[0]) if n.value else None
+
+    def rollback_branch(self, uid):
+        self._check(lib().lt_rollback_branch(self.h, uid), "lt_rollback_branch")
+
+    def commit_branch(self, uid):
+        self._check(lib().lt_commit_branch(self.h, uid), "lt_commit_branch")
 
     def read_log(self, n):
         np = self.np

@@ -145,16 +145,27 @@ struct GemmShape {
 };
 
 // Sum of the partials of output feature n for row i (fixed CTA order).
-// Partial layout: part[((c * jmax + j) * ncols + i) * 128 + (n % 128)].
+// Partial layout: part[((c * jmax + j) * ncols + i) * 128 + (n % 128)].  The first
+// 8 partials are issued as independent loads (they live in L2), so a reduction
+// costs about one L2 round trip instead of one per partial.
 __device__ __forceinline__ float sk_reduce(const float* __restrict__ part, const GemmShape& s,
                                            int ncols, int i, int n) {
+  constexpr int PB = 8;
   const int t = n >> 7, r = n & 127;
   const int c_lo = __ldg(s.tile_c + 2 * t), c_hi = __ldg(s.tile_c + 2 * t + 1);
-  float acc = 0.f;
-  for (int c = c_lo; c <= c_hi; ++c) {
-    const int j = t - __ldg(s.cta_t0 + c);
-    acc += part[(((size_t)c * s.jmax + j) * ncols + i) * 128 + r];
+  float v[PB];
+#pragma unroll
+  for (int k = 0; k < PB; ++k) {
+    const int c = c_lo + k;
+    v[k] = c <= c_hi
+               ? __ldcg(part + (((size_t)c * s.jmax + (t - __ldg(s.cta_t0 + c))) * ncols + i) * 128 + r)
+               : 0.f;
   }
+  float acc = 0.f;
+#pragma unroll
+  for (int k = 0; k < PB; ++k) acc += v[k];
+  for (int c = c_lo + PB; c <= c_hi; ++c)
+    acc += __ldcg(part + (((size_t)c * s.jmax + (t - __ldg(s.cta_t0 + c))) * ncols + i) * 128 + r);
   return acc;
 }
 

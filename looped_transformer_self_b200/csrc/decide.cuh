@@ -182,12 +182,24 @@ __global__ void __launch_bounds__(1024)
   float* p = P + (size_t)i * V;
   float best = -INFINITY;
   int bi = 0x7fffffff;
-  for (int j = threadIdx.x; j < V; j += blockDim.x) {
-    const float v = sk_reduce(part, s, C, i, j);
-    z[j] = v;
-    if (better_max(v, j, best, bi)) {
-      best = v;
-      bi = j;
+  // four elements per round so their partial loads overlap
+  for (int j0 = threadIdx.x; j0 < V; j0 += 4 * blockDim.x) {
+    float v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int j = j0 + u * blockDim.x;
+      v[u] = j < V ? sk_reduce(part, s, C, i, j) : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int j = j0 + u * blockDim.x;
+      if (j < V) {
+        z[j] = v[u];
+        if (better_max(v[u], j, best, bi)) {
+          best = v[u];
+          bi = j;
+        }
+      }
     }
   }
   const int a = block_arg<false>(best, bi, sk, si);
@@ -502,8 +514,60 @@ __device__ int bk_find_uid(const BookSmem& b, int C, int uid) {
   return -1;
 }
 
-__device__ void bk_logic(BookSmem& b, const Dev& D, Ctl& c, int mode) {
+// Is entry k in the subtree of entry r (r itself included)?  A descendant holds
+// r's slot at r's position in its chain.
+__device__ __forceinline__ bool bk_in_subtree(const BookSmem& b, int k, int r) {
+  return k == r || (b.pos[k] > b.pos[r] && b.chain[k * WIN + (b.pos[r] % WIN)] == b.slot[r]);
+}
+
+__device__ void bk_logic(BookSmem& b, const Dev& D, Ctl& c, int mode, int arg) {
   const int C = D.C;
+  if (mode == 2 || mode == 3) {
+    // explicit edits between steps: 2 = roll back branch `arg` (uid) with its
+    // subtree; 3 = commit child `arg` of the root without verification
+    const int e = bk_find_uid(b, C, arg);
+    int root = -1;
+    for (int k = 0; k < C; ++k)
+      if (b.alive[k] && b.pos[k] == c.L - 1) root = k;
+    if (e < 0 || root < 0 || e == root || (mode == 3 && b.parent[e] != b.uid[root])) {
+      set_err(&c.err, DEV_STATE);
+      return;
+    }
+    if (mode == 2) {
+      const int par = bk_find_uid(b, C, b.parent[e]);
+      for (int k = 0; k < C; ++k)
+        if (b.alive[k] && k != e && bk_in_subtree(b, k, e)) {
+          b.alive[k] = 0;
+          bk_free_slot(b, b.slot[k]);
+        }
+      b.alive[e] = 0;
+      bk_free_slot(b, b.slot[e]);
+      if (par >= 0) {
+        if (b.c1[par] == arg) b.c1[par] = -1;
+        if (b.c2[par] == arg) b.c2[par] = -1;
+      }
+      return;
+    }
+    if (c.L >= D.max_ctx) {
+      set_err(&c.err, DEV_NO_ROOT);
+      return;
+    }
+    D.committed[c.L] = b.tok[e];
+    D.log_tok[c.n_commit] = b.tok[e];
+    D.log_src[c.n_commit] = 3;
+    D.log_step[c.n_commit] = c.steps;
+    c.n_commit++;
+    c.L++;
+    for (int k = 0; k < C; ++k) {
+      if (!b.alive[k] || bk_in_subtree(b, k, e)) continue;
+      b.alive[k] = 0;
+      if (k != root) bk_free_slot(b, b.slot[k]);
+    }
+    b.parent[e] = -1;
+    D.lists[c.L - 1] = b.slot[e];
+    if (c.L >= c.target_len) c.finished = 1;
+    return;
+  }
   if (mode == 0 && c.prepared) {
     c.prepared = 0;
     c.steps++;
@@ -559,10 +623,7 @@ __device__ void bk_logic(BookSmem& b, const Dev& D, Ctl& c, int mode) {
       const int surv = bk_find_uid(b, C, src == 1 ? b.c1[root] : src == 2 ? b.c2[root] : -1);
       for (int k = 0; k < C; ++k) {
         if (!b.alive[k]) continue;
-        bool keep = false;
-        if (surv >= 0)
-          keep = k == surv || (b.pos[k] > b.pos[surv] &&
-                               b.chain[k * WIN + (b.pos[surv] % WIN)] == b.slot[surv]);
+        const bool keep = surv >= 0 && bk_in_subtree(b, k, surv);
         if (!keep) {
           b.alive[k] = 0;
           if (k != root) bk_free_slot(b, b.slot[k]);
@@ -601,7 +662,7 @@ __device__ void bk_logic(BookSmem& b, const Dev& D, Ctl& c, int mode) {
   }
 }
 
-__global__ void __launch_bounds__(256) k_book(Dev D, int mode) {
+__global__ void __launch_bounds__(256) k_book(Dev D, int mode, int arg) {
   __shared__ BookSmem b;
   pdl_wait();
   pdl_trigger();
@@ -627,7 +688,7 @@ __global__ void __launch_bounds__(256) k_book(Dev D, int mode) {
   if (threadIdx.x == 0) c = *cg;
   __syncthreads();
   if (threadIdx.x == 0) {
-    if (!c.err) bk_logic(b, D, c, mode);
+    if (!c.err) bk_logic(b, D, c, mode, arg);
     if (c.err) c.finished = 1;
     // rebuild the rows of the prepared step
     int rows = 0, any_new = 0, any_ro = 0;

@@ -45,6 +45,7 @@ struct Handle {
   size_t ws_bytes = 0;
   Dev D;
   float *h = nullptr, *hc = nullptr, *q = nullptr, *attn_part = nullptr, *part = nullptr;
+  int* attn_cnt = nullptr;  // per (row, head) split-arrival counters (kept at zero between uses)
   void *Xd = nullptr, *Xo = nullptr, *Xf = nullptr, *kv = nullptr;
   float2* rope = nullptr;
   int* gemm_tab = nullptr;
@@ -199,6 +200,7 @@ static size_t carve(Handle* H, char* base) {
   H->hc = cv.take<float>((size_t)C * d);
   H->q = cv.take<float>((size_t)C * d);
   H->attn_part = cv.take<float>((size_t)C * m.n_heads * H->max_splits * (m.head_dim + 2));
+  H->attn_cnt = cv.take<int>((size_t)C * m.n_heads);
   const int planes_x = H->f32 ? 2 : 1;  // fp32: hi and lo tf32 planes
   H->Xd = cv.take<char>((size_t)planes_x * C * d * esz);
   H->Xo = cv.take<char>((size_t)planes_x * C * d * esz);
@@ -290,25 +292,25 @@ static cudaError_t gemm(Handle* H, const CUtensorMap& tw, const CUtensorMap& twl
 
 template <typename T, int HD>
 static cudaError_t attention(Handle* H, int gl, const int* tagsrc, int tag_off, const int* mask,
-                             T* Xo) {
+                             T* Xo, bool fused) {
   ProfScope ps(H, 2, 0.0);
   Dev& D = H->D;
   const int C = H->C, Hn = H->m.n_heads;
-  LT_CK(launch(H->use_pdl, k_attn<T, HD>, dim3(C, Hn, H->max_splits), dim3(128), H->stream,
-               (const float*)H->q, (const T*)H->kv, H->plane_base[gl], tagsrc, tag_off, H->S,
-               H->m.d_model, Hn, mask, (const int*)D.r_pos, (const int*)D.r_blen,
-               (const int*)D.r_boff, (const int*)D.lists, (const int*)D.b_chain, (int)WIN,
-               H->max_splits, H->attn_part, &D.ctl->err));
-  return launch(H->use_pdl, k_attn_combine<T, HD>, dim3(C, Hn), dim3(HD), H->stream,
-                (const float*)H->attn_part, mask, (const int*)D.r_pos, Hn, H->max_splits,
-                H->m.d_model, Xo, H->lo_d);
+  auto kern = fused ? k_attn<T, HD, true> : k_attn<T, HD, false>;
+  return launch(H->use_pdl, kern, dim3(C, Hn, H->max_splits), dim3(128), H->stream,
+                (const float*)H->q, (T*)H->kv, H->plane_base[gl], tagsrc, tag_off, H->S,
+                H->m.d_model, Hn, mask, (const int*)D.r_pos, (const int*)D.r_blen,
+                (const int*)D.r_boff, (const int*)D.lists, (const int*)D.b_chain, (int)WIN,
+                H->max_splits, H->attn_part, H->attn_cnt, Xo, H->lo_d, (const float*)H->part,
+                H->sh_qkv, C, (const int*)D.r_slot, (const float2*)H->rope, &D.ctl->err);
 }
 
 // kind: 0 prelude (one cache), 1 shared block (cache of the row's depth), 2 coda
 // (cache of the row's readout depth).
+// fused: decode pass (the QKV epilogue runs inside attention, see k_attn).
 template <typename T>
 static cudaError_t run_layers(Handle* H, int gl0, int n, int kind, const int* mask, float* hbuf,
-                              float scale, const int* flag) {
+                              float scale, const int* flag, bool fused) {
   Dev& D = H->D;
   const lt_model_config& m = H->m;
   const int C = H->C, d = m.d_model;
@@ -324,15 +326,16 @@ static cudaError_t run_layers(Handle* H, int gl0, int n, int kind, const int* ma
       LT_CK(launch(H->use_pdl, k_stage_norm<T>, dim3(C), dim3(EPI_THREADS), H->stream,
                    (const float*)hbuf, mask, (const T*)L.g1, m.rms_eps, d, Xd, H->lo_d));
     LT_CK(gemm<T>(H, L.tm_qkv, L.tm_qkv_lo, H->tm_Xd, H->tm_Xd_lo, H->sh_qkv, flag));
-    LT_CK(launch(H->use_pdl, k_qkv_epi<T>, dim3(C), dim3(EPI_THREADS), H->stream,
-                 (const float*)H->part, H->sh_qkv, C, mask, (const int*)D.r_pos,
-                 (const int*)D.r_slot, tagsrc, tag_off, H->plane_base[gl], H->S, d, m.head_dim,
-                 (const float2*)H->rope, (T*)H->kv, H->q, &D.ctl->err));
+    if (!fused)
+      LT_CK(launch(H->use_pdl, k_qkv_epi<T>, dim3(C), dim3(EPI_THREADS), H->stream,
+                   (const float*)H->part, H->sh_qkv, C, mask, (const int*)D.r_pos,
+                   (const int*)D.r_slot, tagsrc, tag_off, H->plane_base[gl], H->S, d, m.head_dim,
+                   (const float2*)H->rope, (T*)H->kv, H->q, &D.ctl->err));
     switch (m.head_dim) {
-      case 32: LT_CK((attention<T, 32>(H, gl, tagsrc, tag_off, mask, Xo))); break;
-      case 64: LT_CK((attention<T, 64>(H, gl, tagsrc, tag_off, mask, Xo))); break;
-      case 96: LT_CK((attention<T, 96>(H, gl, tagsrc, tag_off, mask, Xo))); break;
-      default: LT_CK((attention<T, 128>(H, gl, tagsrc, tag_off, mask, Xo))); break;
+      case 32: LT_CK((attention<T, 32>(H, gl, tagsrc, tag_off, mask, Xo, fused))); break;
+      case 64: LT_CK((attention<T, 64>(H, gl, tagsrc, tag_off, mask, Xo, fused))); break;
+      case 96: LT_CK((attention<T, 96>(H, gl, tagsrc, tag_off, mask, Xo, fused))); break;
+      default: LT_CK((attention<T, 128>(H, gl, tagsrc, tag_off, mask, Xo, fused))); break;
     }
     LT_CK(gemm<T>(H, L.tm_o, L.tm_o_lo, H->tm_Xo, H->tm_Xo_lo, H->sh_o, flag));
     LT_CK(launch(H->use_pdl, k_resid_epi<T>, dim3(C), dim3(EPI_THREADS), H->stream,
@@ -353,7 +356,7 @@ static cudaError_t run_layers(Handle* H, int gl0, int n, int kind, const int* ma
 // Readout C of the rows in D.m_ro: coda layers on a copy of the state, final
 // norm, LM head, processing.
 template <typename T>
-static cudaError_t run_readout(Handle* H, const int* flag) {
+static cudaError_t run_readout(Handle* H, const int* flag, bool fused) {
   Dev& D = H->D;
   const lt_model_config& m = H->m;
   const int C = H->C, d = m.d_model;
@@ -361,7 +364,7 @@ static cudaError_t run_readout(Handle* H, const int* flag) {
   if (m.n_coda > 0) {
     LT_CK(launch(H->use_pdl, k_copy_rows<T>, dim3(C), dim3(EPI_THREADS), H->stream,
                  (const float*)H->h, (const int*)D.m_ro, d, H->hc));
-    LT_CK(run_layers<T>(H, m.n_prelude + m.n_core, m.n_coda, 2, D.m_ro, H->hc, 1.f, flag));
+    LT_CK(run_layers<T>(H, m.n_prelude + m.n_core, m.n_coda, 2, D.m_ro, H->hc, 1.f, flag, fused));
     src = H->hc;
   }
   LT_CK(launch(H->use_pdl, k_stage_norm<T>, dim3(C), dim3(EPI_THREADS), H->stream,
@@ -383,14 +386,14 @@ static cudaError_t decode_step(Handle* H) {
                (const int*)D.r_tok, (const int*)D.m_new, m.d_model, m.vocab, H->h, &ctl->err));
   H->prof_cat = 1;
   if (m.n_prelude > 0)
-    LT_CK(run_layers<T>(H, 0, m.n_prelude, 0, D.m_new, H->h, 1.f, &ctl->flag_new));
+    LT_CK(run_layers<T>(H, 0, m.n_prelude, 0, D.m_new, H->h, 1.f, &ctl->flag_new, true));
   H->prof_cat = 0;
   LT_CK(run_layers<T>(H, m.n_prelude, m.n_core, 1, D.m_alive, H->h, m.resid_scale,
-                      &ctl->flag_run));
+                      &ctl->flag_run, true));
   H->prof_cat = 1;
-  LT_CK(run_readout<T>(H, &ctl->flag_ro));
+  LT_CK(run_readout<T>(H, &ctl->flag_ro, true));
   LT_CK(launch(H->use_pdl, k_decide, dim3(C), dim3(1024), H->stream, D));
-  return launch(H->use_pdl, k_book, dim3(1), dim3(256), H->stream, D, 0);
+  return launch(H->use_pdl, k_book, dim3(1), dim3(256), H->stream, D, 0, 0);
 }
 
 static cudaError_t step_once(Handle* H) {
@@ -507,6 +510,10 @@ extern "C" int lt_create(const lt_model_config* m, const lt_decode_config* dc, v
     delete hd;
     return LT_ERR_SHAPE;
   }
+  if (cudaMemsetAsync(H->attn_cnt, 0, (size_t)H->C * m->n_heads * 4, H->stream) != cudaSuccess) {
+    delete hd;
+    return LT_ERR_CUDA;
+  }
   const int half = m->head_dim / 2;
   k_rope_table<<<(H->max_pos * half + 255) / 256, 256, 0, H->stream>>>(H->rope, H->max_pos,
                                                                         m->head_dim, m->rope_theta);
@@ -609,18 +616,18 @@ static int prefill_t(lt_handle* hd, const int32_t* h_tokens, int n, int32_t* h_f
     if ((e = launch(false, k_embed<T>, dim3(C), dim3(EPI_THREADS), st, (const T*)H->embed,
                     (const int*)D.r_tok, (const int*)D.m_new, m.d_model, m.vocab, H->h, &D.ctl->err)))
       return cuda_fail(hd, e, "embed");
-    if (m.n_prelude > 0 && (e = run_layers<T>(H, 0, m.n_prelude, 0, D.m_alive, H->h, 1.f, nullptr)))
+    if (m.n_prelude > 0 && (e = run_layers<T>(H, 0, m.n_prelude, 0, D.m_alive, H->h, 1.f, nullptr, false)))
       return cuda_fail(hd, e, "prelude");
     for (int r = 1; r <= m.R; ++r) {
       const int tag = D.tag_of_depth[r];
       if ((e = launch(false, k_prefill_rows, dim3(1), dim3(64), st, D, c0p, cnt, n, r, tag)))
         return cuda_fail(hd, e, "rows");
-      if ((e = run_layers<T>(H, gl_core, m.n_core, 1, D.m_alive, H->h, m.resid_scale, nullptr)))
+      if ((e = run_layers<T>(H, gl_core, m.n_core, 1, D.m_alive, H->h, m.resid_scale, nullptr, false)))
         return cuda_fail(hd, e, "core");
       if (tag < 0) continue;
       const bool need_head = (last && r == m.R) || h_argmax || d_logits;
       if (need_head) {
-        if ((e = run_readout<T>(H, nullptr))) return cuda_fail(hd, e, "readout");
+        if ((e = run_readout<T>(H, nullptr, false))) return cuda_fail(hd, e, "readout");
         if (d_logits)
           for (int k = 0; k < cnt; ++k)
             if ((e = cudaMemcpyAsync(d_logits + ((size_t)(c0p + k) * dep_tags + tag) * m.vocab,
@@ -638,7 +645,7 @@ static int prefill_t(lt_handle* hd, const int32_t* h_tokens, int n, int32_t* h_f
         // coda caches of this readout depth are still needed by later positions
         if ((e = launch(false, k_copy_rows<T>, dim3(C), dim3(EPI_THREADS), st, (const float*)H->h,
                         (const int*)D.m_ro, m.d_model, H->hc)) ||
-            (e = run_layers<T>(H, m.n_prelude + m.n_core, m.n_coda, 2, D.m_ro, H->hc, 1.f, nullptr)))
+            (e = run_layers<T>(H, m.n_prelude + m.n_core, m.n_coda, 2, D.m_ro, H->hc, 1.f, nullptr, false)))
           return cuda_fail(hd, e, "coda");
       }
       if (last && r == m.R) {
@@ -727,7 +734,7 @@ static int begin(lt_handle* hd, int n, int ar) {
   Handle* H = &hd->h;
   cudaError_t e;
   if ((e = launch(false, k_begin, dim3(1), dim3(1), H->stream, H->D.ctl, n, ar)) ||
-      (e = launch(false, k_book, dim3(1), dim3(256), H->stream, H->D, 1)))
+      (e = launch(false, k_book, dim3(1), dim3(256), H->stream, H->D, 1, 0)))
     return cuda_fail(hd, e, "begin");
   H->begun = true;
   return LT_OK;
@@ -983,3 +990,35 @@ extern "C" int lt_get_info(lt_handle* hd, lt_info* out) {
   out->weight_bytes_head = esz * (double)m.vocab * m.d_model;
   return LT_OK;
 }
+
+// Explicit edits of the branch tree between steps (see the header).
+static int tree_edit(lt_handle* hd, int mode, int32_t uid) {
+  if (!hd) return LT_ERR_ARG;
+  Handle* H = &hd->h;
+  if (!H->prefilled || !H->begun) return fail(hd, LT_ERR_STATE, "no decode in progress");
+  std::vector<int> t(12 * H->C);
+  int rc = lt_read_branch_table(hd, t.data());
+  if (rc) return rc;
+  Ctl c;
+  if ((rc = read_ctl(hd, &c))) return rc;
+  const int C = H->C;
+  int e = -1, root = -1;
+  for (int k = 0; k < C; ++k) {
+    if (!t[k]) continue;
+    if (t[C + k] == uid) e = k;
+    if (t[4 * C + k] == c.L - 1) root = k;
+  }
+  if (e < 0) return fail(hd, LT_ERR_ARG, "no live branch with this uid");
+  if (e == root) return fail(hd, LT_ERR_ARG, "the root cannot be edited");
+  if (mode == 3 && (root < 0 || t[2 * C + e] != t[C + root]))
+    return fail(hd, LT_ERR_ARG, "only a child of the root can be committed");
+  if (c.finished) return fail(hd, LT_ERR_STATE, "decode finished");
+  cudaError_t er = launch(false, k_book, dim3(1), dim3(256), H->stream, H->D, mode, (int)uid);
+  if (er) return cuda_fail(hd, er, "tree edit");
+  if ((rc = read_ctl(hd, &c))) return rc;
+  if (c.finished) H->begun = false;
+  return LT_OK;
+}
+
+extern "C" int lt_rollback_branch(lt_handle* hd, int32_t uid) { return tree_edit(hd, 2, uid); }
+extern "C" int lt_commit_branch(lt_handle* hd, int32_t uid) { return tree_edit(hd, 3, uid); }

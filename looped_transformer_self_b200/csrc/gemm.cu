@@ -63,6 +63,13 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar), "l"(policy)
       : "memory");
 }
+// Pulls one weight tile into L2 (no shared memory, no barrier).
+__device__ __forceinline__ void tma_prefetch_l2(const CUtensorMap* map, int x, int y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(x), "r"(y)
+               : "memory");
+}
 __device__ __forceinline__ uint64_t policy_evict_first() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
@@ -230,8 +237,21 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       if constexpr (NSPLIT == 2)
         tma_load_2d(a_base + g * SA + A_BYTES, &tmWlo, kx, t * GEMM_BM, full_bar(g), pol_w);
     }
+    // The rest of this CTA's weight range (up to GEMM_L2_PREFETCH_BYTES) goes to
+    // L2 now, so HBM keeps streaming this GEMM's weights while the kernels in
+    // front of it finish; the ring then refills from L2.
+    const int nl2 = min(u1 - u0, npre + GEMM_L2_PREFETCH_BYTES / (int)SA);
+    for (int g = npre; g < nl2; ++g) {
+      const int uu = u0 + g, t = uu / s.kch;
+      const int kx = (uu - t * s.kch) * BKE;
+      tma_prefetch_l2(&tmW, kx, t * GEMM_BM);
+      if constexpr (NSPLIT == 2) tma_prefetch_l2(&tmWlo, kx, t * GEMM_BM);
+    }
   }
   pdl_wait();
+  // the next kernels may become resident (and a following GEMM may prefetch
+  // its weights) while this one streams
+  pdl_trigger();
   const bool skip = run_flag != nullptr && *run_flag == 0;
   if (skip) {
     if (warp == 0 && lane == 0) {
@@ -359,7 +379,6 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TCOLS)
                  : "memory");
   }
-  pdl_trigger();
 }
 
 // ---------------------------------------------------------------------------

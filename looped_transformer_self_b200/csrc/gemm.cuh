@@ -40,6 +40,9 @@ constexpr int GEMM_THREADS = 192;       // warp 0: TMA, warp 1: MMA, warps 2-5: 
 // weight tiles in flight per SM, well above what HBM latency x bandwidth needs)
 // and lets the next GEMM's CTA become resident, and prefetch, while this one drains.
 constexpr int GEMM_SMEM_BUDGET = 104 * 1024;
+// Weight bytes per CTA requested into L2 ahead of the ring (148 CTAs: ~37 MB,
+// so two GEMMs in flight stay well inside the 126 MB L2).
+constexpr int GEMM_L2_PREFETCH_BYTES = 256 * 1024;
 
 // Plans the stream-K split of one weight matrix.  `grid_cap`: CTAs (#SMs).
 // Fills the host copies of the reducer tables (tile_c [2*tiles], cta_t0 [grid]).

@@ -24,7 +24,7 @@
 namespace lt {
 
 constexpr int ATT_CH = 256;       // positions per attention split (fixed: batch invariant)
-constexpr int EPI_THREADS = 256;
+constexpr int EPI_THREADS = 1024;  // epilogues: many partial reductions in flight per row
 
 // Writes a GEMM operand element.  bf16: rounded.  fp32 with lo != 0: the value
 // is stored as a tf32 pair, hi (low 13 mantissa bits cleared) at X[i] and the
@@ -141,6 +141,8 @@ __global__ void k_qkv_epi(const float* __restrict__ part, const GemmShape s, int
 }
 
 // ---- vector loads of EPL consecutive cache elements ------------------------------
+// Loads go through L2 (ld.global.cg): a fused attention block may read back a
+// cache row it wrote itself, which the non-coherent read-only path would not see.
 template <typename T, int EPL>
 __device__ __forceinline__ void load_vec(const T* __restrict__ p, float* out) {
   constexpr int BYTES = EPL * (int)sizeof(T);
@@ -148,7 +150,7 @@ __device__ __forceinline__ void load_vec(const T* __restrict__ p, float* out) {
     if constexpr (BYTES % 16 == 0) {
 #pragma unroll
       for (int c = 0; c < BYTES / 16; ++c) {
-        uint4 u = __ldg(reinterpret_cast<const uint4*>(p) + c);
+        uint4 u = __ldcg(reinterpret_cast<const uint4*>(p) + c);
         const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&u);
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
@@ -160,7 +162,7 @@ __device__ __forceinline__ void load_vec(const T* __restrict__ p, float* out) {
     } else {
 #pragma unroll
       for (int c = 0; c < BYTES / 4; ++c) {
-        uint32_t u = __ldg(reinterpret_cast<const unsigned int*>(p) + c);
+        uint32_t u = __ldcg(reinterpret_cast<const unsigned int*>(p) + c);
         float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u));
         out[2 * c] = f.x;
         out[2 * c + 1] = f.y;
@@ -170,7 +172,7 @@ __device__ __forceinline__ void load_vec(const T* __restrict__ p, float* out) {
     if constexpr (BYTES % 16 == 0) {
 #pragma unroll
       for (int c = 0; c < BYTES / 16; ++c) {
-        float4 f = __ldg(reinterpret_cast<const float4*>(p) + c);
+        float4 f = __ldcg(reinterpret_cast<const float4*>(p) + c);
         out[4 * c] = f.x;
         out[4 * c + 1] = f.y;
         out[4 * c + 2] = f.z;
@@ -179,7 +181,7 @@ __device__ __forceinline__ void load_vec(const T* __restrict__ p, float* out) {
     } else {
 #pragma unroll
       for (int c = 0; c < BYTES / 8; ++c) {
-        float2 f = __ldg(reinterpret_cast<const float2*>(p) + c);
+        float2 f = __ldcg(reinterpret_cast<const float2*>(p) + c);
         out[2 * c] = f.x;
         out[2 * c + 1] = f.y;
       }
@@ -191,32 +193,53 @@ __device__ __forceinline__ void load_vec(const T* __restrict__ p, float* out) {
 // Block (row i, head h, split sp) covers positions [sp*CH, min(sp*CH+CH, pos+1)) of
 // the row's own prefix (committed slots, then the ancestors' and its own slot),
 // all read from the row's depth plane.  16 lanes share one cache row (HD/16
-// elements each, vector loads); 8 half-warps work on different positions.
-// Output per split: (running max m, sum l, unnormalised acc[HD]).
-template <typename T, int HD>
+// elements each, vector loads); each half-warp keeps ATT_U positions' K and V
+// loads in flight and folds them into an online softmax (one pass over the
+// cache).  The 8 half-warps merge in fixed order; the split's (max, sum,
+// unnormalised acc) goes to `opart`, and the last block of the (row, head) to
+// finish merges all splits in split order and writes the O-GEMM input row
+// (deterministic whichever block comes last).
+//
+// FUSED (decode passes): the block also performs the QKV epilogue for its head
+// -- q from the QKV GEMM partials with RoPE, and, in the block that holds the
+// row's own position, k (RoPE) and v written to the row's cache slot.  This is
+// valid because within one decode pass no row reads a cache row that another
+// row of the same pass writes: a row's ancestors sit at strictly greater depth
+// (planes differ) and siblings never hold each other's positions.  Prefill
+// rows of one chunk do read each other's rows, so prefill runs the separate
+// QKV epilogue first (FUSED = false) and reads q from `q`.
+constexpr int ATT_U = 4;
+
+template <typename T, int HD, bool FUSED>
 __global__ void __launch_bounds__(128) k_attn(
-    const float* __restrict__ q, const T* __restrict__ kv, int plane_base,
+    const float* __restrict__ q, T* __restrict__ kv, int plane_base,
     const int* __restrict__ tagsrc, int tag_off, int S, int d, int H,
     const int* __restrict__ mask, const int* __restrict__ r_pos, const int* __restrict__ r_blen,
     const int* __restrict__ r_boff, const int* __restrict__ lists, const int* __restrict__ chain,
-    int W, int max_splits, float* __restrict__ opart, int* err) {
+    int W, int max_splits, float* __restrict__ opart, int* __restrict__ counters,
+    T* __restrict__ X, size_t lo, const float* __restrict__ part, const GemmShape qs_shape, int C,
+    const int* __restrict__ r_slot, const float2* __restrict__ rope, int* err) {
   constexpr int EPL = HD / 16;
-  __shared__ float qs[HD];
-  __shared__ float sc[ATT_CH];
+  __shared__ float qsm[HD];
   __shared__ int sl[ATT_CH];
-  __shared__ float red[33];
-  __shared__ float accs[8][HD];
+  __shared__ float hm[8], hl[8];
+  __shared__ float hacc[8][HD];
+  __shared__ int last;
   pdl_wait();
   pdl_trigger();
   const int i = blockIdx.x, h = blockIdx.y, sp = blockIdx.z;
-  if (!mask[i]) return;
+  if (!mask[i]) {
+    if (sp == 0)
+      for (int e = threadIdx.x; e < HD; e += blockDim.x)
+        store_act<T>(X + (size_t)i * d + h * HD, e, 0.f, lo);
+    return;
+  }
   const int n = r_pos[i] + 1;
   const int start = sp * ATT_CH;
   if (start >= n) return;
+  const int ns = (n + ATT_CH - 1) / ATT_CH;
   const int cnt = min(ATT_CH, n - start);
   const int plane = plane_base + (tagsrc ? tagsrc[i] : 0) + tag_off;
-  const float scale = rsqrtf((float)HD);
-  for (int e = threadIdx.x; e < HD; e += blockDim.x) qs[e] = q[(size_t)i * d + h * HD + e] * scale;
   const int blen = r_blen[i], boff = r_boff[i];
   for (int t = threadIdx.x; t < cnt; t += blockDim.x) {
     const int j = start + t;
@@ -227,92 +250,144 @@ __global__ void __launch_bounds__(128) k_attn(
     }
     sl[t] = s;
   }
-  __syncthreads();
   const int hw = threadIdx.x >> 4, l16 = threadIdx.x & 15;
-  const size_t head_off = (size_t)h * HD + l16 * EPL;
+  const float scale = rsqrtf((float)HD);
   float qv[EPL];
-#pragma unroll
-  for (int e = 0; e < EPL; ++e) qv[e] = qs[l16 * EPL + e];
-  // scores (both half-warps of a warp run the same trip count: the shuffles
-  // below need the whole warp)
-  for (int tb = hw & ~1; tb < cnt; tb += 8) {
-    const int t = tb + (hw & 1);
-    const bool ok = t < cnt;
-    float kvv[EPL];
-    if (ok) {
-      load_vec<T, EPL>(kv + kv_off<T>(plane, sl[t], 0, S, d) + head_off, kvv);
-    } else {
-#pragma unroll
-      for (int e = 0; e < EPL; ++e) kvv[e] = 0.f;
+  if constexpr (FUSED) {
+    const int pos = n - 1, half = HD / 2;
+    const bool own = sp == ns - 1;  // this block holds the row's own position
+    const int slot = r_slot[i];
+    T* krow = kv + kv_off<T>(plane, slot, 0, S, d) + (size_t)h * HD;
+    T* vrow = kv + kv_off<T>(plane, slot, 1, S, d) + (size_t)h * HD;
+    for (int e = threadIdx.x; e < half; e += blockDim.x) {
+      const float2 cs = rope[(size_t)pos * half + e];
+      const int n1 = h * HD + e, n2 = n1 + half;
+      const float q1 = sk_reduce(part, qs_shape, C, i, n1), q2 = sk_reduce(part, qs_shape, C, i, n2);
+      qsm[e] = q1 * cs.x - q2 * cs.y;
+      qsm[e + half] = q2 * cs.x + q1 * cs.y;
+      if (own) {
+        const float k1 = sk_reduce(part, qs_shape, C, i, d + n1);
+        const float k2 = sk_reduce(part, qs_shape, C, i, d + n2);
+        krow[e] = from_f<T>(k1 * cs.x - k2 * cs.y);
+        krow[e + half] = from_f<T>(k2 * cs.x + k1 * cs.y);
+      }
     }
-    float dot = 0.f;
+    if (own)
+      for (int e = threadIdx.x; e < HD; e += blockDim.x)
+        vrow[e] = from_f<T>(sk_reduce(part, qs_shape, C, i, 2 * d + h * HD + e));
+    __syncthreads();  // the own cache row is complete and visible to this block
 #pragma unroll
-    for (int e = 0; e < EPL; ++e) dot += qv[e] * kvv[e];
+    for (int e = 0; e < EPL; ++e) qv[e] = qsm[l16 * EPL + e] * scale;
+  } else {
+    load_vec<float, EPL>(q + (size_t)i * d + h * HD + l16 * EPL, qv);
 #pragma unroll
-    for (int o = 8; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
-    if (ok && l16 == 0) sc[t] = dot;
+    for (int e = 0; e < EPL; ++e) qv[e] *= scale;
+    __syncthreads();
   }
-  __syncthreads();
-  float mx = -INFINITY;
-  for (int t = threadIdx.x; t < cnt; t += blockDim.x) mx = fmaxf(mx, sc[t]);
-  mx = block_max(mx, red);
-  float ls = 0.f;
-  for (int t = threadIdx.x; t < cnt; t += blockDim.x) {
-    const float w = __expf(sc[t] - mx);
-    sc[t] = w;
-    ls += w;
-  }
-  ls = block_sum(ls, red);  // contains __syncthreads: sc[] is complete below
-  float acc[EPL];
+  const size_t head_off = (size_t)h * HD + l16 * EPL;
+  const T* kbase = kv + kv_off<T>(plane, 0, 0, S, d) + head_off;
+  const T* vbase = kv + kv_off<T>(plane, 0, 1, S, d) + head_off;
+  const size_t slot_stride = (size_t)2 * d;
+  float m = -INFINITY, l = 0.f, acc[EPL];
 #pragma unroll
   for (int e = 0; e < EPL; ++e) acc[e] = 0.f;
-  for (int t = hw; t < cnt; t += 8) {
-    float vv[EPL];
-    load_vec<T, EPL>(kv + kv_off<T>(plane, sl[t], 1, S, d) + head_off, vv);
-    const float w = sc[t];
+  // both half-warps of a warp run the same trip count (the shuffles need the warp)
+  for (int tb = (hw & ~1) * ATT_U; tb < cnt; tb += 8 * ATT_U) {
+    const int t0 = tb + (hw & 1) * ATT_U;
+    float kx[ATT_U][EPL], vx[ATT_U][EPL];
 #pragma unroll
-    for (int e = 0; e < EPL; ++e) acc[e] += w * vv[e];
+    for (int u = 0; u < ATT_U; ++u) {
+      const int t = t0 + u;
+      if (t < cnt) {
+        const size_t off = (size_t)sl[t] * slot_stride;
+        load_vec<T, EPL>(kbase + off, kx[u]);
+        load_vec<T, EPL>(vbase + off, vx[u]);
+      } else {
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) kx[u][e] = vx[u][e] = 0.f;
+      }
+    }
+    float sc[ATT_U];
+#pragma unroll
+    for (int u = 0; u < ATT_U; ++u) {
+      float dot = 0.f;
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) dot += qv[e] * kx[u][e];
+      sc[u] = dot;
+    }
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1)
+#pragma unroll
+      for (int u = 0; u < ATT_U; ++u) sc[u] += __shfl_xor_sync(0xffffffffu, sc[u], o);
+    float mloc = -INFINITY;
+#pragma unroll
+    for (int u = 0; u < ATT_U; ++u)
+      if (t0 + u < cnt) mloc = fmaxf(mloc, sc[u]);
+    if (mloc == -INFINITY) continue;  // nothing valid for this half-warp (uniform per half)
+    const float mnew = fmaxf(m, mloc);
+    const float c = __expf(m - mnew);
+    l *= c;
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) acc[e] *= c;
+#pragma unroll
+    for (int u = 0; u < ATT_U; ++u) {
+      if (t0 + u < cnt) {
+        const float w = __expf(sc[u] - mnew);
+        l += w;
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) acc[e] += w * vx[u][e];
+      }
+    }
+    m = mnew;
+  }
+  if (l16 == 0) {
+    hm[hw] = m;
+    hl[hw] = l;
   }
 #pragma unroll
-  for (int e = 0; e < EPL; ++e) accs[hw][l16 * EPL + e] = acc[e];
+  for (int e = 0; e < EPL; ++e) hacc[hw][l16 * EPL + e] = acc[e];
   __syncthreads();
+  float M = -INFINITY;
+#pragma unroll
+  for (int w = 0; w < 8; ++w) M = fmaxf(M, hm[w]);
   float* out = opart + ((size_t)(i * H + h) * max_splits + sp) * (HD + 2);
   for (int e = threadIdx.x; e < HD; e += blockDim.x) {
     float a = 0.f;
 #pragma unroll
-    for (int w = 0; w < 8; ++w) a += accs[w][e];
+    for (int w = 0; w < 8; ++w)
+      if (hm[w] != -INFINITY) a += hacc[w][e] * __expf(hm[w] - M);
     out[2 + e] = a;
   }
   if (threadIdx.x == 0) {
-    out[0] = mx;
-    out[1] = ls;
+    float L = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w)
+      if (hm[w] != -INFINITY) L += hl[w] * __expf(hm[w] - M);
+    out[0] = M;
+    out[1] = L;
   }
-}
-
-// Combine the splits of (row, head) in split order and write the O-GEMM input row.
-template <typename T, int HD>
-__global__ void k_attn_combine(const float* __restrict__ opart, const int* __restrict__ mask,
-                               const int* __restrict__ r_pos, int H, int max_splits, int d,
-                               T* __restrict__ X, size_t lo) {
-  pdl_wait();
-  pdl_trigger();
-  const int i = blockIdx.x, h = blockIdx.y;
-  T* xr = X + (size_t)i * d + h * HD;
-  if (!mask[i]) {
-    for (int e = threadIdx.x; e < HD; e += blockDim.x) store_act<T>(xr, e, 0.f, lo);
-    return;
+  // the last split block of this (row, head) combines all splits in order
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const int ticket = atomicAdd(&counters[i * H + h], 1);
+    last = ticket == ns - 1;
+    if (last) counters[i * H + h] = 0;
   }
-  const int ns = (r_pos[i] + 1 + ATT_CH - 1) / ATT_CH;
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
   const float* base = opart + (size_t)(i * H + h) * max_splits * (HD + 2);
-  float M = -INFINITY;
-  for (int s = 0; s < ns; ++s) M = fmaxf(M, base[(size_t)s * (HD + 2)]);
-  float L = 0.f;
-  for (int s = 0; s < ns; ++s) L += base[(size_t)s * (HD + 2) + 1] * __expf(base[(size_t)s * (HD + 2)] - M);
+  float Mx = -INFINITY;
+  for (int s2 = 0; s2 < ns; ++s2) Mx = fmaxf(Mx, __ldcg(base + (size_t)s2 * (HD + 2)));
+  float Lx = 0.f;
+  for (int s2 = 0; s2 < ns; ++s2)
+    Lx += __ldcg(base + (size_t)s2 * (HD + 2) + 1) * __expf(__ldcg(base + (size_t)s2 * (HD + 2)) - Mx);
   for (int e = threadIdx.x; e < HD; e += blockDim.x) {
     float o = 0.f;
-    for (int s = 0; s < ns; ++s)
-      o += base[(size_t)s * (HD + 2) + 2 + e] * __expf(base[(size_t)s * (HD + 2)] - M);
-    store_act<T>(xr, e, o / L, lo);
+    for (int s2 = 0; s2 < ns; ++s2)
+      o += __ldcg(base + (size_t)s2 * (HD + 2) + 2 + e) * __expf(__ldcg(base + (size_t)s2 * (HD + 2)) - Mx);
+    store_act<T>(X + (size_t)i * d + h * HD, e, o / Lx, lo);
   }
 }
 

@@ -400,6 +400,51 @@ class SpecDecoder:
             nr = self._new_branch(-1, L - 1, x, {})
             self.cslots.append(nr.slot)
 
+    # -- explicit tree edits between steps ----------------------------------------
+    def _subtree(self, uid: int) -> List[int]:
+        out = []
+        for u in sorted(self.branches):
+            x = self.branches[u]
+            while x is not None and x.uid != uid:
+                x = self.branches.get(x.parent)
+            if x is not None:
+                out.append(u)
+        return out
+
+    def rollback(self, uid: int) -> None:
+        """Prune branch `uid` and all its descendants (not the root); their slots
+        are freed and the parent forgets the child."""
+        b = self.branches[uid]
+        assert uid != self.root().uid
+        for u in self._subtree(uid):
+            self.free.add(self.branches.pop(u).slot)
+        p = self.branches.get(b.parent)
+        if p is not None:
+            if p.child1 == uid:
+                p.child1 = -1
+            if p.child2 == uid:
+                p.child2 = -1
+
+    def commit_branch(self, uid: int) -> None:
+        """Commit a child of the root without full-depth verification (an
+        external acceptance, source 3): its token is appended, every branch
+        outside its subtree is pruned and it becomes the root."""
+        root = self.root()
+        b = self.branches[uid]
+        assert b.parent == root.uid
+        self.committed.append(b.token)
+        self.src.append(3)
+        self.cstep.append(self.stats.steps)
+        keep = set(self._subtree(uid))
+        for u in sorted(self.branches):
+            if u in keep:
+                continue
+            x = self.branches.pop(u)
+            if u != root.uid:
+                self.free.add(x.slot)
+        b.parent = -1
+        self.cslots.append(b.slot)
+
     def done(self) -> bool:
         return len(self.committed) >= self.P + 1 + self.max_new
 

@@ -176,3 +176,94 @@ def test_tiny_sampled_spec_matches_oracle(tiny):
     assert src == sp_o.src and step == sp_o.commit_step
     assert g.read_trace(st["steps"]) == sp_o.trace
     assert st["gate_opens"] == sp_o.stats.gate_opens
+
+
+# ---------------------------------------------------------------------------
+# shapes the tiny model does not reach
+# ---------------------------------------------------------------------------
+
+SMALL_BF16_128 = syn.ModelConfig("bf16_hd128", "bf16", 256, 2, 128, 512, 1000, 0, 3, 0, 4,
+                                 resid_scale=0.5, head_gain=4.0, seed=7)
+SMALL_BF16_96 = syn.ModelConfig("bf16_hd96", "bf16", 192, 2, 96, 384, 700, 1, 2, 1, 6,
+                                resid_scale=0.5, head_gain=4.0, seed=8)
+SMALL_F32_32 = syn.MODELS["tiny"]
+
+
+@pytest.mark.parametrize("cfg,tol,P", [(SMALL_F32_32, TOL_F32, 300),
+                                       (SMALL_BF16_128, 2e-2, 300),
+                                       (SMALL_BF16_96, 2e-2, 280)])
+def test_prefill_logits_multi_split_attention(cfg, tol, P):
+    """Prompts longer than one attention split (256 positions): every readout
+    logit row of the last positions matches the oracle; bf16 models within the
+    the benchmark spec's 2e-2, the fp32 model within 1e-4."""
+    from oracle import decode as D
+    from oracle.model import LoopedModel
+    w = syn.make_weights(cfg)
+    prompt = syn.uniform_prompt(P, cfg.vocab, seed=5)
+    dec = syn.DecodeConfig(1, 2, 0.0, 1.0, 2, 8)
+    tags = sorted({1, 2, cfg.R})
+    g = _decoder(cfg, dec, w, max_ctx=P + 16)
+    first, am, lg = g.prefill(prompt, argmax=True, logits=True)
+    lg = lg.cpu().numpy()
+    zs = D.prefill(D.OracleRows(LoopedModel(cfg, w, P + 4)), prompt, cfg.R, tags,
+                   keep_logits=True)
+    for pos in range(P - 6, P):
+        for t, r in enumerate(tags):
+            assert _rel_linf(lg[pos, t], zs[(pos, r)]) < tol, (pos, r)
+
+
+@pytest.mark.parametrize("cfg", [SMALL_BF16_128, SMALL_BF16_96])
+def test_bf16_greedy_spec_equals_ar_long_context(cfg):
+    """bf16 path: speculative greedy output equals full-depth greedy output bit
+    for bit with contexts spanning several attention splits."""
+    w = syn.make_weights(cfg)
+    prompt = syn.uniform_prompt(270, cfg.vocab, seed=6)
+    # (1, 2) with R = 6 can fork up to 33 branches; (2, 3) stays within 8
+    dec = syn.DecodeConfig(1, 2, 0.0, 1.0, 2, 48) if cfg.R == 4 else syn.DecodeConfig(2, 3, 0.0, 1.0, 2, 48)
+    g = _decoder(cfg, dec, w, max_branches=16, max_ctx=400)
+    g.prefill(prompt)
+    ar, _ = g.generate(dec.max_new, ar=True)
+    g.prefill(prompt)
+    sp, st = g.generate(dec.max_new)
+    assert sp == ar
+    assert st["n_first"] + st["n_second"] + st["n_fallback"] == dec.max_new
+
+
+def test_tree_edits_match_oracle(tiny):
+    """lt_rollback_branch / lt_commit_branch between single steps: the GPU's
+    branch rows, slots and commits stay bit-identical to the oracle doing the
+    same edits."""
+    from oracle import decode as D
+    from oracle.model import LoopedModel
+    cfg, w, prompt = tiny
+    dec = syn.DECODES["tiny_greedy"].replace(d1=1, d2=2, max_new=24)
+    g = _decoder(cfg, dec, w, max_branches=16)
+    first, _, _ = g.prefill(prompt)
+    sd = D.SpecDecoder(D.OracleRows(LoopedModel(cfg, w, 256)), prompt, cfg.R, dec.d1, dec.d2,
+                       dec.max_new, 0.0, 1.0, dec.seed, 256)
+    assert sd.committed[-1] == first
+    edits = 0
+    for step in range(1, 21):
+        g.step()
+        sd.step()
+        if step in (5, 11):
+            root = sd.root().uid
+            uid = max(u for u in sd.branches if u != root)
+            g.rollback_branch(uid)
+            sd.rollback(uid)
+            edits += 1
+        if step == 8 and sd.root().child1 in sd.branches:
+            uid = sd.root().child1
+            g.commit_branch(uid)
+            sd.commit_branch(uid)
+            edits += 1
+    assert edits == 3
+    assert g.read_trace(sd.stats.steps) == sd.trace
+    toks, slots = g.read_committed()
+    assert toks == sd.committed and slots == sd.cslots
+    n = len(sd.src)
+    _, src, step = g.read_log(n)
+    assert src == sd.src and step == sd.cstep
+    table = g.read_table()
+    live = sorted(int(table[1, k]) for k in range(table.shape[1]) if table[0, k])
+    assert live == sorted(sd.branches)

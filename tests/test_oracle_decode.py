@@ -120,3 +120,49 @@ def test_eq8_printed_depths():
         eps = 1e-6
         assert abs((f(o1 + eps, o2) - f(o1 - eps, o2)) / (2 * eps)) < 1e-5
         assert abs((f(o1, o2 + eps) - f(o1, o2 - eps)) / (2 * eps)) < 1e-5
+
+
+def test_rollback_keeps_output_lossless_and_commit_branch_edits_tree():
+    """Rolling back a speculative branch only discards work: greedy output is
+    unchanged.  Committing a root child appends its token, re-roots on it and
+    keeps only its subtree."""
+    cfg, w = _tiny()
+    prompt = syn.prompt_for("tiny", 16)
+    n = 14
+    ref = D.decode_ar(D.OracleRows(LoopedModel(cfg, w, 128)), prompt, cfg.R, n, 0.0, 1.0, 2)
+    sd = D.SpecDecoder(D.OracleRows(LoopedModel(cfg, w, 128)), prompt, cfg.R, 1, 2, n, 0.0, 1.0,
+                       2, 128)
+    rolled = 0
+    while not sd.done():
+        sd.step()
+        root = sd.root().uid if not sd.done() else None
+        others = [u for u in sd.branches if u != root]
+        if others and rolled < 3 and sd.stats.steps % 5 == 0:
+            sd.rollback(max(others))
+            rolled += 1
+            live = [b.slot for b in sd.branches.values()]
+            assert len(set(live)) == len(live) and not (set(live) & sd.free)
+    assert rolled == 3 and sd.committed[len(prompt):] == ref.tokens
+
+    sd = D.SpecDecoder(D.OracleRows(LoopedModel(cfg, w, 128)), prompt, cfg.R, 1, 2, n, 0.0, 1.0,
+                       2, 128)
+    for _ in range(3):
+        sd.step()
+    root = sd.root()
+    child = sd.branches[root.child1]
+    L = len(sd.committed)
+    sd.commit_branch(child.uid)
+    assert sd.committed[-1] == child.token and len(sd.committed) == L + 1
+    assert sd.root().uid == child.uid and sd.src[-1] == 3
+    assert sd.cslots[-1] == child.slot and root.slot in sd.cslots
+    for b in sd.branches.values():
+        assert b.uid == child.uid or child.uid in _ancestors(sd, b)
+
+
+def _ancestors(sd, b):
+    out = []
+    x = sd.branches.get(b.parent)
+    while x is not None:
+        out.append(x.uid)
+        x = sd.branches.get(x.parent)
+    return out
