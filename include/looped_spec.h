@@ -196,6 +196,26 @@ typedef struct {
 } lt_info;
 int lt_get_info(lt_handle* h, lt_info* out);
 
+/*
+ * One shared-block pass over caller-specified rows (the mixed-depth step of
+ * sections 1 / 2.2 in isolation, for kernel sweeps): row i sits at loop depth
+ * h_depth[i] in 1..R and position h_pos[i]; it attends over the slots
+ * d_lists[h_list_off[i] + j], j = 0..h_pos[i] (device int32; the last one is its
+ * own slot, where its K/V rows are written) in the cache planes of its depth.
+ * d_hidden [n_rows][d_model] fp32 (device) holds H^(r-1) on entry and H^(r)
+ * after all n_core layers on return.  n_rows <= max_branches.  iters > 1 or
+ * h_ms != NULL: the pass is captured once as a CUDA graph and replayed iters
+ * times (each replay continues from the previous output), h_ms[k] = replay k's
+ * time in ms (CUDA events on the handle's stream).  Resets any decode state.
+ */
+int lt_block_pass(lt_handle* h, int n_rows, const int32_t* h_depth, const int32_t* h_pos,
+                  const int32_t* d_lists, const int32_t* h_list_off, float* d_hidden, int iters,
+                  float* h_ms);
+/* KV pool of a handle, for callers that fill caches (sweeps, tests): layout
+ * [plane][slot][K|V][d_model] in the model dtype; the plane of shared-block
+ * layer l at depth r is plane_core0 + l * R + (r - 1). */
+int lt_kv_pool(lt_handle* h, void** d_pool, size_t* bytes, int* n_planes, int* n_slots,
+               int* plane_core0);
 int lt_reset(lt_handle* h);
 const char* lt_last_error(const lt_handle* h);
 void lt_destroy(lt_handle* h);

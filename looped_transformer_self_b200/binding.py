@@ -105,6 +105,9 @@ def _declare(L):
     L.lt_read_committed.argtypes = [_vp, _ip, _ip, ctypes.POINTER(_i)]
     L.lt_read_branch_table.argtypes = [_vp, _ip]
     L.lt_read_readouts.argtypes = [_vp, _vp, _vp, _ip, _ip]
+    L.lt_block_pass.argtypes = [_vp, _i, _ip, _ip, _vp, _ip, _vp, _i, ctypes.POINTER(ctypes.c_float)]
+    L.lt_kv_pool.argtypes = [_vp, ctypes.POINTER(_vp), ctypes.POINTER(_sz), ctypes.POINTER(_i),
+                             ctypes.POINTER(_i), ctypes.POINTER(_i)]
     L.lt_rollback_branch.argtypes = [_vp, ctypes.c_int32]
     L.lt_commit_branch.argtypes = [_vp, ctypes.c_int32]
     L.lt_profile_steps.argtypes = [_vp, _i, _i, ctypes.POINTER(ProfileC)]
@@ -259,6 +262,29 @@ class Decoder:
         self._check(lib().lt_decode_step(self.h, 1 if ar else 0, _i32p(tok), ctypes.byref(n)),
                     "lt_decode_step")
         return int(tok[0]) if n.value else None
+
+    def kv_pool(self):
+        """(torch view of the KV pool [planes, slots, 2, d], plane of core layer 0)."""
+        p, nb, npl, ns, pc0 = _vp(), _sz(), _i(), _i(), _i()
+        self._check(lib().lt_kv_pool(self.h, ctypes.byref(p), ctypes.byref(nb), ctypes.byref(npl),
+                                     ctypes.byref(ns), ctypes.byref(pc0)), "lt_kv_pool")
+        dt = torch.float32 if self.cfg.dtype == "f32" else torch.bfloat16
+        off = p.value - self.workspace.data_ptr()
+        raw = self.workspace[off:off + nb.value]
+        view = raw.view(dt).view(npl.value, ns.value, 2, self.cfg.d_model)
+        return view, pc0.value
+
+    def block_pass(self, depth, pos, lists, list_off, hidden, iters=1, timed=False):
+        """One shared-block pass; lists: device int32 tensor; hidden: device fp32
+        [n_rows, d] (updated in place).  Returns per-replay ms when timed."""
+        np = self.np
+        dep = np.ascontiguousarray(depth, dtype=np.int32)
+        ps = np.ascontiguousarray(pos, dtype=np.int32)
+        off = np.ascontiguousarray(list_off, dtype=np.int32)
+        ms = (ctypes.c_float * iters)() if timed else None
+        self._check(lib().lt_block_pass(self.h, len(dep), _i32p(dep), _i32p(ps), lists.data_ptr(),
+                                        _i32p(off), hidden.data_ptr(), iters, ms), "lt_block_pass")
+        return list(ms) if timed else None
 
     def rollback_branch(self, uid):
         self._check(lib().lt_rollback_branch(self.h, uid), "lt_rollback_branch")

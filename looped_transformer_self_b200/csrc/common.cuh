@@ -169,6 +169,47 @@ __device__ __forceinline__ float sk_reduce(const float* __restrict__ part, const
   return acc;
 }
 
+// ---- in-GEMM epilogues --------------------------------------------------------------
+// The CTA whose segment completes a group of output tiles (the last to arrive
+// on the group's counter) reduces the group's partials in fixed CTA order and
+// applies the epilogue, so no separate epilogue kernel is needed.
+//
+// RMSNorm is applied by its consumers: a GEMM operand row is X = g (.) h
+// (unnormalised) and the per-row factor r = 1 / sqrt(mean(h^2) + eps) -- which
+// commutes with the matmul -- multiplies the GEMM's reduced output.  Sums of
+// squares come as per-128-feature tile parts ssq[t][row], added in tile order.
+enum EpiKind : int { EPI_NONE = 0, EPI_RESID = 1, EPI_SWIGLU = 2 };
+
+struct GemmEpi {
+  int kind;
+  int* counters;       // [groups] arrivals, zero between launches (the last arrival resets)
+  const int* need;     // [groups] segments that complete a group
+  const int* mask;     // [ncols] rows taking part
+  // EPI_RESID (group = one tile of h's features):
+  //   h[i][n] += scale * y;  X[i][n] = g[n] * h[i][n] (if g);  ssq_out[t][i] = sum_n h[i][n]^2
+  float* h;
+  float scale;
+  const void* g;
+  void* X;
+  size_t lo;           // lo-plane offset of X (split tf32), 0 otherwise
+  float* ssq_out;
+  // EPI_SWIGLU (group = gate tile t with up tile t + ffn/128):
+  //   X[i][n] = SiLU(r_i * gate) * (r_i * up), r_i from ssq_in
+  const float* ssq_in;
+  int ssq_tiles;       // tiles of the normalised row (ceil(d / 128))
+  float eps;
+  int d;               // features of h (RESID) / of the normalised row (SWIGLU)
+  int ffn;
+};
+
+// 1 / sqrt(mean(h_i^2) + eps) from per-tile sum-of-squares parts (fixed order).
+__device__ __forceinline__ float inv_rms_parts(const float* __restrict__ ssq, int tiles,
+                                               int ncols, int i, int d, float eps) {
+  float s = 0.f;
+  for (int t = 0; t < tiles; ++t) s += __ldcg(ssq + (size_t)t * ncols + i);
+  return rsqrtf(s / d + eps);
+}
+
 // ---- programmatic dependent launch ---------------------------------------------
 __device__ __forceinline__ void pdl_wait() {
   asm volatile("griddepcontrol.wait;" ::: "memory");

@@ -166,7 +166,8 @@ __device__ __forceinline__ unsigned long long suffix_scan_1024(unsigned long lon
 __global__ void __launch_bounds__(1024)
     k_readout(const float* __restrict__ part, const GemmShape s, int C,
               const int* __restrict__ mask, int V, int greedy, float T, float top_p,
-              float* __restrict__ logits, float* __restrict__ P, int* __restrict__ arg) {
+              float* __restrict__ logits, float* __restrict__ P, int* __restrict__ arg,
+              const float* __restrict__ ssq, int ssq_tiles, int d, float eps) {
   __shared__ float sk[33];
   __shared__ int si[33];
   __shared__ float red[33];
@@ -180,6 +181,7 @@ __global__ void __launch_bounds__(1024)
   if (!mask[i]) return;
   float* z = logits + (size_t)i * V;
   float* p = P + (size_t)i * V;
+  const float rr = inv_rms_parts(ssq, ssq_tiles, C, i, d, eps);  // final RMSNorm factor
   float best = -INFINITY;
   int bi = 0x7fffffff;
   // four elements per round so their partial loads overlap
@@ -188,7 +190,7 @@ __global__ void __launch_bounds__(1024)
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const int j = j0 + u * blockDim.x;
-      v[u] = j < V ? sk_reduce(part, s, C, i, j) : 0.f;
+      v[u] = j < V ? rr * sk_reduce(part, s, C, i, j) : 0.f;
     }
 #pragma unroll
     for (int u = 0; u < 4; ++u) {

@@ -46,6 +46,13 @@ struct Handle {
   Dev D;
   float *h = nullptr, *hc = nullptr, *q = nullptr, *attn_part = nullptr, *part = nullptr;
   int* attn_cnt = nullptr;  // per (row, head) split-arrival counters (kept at zero between uses)
+  const int* lists_override = nullptr;  // caller slot lists of lt_block_pass
+  cudaGraphExec_t pass_graph = nullptr;
+  int pass_graph_rows = -1;
+  float* ssq = nullptr;     // [ceil(d/128)][C] sum-of-squares parts of the pending RMSNorm
+  int ssq_tiles = 0;
+  int *cnt_o = nullptr, *cnt_gu = nullptr, *cnt_d = nullptr;     // in-GEMM epilogue counters
+  int *need_o = nullptr, *need_gu = nullptr, *need_d = nullptr;  // arrivals completing a group
   void *Xd = nullptr, *Xo = nullptr, *Xf = nullptr, *kv = nullptr;
   float2* rope = nullptr;
   int* gemm_tab = nullptr;
@@ -151,12 +158,13 @@ static int validate(const lt_model_config* m, const lt_decode_config* dc, std::s
   if (m->n_core < 1 || m->n_prelude < 0 || m->n_coda < 0) return bad("layer counts");
   const int esz = m->dtype == LT_F32 ? 4 : 2;
   if ((m->d_model * esz) % 16 || (m->ffn * esz) % 16) return bad("d_model/ffn rows must be 16-byte multiples");
+  if (m->ffn % 128) return bad("ffn must be a multiple of 128 (SwiGLU tiles pair gate with up)");
   const int C = dc->max_branches;
   if (C != 8 && C != 16 && C != 32 && C != 64) return bad("max_branches must be 8, 16, 32 or 64");
   if (dc->d1 < 0 || dc->d1 >= m->R || dc->d2 < 0 || (dc->d2 && (dc->d2 <= dc->d1 || dc->d2 >= m->R)))
     return bad("need 1 <= d1 < d2 < R (d2 = 0: single proposal)");
   if (dc->max_ctx < 2) return bad("max_ctx");
-  if (dc->max_ctx + C + 8 > MAX_SLOT_WORDS * 32) return bad("max_ctx too large for the slot bitmap");
+  if (dc->max_ctx + C + 8 > (1 << 24)) return bad("max_ctx too large");
   if (dc->temperature < 0.f || !(dc->top_p > 0.f) || dc->top_p > 1.f) return bad("temperature/top_p");
   if (dc->second_mode < 0 || dc->second_mode > 2) return bad("second_mode");
   return LT_OK;
@@ -201,6 +209,14 @@ static size_t carve(Handle* H, char* base) {
   H->q = cv.take<float>((size_t)C * d);
   H->attn_part = cv.take<float>((size_t)C * m.n_heads * H->max_splits * (m.head_dim + 2));
   H->attn_cnt = cv.take<int>((size_t)C * m.n_heads);
+  H->ssq_tiles = (d + 127) / 128;
+  H->ssq = cv.take<float>((size_t)H->ssq_tiles * C);
+  H->cnt_o = cv.take<int>(H->ssq_tiles);
+  H->cnt_d = cv.take<int>(H->ssq_tiles);
+  H->cnt_gu = cv.take<int>(f / 128);
+  H->need_o = cv.take<int>(H->ssq_tiles);
+  H->need_d = cv.take<int>(H->ssq_tiles);
+  H->need_gu = cv.take<int>(f / 128);
   const int planes_x = H->f32 ? 2 : 1;  // fp32: hi and lo tf32 planes
   H->Xd = cv.take<char>((size_t)planes_x * C * d * esz);
   H->Xo = cv.take<char>((size_t)planes_x * C * d * esz);
@@ -278,7 +294,7 @@ static void plan(Handle* H) {
 template <typename T>
 static cudaError_t gemm(Handle* H, const CUtensorMap& tw, const CUtensorMap& twl,
                         const CUtensorMap& tx, const CUtensorMap& txl, const GemmShape& s,
-                        const int* flag) {
+                        const int* flag, const GemmEpi* epi = nullptr) {
   const double esz = H->f32 ? 4.0 : 2.0, split = H->mode == 2 ? 2.0 : 1.0;
   // algorithmic bytes: the weight matrix (both tf32 halves when split), the
   // activation rows and the fp32 result rows
@@ -287,7 +303,7 @@ static cudaError_t gemm(Handle* H, const CUtensorMap& tw, const CUtensorMap& twl
   ProfScope ps(H, H->prof_cat, bytes);
   if (H->counting) H->kernels_per_step++;
   return gemm_launch(tw, twl, tx, txl, H->part, s, H->C, H->mode, flag, &H->D.ctl->err,
-                     H->stream, H->use_pdl);
+                     H->stream, H->use_pdl, epi);
 }
 
 template <typename T, int HD>
@@ -300,9 +316,11 @@ static cudaError_t attention(Handle* H, int gl, const int* tagsrc, int tag_off, 
   return launch(H->use_pdl, kern, dim3(C, Hn, H->max_splits), dim3(128), H->stream,
                 (const float*)H->q, (T*)H->kv, H->plane_base[gl], tagsrc, tag_off, H->S,
                 H->m.d_model, Hn, mask, (const int*)D.r_pos, (const int*)D.r_blen,
-                (const int*)D.r_boff, (const int*)D.lists, (const int*)D.b_chain, (int)WIN,
+                (const int*)D.r_boff, H->lists_override ? H->lists_override : (const int*)D.lists,
+                (const int*)D.b_chain, (int)WIN,
                 H->max_splits, H->attn_part, H->attn_cnt, Xo, H->lo_d, (const float*)H->part,
-                H->sh_qkv, C, (const int*)D.r_slot, (const float2*)H->rope, &D.ctl->err);
+                H->sh_qkv, C, (const int*)D.r_slot, (const float2*)H->rope, (const float*)H->ssq,
+                H->ssq_tiles, H->m.rms_eps, &D.ctl->err);
 }
 
 // kind: 0 prelude (one cache), 1 shared block (cache of the row's depth), 2 coda
@@ -319,36 +337,53 @@ static cudaError_t run_layers(Handle* H, int gl0, int n, int kind, const int* ma
   T* Xd = (T*)H->Xd;
   T* Xo = (T*)H->Xo;
   T* Xf = (T*)H->Xf;
+  GemmEpi eo = {}, egu = {}, ed = {};
+  eo.kind = ed.kind = EPI_RESID;
+  eo.counters = H->cnt_o;
+  eo.need = H->need_o;
+  ed.counters = H->cnt_d;
+  ed.need = H->need_d;
+  eo.mask = ed.mask = egu.mask = mask;
+  eo.h = ed.h = hbuf;
+  eo.scale = ed.scale = scale;
+  eo.X = ed.X = H->Xd;
+  eo.lo = ed.lo = H->lo_d;
+  eo.ssq_out = ed.ssq_out = H->ssq;
+  eo.d = ed.d = egu.d = d;
+  egu.kind = EPI_SWIGLU;
+  egu.counters = H->cnt_gu;
+  egu.need = H->need_gu;
+  egu.ssq_in = H->ssq;
+  egu.ssq_tiles = H->ssq_tiles;
+  egu.eps = m.rms_eps;
+  egu.ffn = egu.d = m.ffn;
+  egu.d = d;
+  egu.X = H->Xf;
+  egu.lo = H->lo_f;
   for (int l = 0; l < n; ++l) {
     const int gl = gl0 + l;
     const LayerW& L = H->layers[gl];
     if (l == 0)
       LT_CK(launch(H->use_pdl, k_stage_norm<T>, dim3(C), dim3(EPI_THREADS), H->stream,
-                   (const float*)hbuf, mask, (const T*)L.g1, m.rms_eps, d, Xd, H->lo_d));
+                   (const float*)hbuf, mask, (const T*)L.g1, d, C, Xd, H->lo_d, H->ssq));
     LT_CK(gemm<T>(H, L.tm_qkv, L.tm_qkv_lo, H->tm_Xd, H->tm_Xd_lo, H->sh_qkv, flag));
     if (!fused)
       LT_CK(launch(H->use_pdl, k_qkv_epi<T>, dim3(C), dim3(EPI_THREADS), H->stream,
                    (const float*)H->part, H->sh_qkv, C, mask, (const int*)D.r_pos,
                    (const int*)D.r_slot, tagsrc, tag_off, H->plane_base[gl], H->S, d, m.head_dim,
-                   (const float2*)H->rope, (T*)H->kv, H->q, &D.ctl->err));
+                   (const float2*)H->rope, (T*)H->kv, H->q, (const float*)H->ssq, H->ssq_tiles,
+                   m.rms_eps, &D.ctl->err));
     switch (m.head_dim) {
       case 32: LT_CK((attention<T, 32>(H, gl, tagsrc, tag_off, mask, Xo, fused))); break;
       case 64: LT_CK((attention<T, 64>(H, gl, tagsrc, tag_off, mask, Xo, fused))); break;
       case 96: LT_CK((attention<T, 96>(H, gl, tagsrc, tag_off, mask, Xo, fused))); break;
       default: LT_CK((attention<T, 128>(H, gl, tagsrc, tag_off, mask, Xo, fused))); break;
     }
-    LT_CK(gemm<T>(H, L.tm_o, L.tm_o_lo, H->tm_Xo, H->tm_Xo_lo, H->sh_o, flag));
-    LT_CK(launch(H->use_pdl, k_resid_epi<T>, dim3(C), dim3(EPI_THREADS), H->stream,
-                 (const float*)H->part, H->sh_o, C, mask, hbuf, scale, (const T*)L.g2,
-                 m.rms_eps, d, Xd, H->lo_d));
-    LT_CK(gemm<T>(H, L.tm_gu, L.tm_gu_lo, H->tm_Xd, H->tm_Xd_lo, H->sh_gu, flag));
-    LT_CK(launch(H->use_pdl, k_gu_epi<T>, dim3(C, 4), dim3(EPI_THREADS), H->stream,
-                 (const float*)H->part, H->sh_gu, C, mask, m.ffn, Xf, H->lo_f));
-    LT_CK(gemm<T>(H, L.tm_d, L.tm_d_lo, H->tm_Xf, H->tm_Xf_lo, H->sh_d, flag));
-    const T* gnext = (l + 1 < n) ? (const T*)H->layers[gl + 1].g1 : nullptr;
-    LT_CK(launch(H->use_pdl, k_resid_epi<T>, dim3(C), dim3(EPI_THREADS), H->stream,
-                 (const float*)H->part, H->sh_d, C, mask, hbuf, scale, gnext, m.rms_eps, d, Xd,
-                 H->lo_d));
+    eo.g = L.g2;  // O: h += s * o W_o^T; X = g2 (.) h for the gate/up GEMM
+    LT_CK(gemm<T>(H, L.tm_o, L.tm_o_lo, H->tm_Xo, H->tm_Xo_lo, H->sh_o, flag, &eo));
+    LT_CK(gemm<T>(H, L.tm_gu, L.tm_gu_lo, H->tm_Xd, H->tm_Xd_lo, H->sh_gu, flag, &egu));
+    ed.g = (l + 1 < n) ? H->layers[gl + 1].g1 : nullptr;  // next layer's g1 (.) h
+    LT_CK(gemm<T>(H, L.tm_d, L.tm_d_lo, H->tm_Xf, H->tm_Xf_lo, H->sh_d, flag, &ed));
   }
   return cudaSuccess;
 }
@@ -368,12 +403,12 @@ static cudaError_t run_readout(Handle* H, const int* flag, bool fused) {
     src = H->hc;
   }
   LT_CK(launch(H->use_pdl, k_stage_norm<T>, dim3(C), dim3(EPI_THREADS), H->stream,
-               (const float*)src, (const int*)D.m_ro, (const T*)H->final_norm, m.rms_eps, d,
-               (T*)H->Xd, H->lo_d));
+               (const float*)src, (const int*)D.m_ro, (const T*)H->final_norm, d, C, (T*)H->Xd,
+               H->lo_d, H->ssq));
   LT_CK(gemm<T>(H, H->tm_head, H->tm_head_lo, H->tm_Xd, H->tm_Xd_lo, H->sh_head, flag));
   return launch(H->use_pdl, k_readout, dim3(C), dim3(1024), H->stream, (const float*)H->part,
                 H->sh_head, C, (const int*)D.m_ro, m.vocab, D.greedy, D.T, D.top_p, D.logits,
-                D.P, D.ro_arg);
+                D.P, D.ro_arg, (const float*)H->ssq, H->ssq_tiles, d, m.rms_eps);
 }
 
 template <typename T>
@@ -498,6 +533,24 @@ extern "C" int lt_create(const lt_model_config* m, const lt_decode_config* dc, v
   for (int k = 0; k < 5; ++k) {
     shapes[k]->tile_c = H->gemm_tab + offs[k];
     shapes[k]->cta_t0 = H->gemm_tab + offs[k] + 2 * shapes[k]->tiles;
+  }
+  {  // arrivals that complete each epilogue group (O / down: per tile; gate/up: per pair)
+    std::vector<int> need_o(H->ssq_tiles), need_d(H->ssq_tiles), need_gu(f / 128);
+    gemm_group_need(H->sh_o, tab.data() + offs[1], 0, need_o.data());
+    gemm_group_need(H->sh_gu, tab.data() + offs[2], 2, need_gu.data());
+    gemm_group_need(H->sh_d, tab.data() + offs[3], 0, need_d.data());
+    const size_t esz = H->f32 ? 4 : 2, px = H->f32 ? 2 : 1;
+    if (cudaMemcpy(H->need_o, need_o.data(), need_o.size() * 4, cudaMemcpyHostToDevice) ||
+        cudaMemcpy(H->need_d, need_d.data(), need_d.size() * 4, cudaMemcpyHostToDevice) ||
+        cudaMemcpy(H->need_gu, need_gu.data(), need_gu.size() * 4, cudaMemcpyHostToDevice) ||
+        cudaMemset(H->cnt_o, 0, need_o.size() * 4) || cudaMemset(H->cnt_d, 0, need_d.size() * 4) ||
+        cudaMemset(H->cnt_gu, 0, need_gu.size() * 4) ||
+        cudaMemset(H->Xd, 0, px * H->C * d * esz) || cudaMemset(H->Xo, 0, px * H->C * d * esz) ||
+        cudaMemset(H->Xf, 0, px * H->C * f * esz) ||
+        cudaMemset(H->ssq, 0, (size_t)H->ssq_tiles * H->C * 4)) {
+      delete hd;
+      return LT_ERR_CUDA;
+    }
   }
   // activation tensor maps (B operands)
   const size_t esz = H->f32 ? 4 : 2;
@@ -674,6 +727,8 @@ extern "C" int lt_prefill(lt_handle* hd, const int32_t* h_tokens, int n, int32_t
   Handle* H = &hd->h;
   if (!H->loaded) return fail(hd, LT_ERR_STATE, "weights not loaded");
   if (n + 1 > H->dc.max_ctx) return fail(hd, LT_ERR_CAPACITY, "prompt longer than max_ctx - 1");
+  if (H->S > MAX_SLOT_WORDS * 32)
+    return fail(hd, LT_ERR_CAPACITY, "decoding needs max_ctx + max_branches + 8 <= 65536 slots");
   for (int k = 0; k < n; ++k)
     if (h_tokens[k] < 0 || h_tokens[k] >= H->m.vocab) return fail(hd, LT_ERR_ARG, "token id out of range");
   return H->f32 ? prefill_t<float>(hd, h_tokens, n, h_first, h_argmax, d_logits)
@@ -895,6 +950,7 @@ extern "C" const char* lt_last_error(const lt_handle* hd) {
 extern "C" void lt_destroy(lt_handle* hd) {
   if (!hd) return;
   if (hd->h.graph) cudaGraphExecDestroy(hd->h.graph);
+  if (hd->h.pass_graph) cudaGraphExecDestroy(hd->h.pass_graph);
   delete hd;
 }
 
@@ -1022,3 +1078,116 @@ static int tree_edit(lt_handle* hd, int mode, int32_t uid) {
 
 extern "C" int lt_rollback_branch(lt_handle* hd, int32_t uid) { return tree_edit(hd, 2, uid); }
 extern "C" int lt_commit_branch(lt_handle* hd, int32_t uid) { return tree_edit(hd, 3, uid); }
+
+// ---------------------------------------------------------------------------
+// one shared-block pass over caller-specified rows (kernel sweep)
+// ---------------------------------------------------------------------------
+__global__ void k_pass_rows(Dev D, int n, const int* __restrict__ lists) {
+  pdl_wait();
+  pdl_trigger();
+  for (int k = threadIdx.x; k < D.C; k += blockDim.x) {
+    const int on = k < n;
+    const int pos = on ? D.r_pos[k] : 0;
+    D.m_alive[k] = on;
+    D.m_new[k] = 0;
+    D.m_ro[k] = 0;
+    D.r_ro[k] = -1;
+    D.r_slot[k] = on ? lists[D.r_boff[k] + pos] : 0;
+    D.r_blen[k] = pos + 1;
+  }
+}
+
+extern "C" int lt_kv_pool(lt_handle* hd, void** d_pool, size_t* bytes, int* n_planes,
+                          int* n_slots, int* plane_core0) {
+  if (!hd) return LT_ERR_ARG;
+  Handle* H = &hd->h;
+  if (d_pool) *d_pool = H->kv;
+  if (bytes) *bytes = (size_t)H->planes * H->S * 2 * H->m.d_model * (H->f32 ? 4 : 2);
+  if (n_planes) *n_planes = H->planes;
+  if (n_slots) *n_slots = H->S;
+  if (plane_core0) *plane_core0 = H->plane_base[H->m.n_prelude];
+  return LT_OK;
+}
+
+extern "C" int lt_block_pass(lt_handle* hd, int n_rows, const int32_t* h_depth,
+                             const int32_t* h_pos, const int32_t* d_lists,
+                             const int32_t* h_list_off, float* d_hidden, int iters,
+                             float* h_ms) {
+  if (!hd || !h_depth || !h_pos || !d_lists || !h_list_off || !d_hidden || iters < 1)
+    return LT_ERR_ARG;
+  Handle* H = &hd->h;
+  if (!H->loaded) return fail(hd, LT_ERR_STATE, "weights not loaded");
+  const int C = H->C, d = H->m.d_model;
+  if (n_rows < 1 || n_rows > C) return fail(hd, LT_ERR_CAPACITY, "n_rows exceeds max_branches");
+  std::vector<int> pos(C, 0), dep(C, 1), off(C, 0);
+  for (int i = 0; i < n_rows; ++i) {
+    if (h_depth[i] < 1 || h_depth[i] > H->m.R) return fail(hd, LT_ERR_ARG, "depth out of 1..R");
+    if (h_pos[i] < 0 || h_pos[i] >= H->max_pos) return fail(hd, LT_ERR_ARG, "position out of range");
+    if (h_list_off[i] < 0) return fail(hd, LT_ERR_ARG, "negative list offset");
+    pos[i] = h_pos[i];
+    dep[i] = h_depth[i];
+    off[i] = h_list_off[i];
+  }
+  Dev& D = H->D;
+  cudaStream_t st = H->stream;
+  cudaError_t e;
+  if ((e = cudaMemcpyAsync(D.r_pos, pos.data(), C * 4, cudaMemcpyHostToDevice, st)) ||
+      (e = cudaMemcpyAsync(D.r_depth, dep.data(), C * 4, cudaMemcpyHostToDevice, st)) ||
+      (e = cudaMemcpyAsync(D.r_boff, off.data(), C * 4, cudaMemcpyHostToDevice, st)) ||
+      (e = launch(false, k_pass_rows, dim3(1), dim3(64), st, D, n_rows, (const int*)d_lists)) ||
+      (e = cudaMemcpyAsync(H->h, d_hidden, (size_t)n_rows * d * 4, cudaMemcpyDeviceToDevice, st)))
+    return cuda_fail(hd, e, "block pass setup");
+  H->prefilled = false;  // the row arrays and caches no longer hold a decode state
+  H->begun = false;
+  H->lists_override = d_lists;
+  auto pass = [&]() -> cudaError_t {
+    return H->f32 ? run_layers<float>(H, H->m.n_prelude, H->m.n_core, 1, D.m_alive, H->h,
+                                      H->m.resid_scale, nullptr, true)
+                  : run_layers<__nv_bfloat16>(H, H->m.n_prelude, H->m.n_core, 1, D.m_alive,
+                                              H->h, H->m.resid_scale, nullptr, true);
+  };
+  int rc = LT_OK;
+  if (iters == 1 && !h_ms) {
+    if ((e = pass())) rc = cuda_fail(hd, e, "block pass");
+  } else {
+    // one graph of the pass, replayed; events on the handle's stream around each replay
+    if (H->pass_graph && H->pass_graph_rows != n_rows) {
+      cudaGraphExecDestroy(H->pass_graph);
+      H->pass_graph = nullptr;
+    }
+    if (!H->pass_graph) {
+      cudaGraph_t g = nullptr;
+      if ((e = cudaStreamBeginCapture(st, cudaStreamCaptureModeThreadLocal))) {
+        H->lists_override = nullptr;
+        return cuda_fail(hd, e, "capture");
+      }
+      cudaError_t e2 = pass();
+      e = cudaStreamEndCapture(st, &g);
+      if (e2 || e || (e = cudaGraphInstantiate(&H->pass_graph, g, 0))) {
+        if (g) cudaGraphDestroy(g);
+        H->lists_override = nullptr;
+        return cuda_fail(hd, e2 ? e2 : e, "pass graph");
+      }
+      cudaGraphDestroy(g);
+      H->pass_graph_rows = n_rows;
+    }
+    std::vector<cudaEvent_t> ev(iters + 1);
+    for (auto& x : ev) cudaEventCreate(&x);
+    cudaEventRecord(ev[0], st);
+    for (int k = 0; k < iters && !rc; ++k) {
+      if ((e = cudaGraphLaunch(H->pass_graph, st))) rc = cuda_fail(hd, e, "pass replay");
+      cudaEventRecord(ev[k + 1], st);
+    }
+    if (!rc && (e = cudaStreamSynchronize(st))) rc = cuda_fail(hd, e, "pass sync");
+    if (!rc && h_ms)
+      for (int k = 0; k < iters; ++k) cudaEventElapsedTime(&h_ms[k], ev[k], ev[k + 1]);
+    for (auto& x : ev) cudaEventDestroy(x);
+  }
+  H->lists_override = nullptr;
+  if (rc) return rc;
+  if ((e = cudaMemcpyAsync(d_hidden, H->h, (size_t)n_rows * d * 4, cudaMemcpyDeviceToDevice, st)) ||
+      (e = cudaStreamSynchronize(st)))
+    return cuda_fail(hd, e, "block pass result");
+  Ctl c;
+  return read_ctl(hd, &c);
+}

@@ -2,6 +2,7 @@
 #include <stdio.h>
 
 #include <algorithm>
+#include <type_traits>
 
 #include "gemm.cuh"
 
@@ -143,6 +144,111 @@ constexpr int tmem_cols() {
 }
 
 // ---------------------------------------------------------------------------
+// in-GEMM epilogues (run by the 4 drain warps of the CTA completing a group)
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void drain_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+template <typename TX>
+__device__ __forceinline__ void store_x(TX* X, size_t idx, float v, size_t lo);
+template <>
+__device__ __forceinline__ void store_x<__nv_bfloat16>(__nv_bfloat16* X, size_t idx, float v,
+                                                       size_t) {
+  X[idx] = __float2bfloat16_rn(v);
+}
+template <>
+__device__ __forceinline__ void store_x<float>(float* X, size_t idx, float v, size_t lo) {
+  if (lo) {  // split tf32 pair
+    const float hi = __uint_as_float(__float_as_uint(v) & 0xFFFFE000u);
+    X[idx] = hi;
+    X[lo + idx] = v - hi;
+  } else {
+    X[idx] = v;
+  }
+}
+template <typename TX>
+__device__ __forceinline__ float load_g(const void* g, int n) {
+  return (float)(reinterpret_cast<const TX*>(g)[n]);
+}
+
+struct EpiSmem {
+  int rows[64];      // active rows of this launch
+  int nact;
+  int last;          // group completed by this CTA, or -1
+  float inv[64];     // per active row: 1 / rms (SwiGLU)
+  float wsum[4][64]; // per warp, per active row: partial sum of squares
+};
+
+// Residual epilogue of one tile: h += scale * y; X = g (.) h; sum-of-squares part.
+template <typename TX>
+__device__ void epi_resid(const GemmEpi& ep, const float* __restrict__ part, const GemmShape& s,
+                          int ncols, int t, int et, EpiSmem& sm) {
+  const int n = t * 128 + et;
+  const bool valid = n < s.n_out;
+  const int lane = et & 31, w = et >> 5;
+  for (int k0 = 0; k0 < sm.nact; k0 += 4) {
+    float y[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int k = k0 + u;
+      y[u] = (valid && k < sm.nact) ? sk_reduce(part, s, ncols, sm.rows[k], n) : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int k = k0 + u;
+      if (k >= sm.nact) break;
+      const int i = sm.rows[k];
+      float hv = 0.f;
+      if (valid) {
+        float* hp = ep.h + (size_t)i * ep.d + n;
+        hv = *hp + ep.scale * y[u];
+        *hp = hv;
+        if (ep.g)
+          store_x<TX>(reinterpret_cast<TX*>(ep.X), (size_t)i * ep.d + n, load_g<TX>(ep.g, n) * hv,
+                      ep.lo);
+      }
+      float sq = hv * hv;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
+      if (lane == 0) sm.wsum[w][k] = sq;
+    }
+  }
+  drain_sync();
+  if (et < sm.nact) {
+    const float v = sm.wsum[0][et] + sm.wsum[1][et] + sm.wsum[2][et] + sm.wsum[3][et];
+    ep.ssq_out[(size_t)t * ncols + sm.rows[et]] = v;
+  }
+}
+
+// SwiGLU epilogue of one (gate tile, up tile) pair.
+template <typename TX>
+__device__ void epi_swiglu(const GemmEpi& ep, const float* __restrict__ part, const GemmShape& s,
+                           int ncols, int t, int et, EpiSmem& sm) {
+  if (et < sm.nact)
+    sm.inv[et] = inv_rms_parts(ep.ssq_in, ep.ssq_tiles, ncols, sm.rows[et], ep.d, ep.eps);
+  drain_sync();
+  const int n = t * 128 + et;
+  if (n >= ep.ffn) return;
+  for (int k0 = 0; k0 < sm.nact; k0 += 2) {
+    float gv[2], uv[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int k = k0 + u;
+      gv[u] = k < sm.nact ? sk_reduce(part, s, ncols, sm.rows[k], n) : 0.f;
+      uv[u] = k < sm.nact ? sk_reduce(part, s, ncols, sm.rows[k], ep.ffn + n) : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int k = k0 + u;
+      if (k >= sm.nact) break;
+      const float r = sm.inv[k];
+      const float g = r * gv[u], up = r * uv[u];
+      store_x<TX>(reinterpret_cast<TX*>(ep.X), (size_t)sm.rows[k] * ep.ffn + n,
+                  g / (1.f + __expf(-g)) * up, ep.lo);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
 // kernel
 // ---------------------------------------------------------------------------
 // MODE 0: bf16 operands.  MODE 1: tf32 operands.  MODE 2: fp32 operands as
@@ -154,7 +260,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     k_gemm(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmWlo,
            const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmXlo,
            float* __restrict__ part, const GemmShape s, const int stages,
-           const int* __restrict__ run_flag, int* __restrict__ err) {
+           const int* __restrict__ run_flag, int* __restrict__ err, const GemmEpi ep) {
+  using TX = typename std::conditional<MODE == 0, __nv_bfloat16, float>::type;
+  __shared__ EpiSmem esm;
   constexpr bool TF32 = MODE != 0;
   constexpr int NSPLIT = MODE == 2 ? 2 : 1;
   constexpr uint32_t A_BYTES = GEMM_BM * GEMM_CHUNK_BYTES;
@@ -340,8 +448,15 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       mbar_wait(drain_bar, 0, &dummy);
     }
   } else if (warp >= 2) {
-    // ---------------- drain: TMEM -> fp32 partials ----------------
+    // ---------------- drain: TMEM -> fp32 partials (+ group epilogue) ----------------
     const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int et = threadIdx.x - 64;  // 0..127 over the drain warps
+    if (ep.kind != EPI_NONE && et == 0) {
+      int na = 0;
+      for (int i = 0; i < NC; ++i)
+        if (ep.mask[i]) esm.rows[na++] = i;
+      esm.nact = na;
+    }
     int seg = 0;
     for (int u = u0; u < u1; ++seg) {
       const int t = u / s.kch;
@@ -359,6 +474,25 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       float* dst = part + ((size_t)(c * s.jmax + seg) * NC) * GEMM_BM + q * 32 + lane;
 #pragma unroll
       for (int i = 0; i < NC; ++i) dst[(size_t)i * GEMM_BM] = __uint_as_float(r[i]);
+      if (ep.kind != EPI_NONE) {
+        // publish this segment; the arrival that completes the group runs its epilogue
+        __threadfence();
+        drain_sync();
+        if (et == 0) {
+          const int grp = ep.kind == EPI_SWIGLU ? t % (ep.ffn / GEMM_BM) : t;
+          const int old = atomicAdd(ep.counters + grp, 1);
+          esm.last = (old + 1 == ep.need[grp]) ? grp : -1;
+          if (esm.last >= 0) ep.counters[grp] = 0;
+        }
+        drain_sync();
+        const int grp = esm.last;
+        if (grp >= 0) {
+          __threadfence();
+          if (ep.kind == EPI_RESID) epi_resid<TX>(ep, part, s, NC, grp, et, esm);
+          else epi_swiglu<TX>(ep, part, s, NC, grp, et, esm);
+        }
+        drain_sync();
+      }
       u = seg_end;
     }
   }
@@ -426,6 +560,15 @@ void gemm_plan(int n_out, int k, bool f32, int grid_cap, GemmShape* s, int* tile
   s->cta_t0 = nullptr;
 }
 
+void gemm_group_need(const GemmShape& s, const int* tile_c_host, int group_tiles, int* need) {
+  const int groups = group_tiles > 0 ? s.tiles / group_tiles : s.tiles;
+  for (int g = 0; g < groups; ++g) need[g] = 0;
+  for (int t = 0; t < s.tiles; ++t) {
+    const int g = group_tiles > 0 ? t % groups : t;
+    need[g] += tile_c_host[2 * t + 1] - tile_c_host[2 * t] + 1;
+  }
+}
+
 size_t gemm_part_bytes(const GemmShape& s, int ncols) {
   return (size_t)s.grid * s.jmax * ncols * GEMM_BM * sizeof(float);
 }
@@ -469,7 +612,7 @@ template <int MODE, int NC>
 static cudaError_t launch_t(const CUtensorMap& tmW, const CUtensorMap& tmWlo,
                             const CUtensorMap& tmX, const CUtensorMap& tmXlo, float* part,
                             const GemmShape& s, const int* run_flag, int* err,
-                            cudaStream_t stream, bool pdl) {
+                            cudaStream_t stream, bool pdl, const GemmEpi& ep) {
   const int nsplit = MODE == 2 ? 2 : 1;
   const int stages = stages_for(NC, nsplit);
   const size_t smem = smem_bytes(NC, stages, nsplit);
@@ -491,17 +634,21 @@ static cudaError_t launch_t(const CUtensorMap& tmW, const CUtensorMap& tmWlo,
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
   return cudaLaunchKernelEx(&cfg, k_gemm<MODE, NC>, tmW, tmWlo, tmX, tmXlo, part, s, stages,
-                            run_flag, err);
+                            run_flag, err, ep);
 }
 
 cudaError_t gemm_launch(const CUtensorMap& tmW, const CUtensorMap& tmWlo, const CUtensorMap& tmX,
                         const CUtensorMap& tmXlo, float* part, const GemmShape& s, int ncols,
-                        int mode, const int* run_flag, int* err, cudaStream_t stream, bool pdl) {
+                        int mode, const int* run_flag, int* err, cudaStream_t stream, bool pdl,
+                        const GemmEpi* epi) {
+  GemmEpi none = {};
+  none.kind = EPI_NONE;
+  const GemmEpi& ep = epi ? *epi : none;
 #define LT_GEMM_CASE(N)                                                                      \
   case N:                                                                                    \
-    return mode == 2   ? launch_t<2, N>(tmW, tmWlo, tmX, tmXlo, part, s, run_flag, err, stream, pdl) \
-           : mode == 1 ? launch_t<1, N>(tmW, tmWlo, tmX, tmXlo, part, s, run_flag, err, stream, pdl) \
-                       : launch_t<0, N>(tmW, tmWlo, tmX, tmXlo, part, s, run_flag, err, stream, pdl);
+    return mode == 2   ? launch_t<2, N>(tmW, tmWlo, tmX, tmXlo, part, s, run_flag, err, stream, pdl, ep) \
+           : mode == 1 ? launch_t<1, N>(tmW, tmWlo, tmX, tmXlo, part, s, run_flag, err, stream, pdl, ep) \
+                       : launch_t<0, N>(tmW, tmWlo, tmX, tmXlo, part, s, run_flag, err, stream, pdl, ep);
   switch (ncols) {
     LT_GEMM_CASE(8)
     LT_GEMM_CASE(16)

@@ -58,9 +58,16 @@ int make_tmap(CUtensorMap* map, const void* base, bool f32, uint64_t rows, uint6
 // split tf32 (tmWlo / tmXlo map the low parts; ignored otherwise).  run_flag
 // (device, may be null): skip when *run_flag == 0.  pdl: launch with
 // programmatic stream serialization.
+// epi (may be null): in-GEMM epilogue run by the CTA completing each tile group.
 cudaError_t gemm_launch(const CUtensorMap& tmW, const CUtensorMap& tmWlo, const CUtensorMap& tmX,
                         const CUtensorMap& tmXlo, float* part, const GemmShape& s, int ncols,
-                        int mode, const int* run_flag, int* err, cudaStream_t stream, bool pdl);
+                        int mode, const int* run_flag, int* err, cudaStream_t stream, bool pdl,
+                        const GemmEpi* epi = nullptr);
+
+// Segments that complete each epilogue group (host).  group_tiles 0: one group
+// per tile; else groups = tiles / group_tiles and tile t belongs to t % groups
+// (SwiGLU: gate tile t pairs with up tile t + groups).
+void gemm_group_need(const GemmShape& s, const int* tile_c_host, int group_tiles, int* need);
 
 // hi = src with the low 13 mantissa bits cleared (exact in tf32), lo = src - hi.
 cudaError_t split_tf32(const float* src, float* hi, float* lo, size_t n, cudaStream_t stream);

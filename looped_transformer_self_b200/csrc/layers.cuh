@@ -23,7 +23,7 @@
 
 namespace lt {
 
-constexpr int ATT_CH = 256;       // positions per attention split (fixed: batch invariant)
+constexpr int ATT_CH = 128;       // positions per attention split (fixed: batch invariant)
 constexpr int EPI_THREADS = 1024;  // epilogues: many partial reductions in flight per row
 
 // Writes a GEMM operand element.  bf16: rounded.  fp32 with lo != 0: the value
@@ -70,27 +70,43 @@ __global__ void k_embed(const T* __restrict__ E, const int* __restrict__ tok,
     h[(size_t)i * d + n] = to_f<T>(E[(size_t)t * d + n]);
 }
 
-// ---- X = RMSNorm(h) * g for masked rows, zeros elsewhere ----------------------
+// ---- GEMM operand X = g (.) h for masked rows, plus the per-128-feature tile
+// parts of sum(h^2) that the consumers turn into the RMSNorm factor -------------
+// (RMSNorm's per-row factor commutes with the matmul, so the GEMM consumers
+// apply it; masked rows keep whatever X held -- their columns are ignored.)
 template <typename T>
 __global__ void k_stage_norm(const float* __restrict__ h, const int* __restrict__ mask,
-                             const T* __restrict__ g, float eps, int d, T* __restrict__ X,
-                             size_t lo) {
-  __shared__ float red[33];
+                             const T* __restrict__ g, int d, int C, T* __restrict__ X, size_t lo,
+                             float* __restrict__ ssq) {
+  __shared__ float wsum[32];
   pdl_wait();
   pdl_trigger();
   const int i = blockIdx.x;
+  if (!mask[i]) return;
   const float* hr = h + (size_t)i * d;
   T* xr = X + (size_t)i * d;
-  if (!mask[i]) {
-    for (int n = threadIdx.x; n < d; n += blockDim.x) store_act<T>(xr, n, 0.f, lo);
-    return;
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  for (int base = 0; base < d; base += blockDim.x) {
+    const int n = base + threadIdx.x;
+    float sq = 0.f;
+    if (n < d) {
+      const float v = hr[n];
+      store_act<T>(xr, n, to_f<T>(g[n]) * v, lo);
+      sq = v * v;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
+    if (lane == 0) wsum[w] = sq;
+    __syncthreads();
+    if (threadIdx.x < blockDim.x / 128) {
+      const int t = base / 128 + threadIdx.x;
+      if (t * 128 < d) {
+        const int w0 = 4 * threadIdx.x;
+        ssq[(size_t)t * C + i] = wsum[w0] + wsum[w0 + 1] + wsum[w0 + 2] + wsum[w0 + 3];
+      }
+    }
+    __syncthreads();
   }
-  float ss = 0.f;
-  for (int n = threadIdx.x; n < d; n += blockDim.x) ss += hr[n] * hr[n];
-  ss = block_sum(ss, red);
-  const float inv = rsqrtf(ss / d + eps);
-  for (int n = threadIdx.x; n < d; n += blockDim.x)
-    store_act<T>(xr, n, hr[n] * inv * to_f<T>(g[n]), lo);
 }
 
 template <typename T>
@@ -110,11 +126,13 @@ __global__ void k_qkv_epi(const float* __restrict__ part, const GemmShape s, int
                           const int* __restrict__ r_slot, const int* __restrict__ tagsrc,
                           int tag_off, int plane_base, int S, int d, int hd,
                           const float2* __restrict__ rope, T* __restrict__ kv,
-                          float* __restrict__ q, int* err) {
+                          float* __restrict__ q, const float* __restrict__ ssq, int ssq_tiles,
+                          float eps, int* err) {
   pdl_wait();
   pdl_trigger();
   const int i = blockIdx.x;
   if (!mask[i]) return;
+  const float r = inv_rms_parts(ssq, ssq_tiles, C, i, d, eps);
   const int pos = r_pos[i], slot = r_slot[i];
   const int tag = (tagsrc ? tagsrc[i] : 0) + tag_off;
   if (slot < 0 || slot >= S) {
@@ -129,15 +147,16 @@ __global__ void k_qkv_epi(const float* __restrict__ part, const GemmShape s, int
     const int head = p / half, e = p - head * half;
     const int n1 = head * hd + e, n2 = n1 + half;
     const float2 cs = rope[(size_t)pos * half + e];
-    const float q1 = sk_reduce(part, s, C, i, n1), q2 = sk_reduce(part, s, C, i, n2);
+    const float q1 = r * sk_reduce(part, s, C, i, n1), q2 = r * sk_reduce(part, s, C, i, n2);
     q[(size_t)i * d + n1] = q1 * cs.x - q2 * cs.y;
     q[(size_t)i * d + n2] = q2 * cs.x + q1 * cs.y;
-    const float k1 = sk_reduce(part, s, C, i, d + n1), k2 = sk_reduce(part, s, C, i, d + n2);
+    const float k1 = r * sk_reduce(part, s, C, i, d + n1);
+    const float k2 = r * sk_reduce(part, s, C, i, d + n2);
     krow[n1] = from_f<T>(k1 * cs.x - k2 * cs.y);
     krow[n2] = from_f<T>(k2 * cs.x + k1 * cs.y);
   }
   for (int n = threadIdx.x; n < d; n += blockDim.x)
-    vrow[n] = from_f<T>(sk_reduce(part, s, C, i, 2 * d + n));
+    vrow[n] = from_f<T>(r * sk_reduce(part, s, C, i, 2 * d + n));
 }
 
 // ---- vector loads of EPL consecutive cache elements ------------------------------
@@ -189,6 +208,47 @@ __device__ __forceinline__ void load_vec(const T* __restrict__ p, float* out) {
   }
 }
 
+// ---- raw cache words: loaded now, converted when used (keeps 8 positions of K
+// and V in flight per lane without 128 float registers) -----------------------------
+template <typename T, int EPL>
+struct RawVec {
+  static constexpr int BYTES = EPL * (int)sizeof(T);
+  static constexpr int WORDS = BYTES / 4;
+  uint32_t w[WORDS];
+  __device__ __forceinline__ void load(const T* p) {
+    if constexpr (BYTES % 16 == 0) {
+#pragma unroll
+      for (int c = 0; c < BYTES / 16; ++c) {
+        const uint4 u = __ldcg(reinterpret_cast<const uint4*>(p) + c);
+        w[4 * c] = u.x;
+        w[4 * c + 1] = u.y;
+        w[4 * c + 2] = u.z;
+        w[4 * c + 3] = u.w;
+      }
+    } else if constexpr (BYTES % 8 == 0) {
+#pragma unroll
+      for (int c = 0; c < BYTES / 8; ++c) {
+        const uint2 u = __ldcg(reinterpret_cast<const uint2*>(p) + c);
+        w[2 * c] = u.x;
+        w[2 * c + 1] = u.y;
+      }
+    } else {
+#pragma unroll
+      for (int c = 0; c < WORDS; ++c) w[c] = __ldcg(reinterpret_cast<const unsigned int*>(p) + c);
+    }
+  }
+  __device__ __forceinline__ void zero() {
+#pragma unroll
+    for (int c = 0; c < WORDS; ++c) w[c] = 0u;
+  }
+  __device__ __forceinline__ float get(int e) const {
+    if constexpr (sizeof(T) == 2)
+      return __uint_as_float((e & 1) ? (w[e >> 1] & 0xFFFF0000u) : (w[e >> 1] << 16));
+    else
+      return __uint_as_float(w[e]);
+  }
+};
+
 // ---- paged, per-depth, branch-aware decode attention ------------------------------
 // Block (row i, head h, split sp) covers positions [sp*CH, min(sp*CH+CH, pos+1)) of
 // the row's own prefix (committed slots, then the ancestors' and its own slot),
@@ -208,7 +268,7 @@ __device__ __forceinline__ void load_vec(const T* __restrict__ p, float* out) {
 // (planes differ) and siblings never hold each other's positions.  Prefill
 // rows of one chunk do read each other's rows, so prefill runs the separate
 // QKV epilogue first (FUSED = false) and reads q from `q`.
-constexpr int ATT_U = 4;
+constexpr int ATT_U = 8;  // positions per half-warp in flight
 
 template <typename T, int HD, bool FUSED>
 __global__ void __launch_bounds__(128) k_attn(
@@ -218,7 +278,8 @@ __global__ void __launch_bounds__(128) k_attn(
     const int* __restrict__ r_boff, const int* __restrict__ lists, const int* __restrict__ chain,
     int W, int max_splits, float* __restrict__ opart, int* __restrict__ counters,
     T* __restrict__ X, size_t lo, const float* __restrict__ part, const GemmShape qs_shape, int C,
-    const int* __restrict__ r_slot, const float2* __restrict__ rope, int* err) {
+    const int* __restrict__ r_slot, const float2* __restrict__ rope,
+    const float* __restrict__ ssq, int ssq_tiles, float eps, int* err) {
   constexpr int EPL = HD / 16;
   __shared__ float qsm[HD];
   __shared__ int sl[ATT_CH];
@@ -256,25 +317,30 @@ __global__ void __launch_bounds__(128) k_attn(
   if constexpr (FUSED) {
     const int pos = n - 1, half = HD / 2;
     const bool own = sp == ns - 1;  // this block holds the row's own position
+    const float rr = inv_rms_parts(ssq, ssq_tiles, C, i, d, eps);
     const int slot = r_slot[i];
     T* krow = kv + kv_off<T>(plane, slot, 0, S, d) + (size_t)h * HD;
     T* vrow = kv + kv_off<T>(plane, slot, 1, S, d) + (size_t)h * HD;
-    for (int e = threadIdx.x; e < half; e += blockDim.x) {
+    for (int t = threadIdx.x; t < 2 * half; t += blockDim.x) {
+      const int e = t < half ? t : t - half;  // q pairs on the first threads, k pairs on the next
+      const bool is_k = t >= half;
+      if (is_k && !own) continue;
       const float2 cs = rope[(size_t)pos * half + e];
-      const int n1 = h * HD + e, n2 = n1 + half;
-      const float q1 = sk_reduce(part, qs_shape, C, i, n1), q2 = sk_reduce(part, qs_shape, C, i, n2);
-      qsm[e] = q1 * cs.x - q2 * cs.y;
-      qsm[e + half] = q2 * cs.x + q1 * cs.y;
-      if (own) {
-        const float k1 = sk_reduce(part, qs_shape, C, i, d + n1);
-        const float k2 = sk_reduce(part, qs_shape, C, i, d + n2);
-        krow[e] = from_f<T>(k1 * cs.x - k2 * cs.y);
-        krow[e + half] = from_f<T>(k2 * cs.x + k1 * cs.y);
+      const int n1 = (is_k ? d : 0) + h * HD + e, n2 = n1 + half;
+      const float a1 = rr * sk_reduce(part, qs_shape, C, i, n1);
+      const float a2 = rr * sk_reduce(part, qs_shape, C, i, n2);
+      const float r1 = a1 * cs.x - a2 * cs.y, r2 = a2 * cs.x + a1 * cs.y;
+      if (is_k) {
+        krow[e] = from_f<T>(r1);
+        krow[e + half] = from_f<T>(r2);
+      } else {
+        qsm[e] = r1;
+        qsm[e + half] = r2;
       }
     }
     if (own)
       for (int e = threadIdx.x; e < HD; e += blockDim.x)
-        vrow[e] = from_f<T>(sk_reduce(part, qs_shape, C, i, 2 * d + h * HD + e));
+        vrow[e] = from_f<T>(rr * sk_reduce(part, qs_shape, C, i, 2 * d + h * HD + e));
     __syncthreads();  // the own cache row is complete and visible to this block
 #pragma unroll
     for (int e = 0; e < EPL; ++e) qv[e] = qsm[l16 * EPL + e] * scale;
@@ -294,17 +360,17 @@ __global__ void __launch_bounds__(128) k_attn(
   // both half-warps of a warp run the same trip count (the shuffles need the warp)
   for (int tb = (hw & ~1) * ATT_U; tb < cnt; tb += 8 * ATT_U) {
     const int t0 = tb + (hw & 1) * ATT_U;
-    float kx[ATT_U][EPL], vx[ATT_U][EPL];
+    RawVec<T, EPL> kx[ATT_U], vx[ATT_U];
 #pragma unroll
     for (int u = 0; u < ATT_U; ++u) {
       const int t = t0 + u;
       if (t < cnt) {
         const size_t off = (size_t)sl[t] * slot_stride;
-        load_vec<T, EPL>(kbase + off, kx[u]);
-        load_vec<T, EPL>(vbase + off, vx[u]);
+        kx[u].load(kbase + off);
+        vx[u].load(vbase + off);
       } else {
-#pragma unroll
-        for (int e = 0; e < EPL; ++e) kx[u][e] = vx[u][e] = 0.f;
+        kx[u].zero();
+        vx[u].zero();
       }
     }
     float sc[ATT_U];
@@ -312,7 +378,7 @@ __global__ void __launch_bounds__(128) k_attn(
     for (int u = 0; u < ATT_U; ++u) {
       float dot = 0.f;
 #pragma unroll
-      for (int e = 0; e < EPL; ++e) dot += qv[e] * kx[u][e];
+      for (int e = 0; e < EPL; ++e) dot += qv[e] * kx[u].get(e);
       sc[u] = dot;
     }
 #pragma unroll
@@ -335,7 +401,7 @@ __global__ void __launch_bounds__(128) k_attn(
         const float w = __expf(sc[u] - mnew);
         l += w;
 #pragma unroll
-        for (int e = 0; e < EPL; ++e) acc[e] += w * vx[u][e];
+        for (int e = 0; e < EPL; ++e) acc[e] += w * vx[u].get(e);
       }
     }
     m = mnew;
@@ -388,55 +454,6 @@ __global__ void __launch_bounds__(128) k_attn(
     for (int s2 = 0; s2 < ns; ++s2)
       o += __ldcg(base + (size_t)s2 * (HD + 2) + 2 + e) * __expf(__ldcg(base + (size_t)s2 * (HD + 2)) - Mx);
     store_act<T>(X + (size_t)i * d + h * HD, e, o / Lx, lo);
-  }
-}
-
-// ---- residual epilogue: h += scale * (X W^T); optional next RMSNorm -> X ----------
-template <typename T>
-__global__ void k_resid_epi(const float* __restrict__ part, const GemmShape s, int C,
-                            const int* __restrict__ mask, float* __restrict__ h, float scale,
-                            const T* __restrict__ g_next, float eps, int d,
-                            T* __restrict__ X, size_t lo) {
-  __shared__ float red[33];
-  pdl_wait();
-  pdl_trigger();
-  const int i = blockIdx.x;
-  T* xr = X + (size_t)i * d;
-  if (!mask[i]) {
-    if (g_next)
-      for (int n = threadIdx.x; n < d; n += blockDim.x) store_act<T>(xr, n, 0.f, lo);
-    return;
-  }
-  float* hr = h + (size_t)i * d;
-  float ss = 0.f;
-  for (int n = threadIdx.x; n < d; n += blockDim.x) {
-    const float v = hr[n] + scale * sk_reduce(part, s, C, i, n);
-    hr[n] = v;
-    ss += v * v;
-  }
-  if (!g_next) return;
-  ss = block_sum(ss, red);
-  const float inv = rsqrtf(ss / d + eps);
-  for (int n = threadIdx.x; n < d; n += blockDim.x)
-    store_act<T>(xr, n, hr[n] * inv * to_f<T>(g_next[n]), lo);
-}
-
-// ---- SwiGLU epilogue: X = SiLU(gate) * up ------------------------------------------
-template <typename T>
-__global__ void k_gu_epi(const float* __restrict__ part, const GemmShape s, int C,
-                         const int* __restrict__ mask, int f, T* __restrict__ X, size_t lo) {
-  pdl_wait();
-  pdl_trigger();
-  const int i = blockIdx.x;
-  T* xr = X + (size_t)i * f;
-  const bool on = mask[i] != 0;
-  for (int n = blockIdx.y * blockDim.x + threadIdx.x; n < f; n += gridDim.y * blockDim.x) {
-    float a = 0.f;
-    if (on) {
-      const float g = sk_reduce(part, s, C, i, n), u = sk_reduce(part, s, C, i, f + n);
-      a = g / (1.f + __expf(-g)) * u;
-    }
-    store_act<T>(xr, n, a, lo);
   }
 }
 

@@ -242,22 +242,22 @@ def test_tree_edits_match_oracle(tiny):
     sd = D.SpecDecoder(D.OracleRows(LoopedModel(cfg, w, 256)), prompt, cfg.R, dec.d1, dec.d2,
                        dec.max_new, 0.0, 1.0, dec.seed, 256)
     assert sd.committed[-1] == first
-    edits = 0
-    for step in range(1, 21):
+    rollbacks = commits = 0
+    for step in range(1, 25):
         g.step()
         sd.step()
-        if step in (5, 11):
-            root = sd.root().uid
-            uid = max(u for u in sd.branches if u != root)
-            g.rollback_branch(uid)
-            sd.rollback(uid)
-            edits += 1
-        if step == 8 and sd.root().child1 in sd.branches:
+        root = sd.root().uid
+        others = [u for u in sd.branches if u != root]
+        if others and ((step >= 5 and rollbacks == 0) or (step >= 13 and rollbacks == 1)):
+            g.rollback_branch(max(others))
+            sd.rollback(max(others))
+            rollbacks += 1
+        elif step >= 9 and commits == 0 and sd.root().child1 in sd.branches:
             uid = sd.root().child1
             g.commit_branch(uid)
             sd.commit_branch(uid)
-            edits += 1
-    assert edits == 3
+            commits += 1
+    assert rollbacks == 2 and commits == 1
     assert g.read_trace(sd.stats.steps) == sd.trace
     toks, slots = g.read_committed()
     assert toks == sd.committed and slots == sd.cslots
