@@ -32,7 +32,8 @@ extern "C" int lt_gemm_scratch_bytes(int dtype, int n_out, int k, int ncols, siz
   if (!bytes || n_out <= 0 || k <= 0) return LT_ERR_ARG;
   GemmShape s;
   gemm_plan(n_out, k, dtype == LT_F32, sm_count(), &s, nullptr, nullptr);
-  *bytes = align256((size_t)(2 * s.tiles + s.grid) * sizeof(int)) + align256(gemm_part_bytes(s, ncols));
+  *bytes = align256((size_t)gemm_table_ints(n_out, k, dtype == LT_F32, sm_count()) * sizeof(int)) +
+           align256(gemm_part_bytes(s, ncols));
   if (dtype == LT_F32) *bytes += 2 * align256((size_t)n_out * k * 4) + 2 * align256((size_t)ncols * k * 4);
   return LT_OK;
 }
@@ -49,7 +50,7 @@ extern "C" int lt_gemm_rows(int dtype, const void* d_w, const void* d_x, float* 
   if (scratch_bytes < need) return LT_ERR_CAPACITY;
   GemmShape s;
   gemm_plan(n_out, k, f32, sm_count(), &s, nullptr, nullptr);
-  std::vector<int> tab(2 * s.tiles + s.grid);
+  std::vector<int> tab(gemm_table_ints(n_out, k, f32, sm_count()));
   gemm_plan(n_out, k, f32, sm_count(), &s, tab.data(), tab.data() + 2 * s.tiles);
   char* cur = (char*)d_scratch;
   int* d_tab = (int*)cur;
@@ -62,6 +63,7 @@ extern "C" int lt_gemm_rows(int dtype, const void* d_w, const void* d_x, float* 
     return LT_ERR_CUDA;
   s.tile_c = d_tab;
   s.cta_t0 = d_tab + 2 * s.tiles;
+  s.tinfo = reinterpret_cast<const int4*>(d_tab + gemm_tinfo_offset(s));
   CUtensorMap tw, tx, twl, txl;
   const void* w_hi = d_w;
   const void* x_hi = d_x;

@@ -142,30 +142,32 @@ struct GemmShape {
   int jmax;      // max tiles one CTA touches
   const int* tile_c;   // device [2*tiles]: first and last CTA covering tile t
   const int* cta_t0;   // device [grid]: first tile of CTA c
+  const int4* tinfo;   // device [tiles]: (first CTA, last CTA, segment index of the first CTA, 0)
 };
 
 // Sum of the partials of output feature n for row i (fixed CTA order).
-// Partial layout: part[((c * jmax + j) * ncols + i) * 128 + (n % 128)].  The first
-// 8 partials are issued as independent loads (they live in L2), so a reduction
-// costs about one L2 round trip instead of one per partial.
+// Partial layout: part[((c * jmax + j) * ncols + i) * 128 + (n % 128)]: CTA c's
+// j-th tile.  A tile's first CTA may have started in an earlier tile (segment
+// j_lo); every later CTA of the tile starts in it (segment 0).  One table load,
+// then up to 16 partials issued as independent loads: two L2 round trips.
 __device__ __forceinline__ float sk_reduce(const float* __restrict__ part, const GemmShape& s,
                                            int ncols, int i, int n) {
-  constexpr int PB = 8;
+  constexpr int PB = 16;
   const int t = n >> 7, r = n & 127;
-  const int c_lo = __ldg(s.tile_c + 2 * t), c_hi = __ldg(s.tile_c + 2 * t + 1);
+  const int4 ti = __ldg(s.tinfo + t);
+  const size_t row = (size_t)i * 128 + r;
+  const size_t cstride = (size_t)s.jmax * ncols * 128;
   float v[PB];
 #pragma unroll
   for (int k = 0; k < PB; ++k) {
-    const int c = c_lo + k;
-    v[k] = c <= c_hi
-               ? __ldcg(part + (((size_t)c * s.jmax + (t - __ldg(s.cta_t0 + c))) * ncols + i) * 128 + r)
-               : 0.f;
+    const int c = ti.x + k;
+    const size_t off = k == 0 ? ((size_t)ti.x * s.jmax + ti.z) * ncols * 128 : (size_t)c * cstride;
+    v[k] = c <= ti.y ? __ldcg(part + off + row) : 0.f;
   }
   float acc = 0.f;
 #pragma unroll
   for (int k = 0; k < PB; ++k) acc += v[k];
-  for (int c = c_lo + PB; c <= c_hi; ++c)
-    acc += __ldcg(part + (((size_t)c * s.jmax + (t - __ldg(s.cta_t0 + c))) * ncols + i) * 128 + r);
+  for (int c = ti.x + PB; c <= ti.y; ++c) acc += __ldcg(part + (size_t)c * cstride + row);
   return acc;
 }
 
@@ -206,7 +208,14 @@ struct GemmEpi {
 __device__ __forceinline__ float inv_rms_parts(const float* __restrict__ ssq, int tiles,
                                                int ncols, int i, int d, float eps) {
   float s = 0.f;
-  for (int t = 0; t < tiles; ++t) s += __ldcg(ssq + (size_t)t * ncols + i);
+  for (int t0 = 0; t0 < tiles; t0 += 16) {  // 16 independent loads per round
+    float v[16];
+#pragma unroll
+    for (int k = 0; k < 16; ++k)
+      v[k] = t0 + k < tiles ? __ldcg(ssq + (size_t)(t0 + k) * ncols + i) : 0.f;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) s += v[k];
+  }
   return rsqrtf(s / d + eps);
 }
 

@@ -196,7 +196,8 @@ static size_t carve(Handle* H, char* base) {
   GemmShape* shapes[] = {&H->sh_qkv, &H->sh_o, &H->sh_gu, &H->sh_d, &H->sh_head};
   const int dims[5][2] = {{3 * d, d}, {d, d}, {2 * f, d}, {d, f}, {V, d}};
   int tab_ints = 0;
-  for (int k = 0; k < 5; ++k) tab_ints += gemm_table_ints(dims[k][0], dims[k][1], H->f32, gc);
+  for (int k = 0; k < 5; ++k)
+    tab_ints += (gemm_table_ints(dims[k][0], dims[k][1], H->f32, gc) + 3) / 4 * 4;
   H->gemm_tab = cv.take<int>(tab_ints);
   size_t part_floats = 0;
   for (int k = 0; k < 5; ++k) {
@@ -518,8 +519,8 @@ extern "C" int lt_create(const lt_model_config* m, const lt_decode_config* dc, v
   std::vector<int> tab;
   std::vector<int> offs;
   for (int k = 0; k < 5; ++k) {
-    const int n = gemm_table_ints(dims[k][0], dims[k][1], H->f32, gc);
-    std::vector<int> t(n);
+    const int n = (gemm_table_ints(dims[k][0], dims[k][1], H->f32, gc) + 3) / 4 * 4;
+    std::vector<int> t(n, 0);
     gemm_plan(dims[k][0], dims[k][1], H->f32, gc, shapes[k], t.data(),
               t.data() + 2 * shapes[k]->tiles);
     offs.push_back((int)tab.size());
@@ -533,6 +534,7 @@ extern "C" int lt_create(const lt_model_config* m, const lt_decode_config* dc, v
   for (int k = 0; k < 5; ++k) {
     shapes[k]->tile_c = H->gemm_tab + offs[k];
     shapes[k]->cta_t0 = H->gemm_tab + offs[k] + 2 * shapes[k]->tiles;
+    shapes[k]->tinfo = reinterpret_cast<const int4*>(H->gemm_tab + offs[k] + gemm_tinfo_offset(*shapes[k]));
   }
   {  // arrivals that complete each epilogue group (O / down: per tile; gate/up: per pair)
     std::vector<int> need_o(H->ssq_tiles), need_d(H->ssq_tiles), need_gu(f / 128);

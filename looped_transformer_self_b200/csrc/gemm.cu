@@ -531,7 +531,11 @@ static size_t smem_bytes(int ncols, int stages, int nsplit) {
 int gemm_table_ints(int n_out, int k, bool f32, int grid_cap) {
   GemmShape s;
   gemm_plan(n_out, k, f32, grid_cap, &s, nullptr, nullptr);
-  return 2 * s.tiles + s.grid;
+  return 2 * s.tiles + s.grid + 4 * s.tiles + 4;  // tile_c, cta_t0, (pad to 16 B), tinfo
+}
+
+int gemm_tinfo_offset(const GemmShape& s) {  // int offset of tinfo within the table block
+  return ((2 * s.tiles + s.grid + 3) / 4) * 4;
 }
 
 void gemm_plan(int n_out, int k, bool f32, int grid_cap, GemmShape* s, int* tile_c,
@@ -554,6 +558,15 @@ void gemm_plan(int n_out, int k, bool f32, int grid_cap, GemmShape* s, int* tile
     for (int t = 0; t < s->tiles; ++t) {
       tile_c[2 * t] = sk_cta_of(t * s->kch, s->units, s->grid);
       tile_c[2 * t + 1] = sk_cta_of(t * s->kch + s->kch - 1, s->units, s->grid);
+    }
+    // tinfo follows cta_t0 (rounded up to 16 bytes): (c_lo, c_hi, j of c_lo, 0)
+    int* ti = tile_c + ((2 * s->tiles + s->grid + 3) / 4) * 4;
+    for (int t = 0; t < s->tiles; ++t) {
+      const int clo = tile_c[2 * t];
+      ti[4 * t] = clo;
+      ti[4 * t + 1] = tile_c[2 * t + 1];
+      ti[4 * t + 2] = t - sk_u0(clo, s->units, s->grid) / s->kch;
+      ti[4 * t + 3] = 0;
     }
   }
   s->tile_c = nullptr;

@@ -45,10 +45,15 @@ constexpr int GEMM_SMEM_BUDGET = 104 * 1024;
 constexpr int GEMM_L2_PREFETCH_BYTES = 256 * 1024;
 
 // Plans the stream-K split of one weight matrix.  `grid_cap`: CTAs (#SMs).
-// Fills the host copies of the reducer tables (tile_c [2*tiles], cta_t0 [grid]).
+// Fills the host copies of the reducer tables: tile_c [2*tiles], cta_t0 [grid]
+// and, when tile_c_host is given, the tinfo block after them (see gemm_table_ints;
+// the caller sizes tile_c_host with gemm_table_ints).
 void gemm_plan(int n_out, int k, bool f32, int grid_cap, GemmShape* s, int* tile_c_host,
                int* cta_t0_host);
-int gemm_table_ints(int n_out, int k, bool f32, int grid_cap);  // 2*tiles + grid
+// Table block of one shape: tile_c [2*tiles], cta_t0 [grid], pad, tinfo [4*tiles]
+// (int4, 16-byte aligned when the block is).  gemm_plan fills it from tile_c_host.
+int gemm_table_ints(int n_out, int k, bool f32, int grid_cap);
+int gemm_tinfo_offset(const GemmShape& s);
 
 // Encodes a K-major 2-D tensor map (rows x k, box box_rows x 128 bytes, 128B swizzle).
 int make_tmap(CUtensorMap* map, const void* base, bool f32, uint64_t rows, uint64_t k,

@@ -286,31 +286,44 @@ __global__ void __launch_bounds__(128) k_attn(
   __shared__ float hm[8], hl[8];
   __shared__ float hacc[8][HD];
   __shared__ int last;
+  const int i = blockIdx.x, h = blockIdx.y, sp = blockIdx.z;
+  // Row bookkeeping, slot lists and the cache rows of earlier positions were
+  // written by kernels that finished before this grid was launched, so they
+  // are read -- and the block's K/V rows are requested into L2 -- before the
+  // dependency wait, while the QKV GEMM in front of this kernel still runs.
+  const bool on = mask[i] != 0;
+  const int n = on ? r_pos[i] + 1 : 0;
+  const int start = sp * ATT_CH;
+  const int ns = (n + ATT_CH - 1) / ATT_CH;
+  const int cnt = start < n ? min(ATT_CH, n - start) : 0;
+  const int plane = plane_base + (on && tagsrc ? tagsrc[i] : 0) + tag_off;
+  if (cnt > 0) {
+    const int blen = r_blen[i], boff = r_boff[i];
+    for (int t = threadIdx.x; t < cnt; t += blockDim.x) {
+      const int j = start + t;
+      int s = j < blen ? lists[boff + j] : chain[i * W + (j % W)];
+      if (s < 0 || s >= S) {
+        set_err(err, DEV_BAD_INDEX);
+        s = 0;
+      }
+      sl[t] = s;
+      const T* kr = kv + kv_off<T>(plane, s, 0, S, d) + (size_t)h * HD;
+      const T* vr = kv + kv_off<T>(plane, s, 1, S, d) + (size_t)h * HD;
+      asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(kr), "r"((int)(HD * sizeof(T)))
+                   : "memory");
+      asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(vr), "r"((int)(HD * sizeof(T)))
+                   : "memory");
+    }
+  }
   pdl_wait();
   pdl_trigger();
-  const int i = blockIdx.x, h = blockIdx.y, sp = blockIdx.z;
-  if (!mask[i]) {
+  if (!on) {
     if (sp == 0)
       for (int e = threadIdx.x; e < HD; e += blockDim.x)
         store_act<T>(X + (size_t)i * d + h * HD, e, 0.f, lo);
     return;
   }
-  const int n = r_pos[i] + 1;
-  const int start = sp * ATT_CH;
-  if (start >= n) return;
-  const int ns = (n + ATT_CH - 1) / ATT_CH;
-  const int cnt = min(ATT_CH, n - start);
-  const int plane = plane_base + (tagsrc ? tagsrc[i] : 0) + tag_off;
-  const int blen = r_blen[i], boff = r_boff[i];
-  for (int t = threadIdx.x; t < cnt; t += blockDim.x) {
-    const int j = start + t;
-    int s = j < blen ? lists[boff + j] : chain[i * W + (j % W)];
-    if (s < 0 || s >= S) {
-      set_err(err, DEV_BAD_INDEX);
-      s = 0;
-    }
-    sl[t] = s;
-  }
+  if (cnt == 0) return;
   const int hw = threadIdx.x >> 4, l16 = threadIdx.x & 15;
   const float scale = rsqrtf((float)HD);
   float qv[EPL];

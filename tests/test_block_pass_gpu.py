@@ -74,6 +74,9 @@ def test_block_pass_timed_replays_are_stable():
     lists, offs, nslots = _layout(depth, lens, seed=3)
     g = Decoder(cfg, syn.DecodeConfig(1, 2, 0.0, 1.0, 2, 4), syn.make_weights(cfg), max_branches=8,
                 max_ctx=200)
+    pool, _ = g.kv_pool()
+    pool.copy_(torch.from_numpy(syn.random_kv(pool.numel() // cfg.d_model, cfg.d_model, seed=9))
+               .view(pool.shape).to(pool.dtype))
     hid = torch.from_numpy(syn.random_hidden(2, cfg.d_model, seed=1)).cuda()
     ms = g.block_pass(depth, lens, torch.from_numpy(lists).cuda(), offs, hid, iters=5, timed=True)
     assert len(ms) == 5 and all(0 < t < 1000 for t in ms)
