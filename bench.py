@@ -184,13 +184,14 @@ def run_ours(args):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     cfg = syn.MODELS[args.model]
-    n_new = args.n_new
+    n_new = args.n_new or syn.DECODES[f"{args.model}_greedy"].max_new
     dec_g = syn.DECODES[f"{args.model}_greedy"].replace(max_new=n_new, seed=2 + rank)
     prompt = syn.prompt_for(args.model, seed=1 + rank)
     P = len(prompt)
     t_w = time.time()
     weights = syn.make_weights(cfg)
-    g = Decoder(cfg, dec_g, weights, max_branches=16, max_ctx=P + 1 + n_new + 8,
+    C = 16 if cfg.R <= 32 else 32
+    g = Decoder(cfg, dec_g, weights, max_branches=C, max_ctx=P + 1 + n_new + 8,
                 trace_steps=0, device=dev)
     t_w = time.time() - t_w
 
@@ -226,7 +227,7 @@ def run_ours(args):
     ar_ms, ar_toks, ar_st = one_generate(ar=True)
     spec_equal_ar = ar_toks == toks
     g_s = Decoder(cfg, syn.DECODES[f"{args.model}_sample"].replace(max_new=n_new, seed=2 + rank),
-                  None, max_branches=16, max_ctx=P + 1 + n_new + 8, device=dev)
+                  None, max_branches=C, max_ctx=P + 1 + n_new + 8, device=dev)
     g_s.weights = g.weights
     g_s.bind_weights()
     g_s.prefill(prompt)
@@ -271,10 +272,11 @@ def run_ours(args):
             "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": total_ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": WORKLOAD, "parallelism": f"replicas x{ws}",
+            "config": {"workload": WORKLOAD if args.model == "ouro14" else args.model,
+                       "parallelism": f"replicas x{ws}",
                        "l2": "no flush: 2.47 GB of weights per pass exceed the 126 MB L2",
                        "resid_scale": cfg.resid_scale, "agreement_d1_vs_R": agree,
-                       "max_branches": 16},
+                       "max_branches": C, "n_new": n_new, "prompt_len": P},
             "speedup_vs_full_depth_ar": (ar_ms / times[-1]),
             "ar_tokens_per_s": n_new / (ar_ms / 1e3),
             "sampled_tokens_per_s": n_new / (sample_ms / 1e3),
@@ -319,7 +321,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--model", default="ouro14")
-    ap.add_argument("--n-new", type=int, default=1024)
+    ap.add_argument("--n-new", type=int, default=None,
+                    help="decode tokens (default: the model's configured count)")
     ap.add_argument("--no-cpu", action="store_true")
     args = ap.parse_args()
     if args.impl == "reference":

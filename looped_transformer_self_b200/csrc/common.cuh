@@ -171,6 +171,55 @@ __device__ __forceinline__ float sk_reduce(const float* __restrict__ part, const
   return acc;
 }
 
+// Same sum with the tile's table entry already in hand (loaded ahead of time).
+__device__ __forceinline__ float sk_reduce_ti(const float* __restrict__ part, const GemmShape& s,
+                                              int4 ti, int ncols, int i, int n) {
+  constexpr int PB = 16;
+  const int r = n & 127;
+  const size_t row = (size_t)i * 128 + r;
+  const size_t cstride = (size_t)s.jmax * ncols * 128;
+  float v[PB];
+#pragma unroll
+  for (int k = 0; k < PB; ++k) {
+    const int c = ti.x + k;
+    const size_t off = k == 0 ? ((size_t)ti.x * s.jmax + ti.z) * ncols * 128 : (size_t)c * cstride;
+    v[k] = c <= ti.y ? __ldcg(part + off + row) : 0.f;
+  }
+  float acc = 0.f;
+#pragma unroll
+  for (int k = 0; k < PB; ++k) acc += v[k];
+  for (int c = ti.x + PB; c <= ti.y; ++c) acc += __ldcg(part + (size_t)c * cstride + row);
+  return acc;
+}
+
+// Sums of one tile's partials for up to four rows at once (each in fixed CTA
+// order): all loads of a round are independent.
+template <int PB>
+__device__ __forceinline__ void tile_sum4(const float* __restrict__ part, const GemmShape& s,
+                                          int4 ti, int ncols, const int* rows4, int nr, int r,
+                                          float out[4]) {
+  const size_t cstride = (size_t)s.jmax * ncols * 128;
+  const size_t base0 = ((size_t)ti.x * s.jmax + ti.z) * ncols * 128 + r;
+  float v[4][PB];
+#pragma unroll
+  for (int k = 0; k < PB; ++k) {
+    const int c = ti.x + k;
+    const size_t off = k == 0 ? base0 : (size_t)c * cstride + r;
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      v[u][k] = (c <= ti.y && u < nr) ? __ldcg(part + off + (size_t)rows4[u] * 128) : 0.f;
+  }
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    float acc = 0.f;
+#pragma unroll
+    for (int k = 0; k < PB; ++k) acc += v[u][k];
+    out[u] = acc;
+  }
+  for (int c = ti.x + PB; c <= ti.y; ++c)
+    for (int u = 0; u < nr; ++u) out[u] += __ldcg(part + (size_t)c * cstride + r + (size_t)rows4[u] * 128);
+}
+
 // ---- in-GEMM epilogues --------------------------------------------------------------
 // The CTA whose segment completes a group of output tiles (the last to arrive
 // on the group's counter) reduces the group's partials in fixed CTA order and

@@ -295,7 +295,8 @@ static void plan(Handle* H) {
 template <typename T>
 static cudaError_t gemm(Handle* H, const CUtensorMap& tw, const CUtensorMap& twl,
                         const CUtensorMap& tx, const CUtensorMap& txl, const GemmShape& s,
-                        const int* flag, const GemmEpi* epi = nullptr) {
+                        const int* flag, const GemmEpi* epi = nullptr,
+                        const CUtensorMap* next_w = nullptr, const GemmShape* next_s = nullptr) {
   const double esz = H->f32 ? 4.0 : 2.0, split = H->mode == 2 ? 2.0 : 1.0;
   // algorithmic bytes: the weight matrix (both tf32 halves when split), the
   // activation rows and the fp32 result rows
@@ -304,7 +305,7 @@ static cudaError_t gemm(Handle* H, const CUtensorMap& tw, const CUtensorMap& twl
   ProfScope ps(H, H->prof_cat, bytes);
   if (H->counting) H->kernels_per_step++;
   return gemm_launch(tw, twl, tx, txl, H->part, s, H->C, H->mode, flag, &H->D.ctl->err,
-                     H->stream, H->use_pdl, epi);
+                     H->stream, H->use_pdl, epi, next_w, next_s);
 }
 
 template <typename T, int HD>
@@ -314,7 +315,8 @@ static cudaError_t attention(Handle* H, int gl, const int* tagsrc, int tag_off, 
   Dev& D = H->D;
   const int C = H->C, Hn = H->m.n_heads;
   auto kern = fused ? k_attn<T, HD, true> : k_attn<T, HD, false>;
-  return launch(H->use_pdl, kern, dim3(C, Hn, H->max_splits), dim3(128), H->stream,
+  // grid: (head, work item); items = active rows' 128-position splits
+  return launch(H->use_pdl, kern, dim3(Hn, C * H->max_splits), dim3(128), H->stream,
                 (const float*)H->q, (T*)H->kv, H->plane_base[gl], tagsrc, tag_off, H->S,
                 H->m.d_model, Hn, mask, (const int*)D.r_pos, (const int*)D.r_blen,
                 (const int*)D.r_boff, H->lists_override ? H->lists_override : (const int*)D.lists,
@@ -337,7 +339,6 @@ static cudaError_t run_layers(Handle* H, int gl0, int n, int kind, const int* ma
   const int tag_off = kind == 1 ? -1 : 0;
   T* Xd = (T*)H->Xd;
   T* Xo = (T*)H->Xo;
-  T* Xf = (T*)H->Xf;
   GemmEpi eo = {}, egu = {}, ed = {};
   eo.kind = ed.kind = EPI_RESID;
   eo.counters = H->cnt_o;
@@ -367,7 +368,9 @@ static cudaError_t run_layers(Handle* H, int gl0, int n, int kind, const int* ma
     if (l == 0)
       LT_CK(launch(H->use_pdl, k_stage_norm<T>, dim3(C), dim3(EPI_THREADS), H->stream,
                    (const float*)hbuf, mask, (const T*)L.g1, d, C, Xd, H->lo_d, H->ssq));
-    LT_CK(gemm<T>(H, L.tm_qkv, L.tm_qkv_lo, H->tm_Xd, H->tm_Xd_lo, H->sh_qkv, flag));
+    // each GEMM requests the next GEMM's weights into L2 (see k_gemm)
+    LT_CK(gemm<T>(H, L.tm_qkv, L.tm_qkv_lo, H->tm_Xd, H->tm_Xd_lo, H->sh_qkv, flag, nullptr,
+                  &L.tm_o, &H->sh_o));
     if (!fused)
       LT_CK(launch(H->use_pdl, k_qkv_epi<T>, dim3(C), dim3(EPI_THREADS), H->stream,
                    (const float*)H->part, H->sh_qkv, C, mask, (const int*)D.r_pos,
@@ -381,10 +384,14 @@ static cudaError_t run_layers(Handle* H, int gl0, int n, int kind, const int* ma
       default: LT_CK((attention<T, 128>(H, gl, tagsrc, tag_off, mask, Xo, fused))); break;
     }
     eo.g = L.g2;  // O: h += s * o W_o^T; X = g2 (.) h for the gate/up GEMM
-    LT_CK(gemm<T>(H, L.tm_o, L.tm_o_lo, H->tm_Xo, H->tm_Xo_lo, H->sh_o, flag, &eo));
-    LT_CK(gemm<T>(H, L.tm_gu, L.tm_gu_lo, H->tm_Xd, H->tm_Xd_lo, H->sh_gu, flag, &egu));
+    LT_CK(gemm<T>(H, L.tm_o, L.tm_o_lo, H->tm_Xo, H->tm_Xo_lo, H->sh_o, flag, &eo, &L.tm_gu,
+                  &H->sh_gu));
+    LT_CK(gemm<T>(H, L.tm_gu, L.tm_gu_lo, H->tm_Xd, H->tm_Xd_lo, H->sh_gu, flag, &egu, &L.tm_d,
+                  &H->sh_d));
     ed.g = (l + 1 < n) ? H->layers[gl + 1].g1 : nullptr;  // next layer's g1 (.) h
-    LT_CK(gemm<T>(H, L.tm_d, L.tm_d_lo, H->tm_Xf, H->tm_Xf_lo, H->sh_d, flag, &ed));
+    const CUtensorMap* nw = (l + 1 < n) ? &H->layers[gl + 1].tm_qkv : (fused ? &H->tm_head : nullptr);
+    const GemmShape* ns = (l + 1 < n) ? &H->sh_qkv : (fused ? &H->sh_head : nullptr);
+    LT_CK(gemm<T>(H, L.tm_d, L.tm_d_lo, H->tm_Xf, H->tm_Xf_lo, H->sh_d, flag, &ed, nw, ns));
   }
   return cudaSuccess;
 }
@@ -535,6 +542,10 @@ extern "C" int lt_create(const lt_model_config* m, const lt_decode_config* dc, v
     shapes[k]->tile_c = H->gemm_tab + offs[k];
     shapes[k]->cta_t0 = H->gemm_tab + offs[k] + 2 * shapes[k]->tiles;
     shapes[k]->tinfo = reinterpret_cast<const int4*>(H->gemm_tab + offs[k] + gemm_tinfo_offset(*shapes[k]));
+  }
+  if (H->sh_o.jmax > 8 || H->sh_gu.jmax > 8 || H->sh_d.jmax > 8) {  // epilogue table slots
+    delete hd;
+    return LT_ERR_SHAPE;
   }
   {  // arrivals that complete each epilogue group (O / down: per tile; gate/up: per pair)
     std::vector<int> need_o(H->ssq_tiles), need_d(H->ssq_tiles), need_gu(f / 128);

@@ -176,32 +176,32 @@ struct EpiSmem {
   int last;          // group completed by this CTA, or -1
   float inv[64];     // per active row: 1 / rms (SwiGLU)
   float wsum[4][64]; // per warp, per active row: partial sum of squares
+  int4 ti[8][2];     // per segment of this CTA: table entries of its group's tiles
 };
 
 // Residual epilogue of one tile: h += scale * y; X = g (.) h; sum-of-squares part.
 template <typename TX>
 __device__ void epi_resid(const GemmEpi& ep, const float* __restrict__ part, const GemmShape& s,
-                          int ncols, int t, int et, EpiSmem& sm) {
+                          int ncols, int t, int seg, int et, EpiSmem& sm) {
   const int n = t * 128 + et;
   const bool valid = n < s.n_out;
   const int lane = et & 31, w = et >> 5;
+  const int4 ti = sm.ti[seg][0];
   for (int k0 = 0; k0 < sm.nact; k0 += 4) {
-    float y[4];
+    const int nr = min(4, sm.nact - k0);
+    float y[4], h0[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u)  // h rows first: their loads overlap the partials'
+      h0[u] = (valid && u < nr) ? __ldcg(ep.h + (size_t)sm.rows[k0 + u] * ep.d + n) : 0.f;
+    tile_sum4<12>(part, s, ti, ncols, sm.rows + k0, nr, n & 127, y);
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      const int k = k0 + u;
-      y[u] = (valid && k < sm.nact) ? sk_reduce(part, s, ncols, sm.rows[k], n) : 0.f;
-    }
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int k = k0 + u;
-      if (k >= sm.nact) break;
-      const int i = sm.rows[k];
+      if (u >= nr) break;
+      const int i = sm.rows[k0 + u];
       float hv = 0.f;
       if (valid) {
-        float* hp = ep.h + (size_t)i * ep.d + n;
-        hv = *hp + ep.scale * y[u];
-        *hp = hv;
+        hv = h0[u] + ep.scale * y[u];
+        ep.h[(size_t)i * ep.d + n] = hv;
         if (ep.g)
           store_x<TX>(reinterpret_cast<TX*>(ep.X), (size_t)i * ep.d + n, load_g<TX>(ep.g, n) * hv,
                       ep.lo);
@@ -209,7 +209,7 @@ __device__ void epi_resid(const GemmEpi& ep, const float* __restrict__ part, con
       float sq = hv * hv;
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
-      if (lane == 0) sm.wsum[w][k] = sq;
+      if (lane == 0) sm.wsum[w][k0 + u] = sq;
     }
   }
   drain_sync();
@@ -219,30 +219,25 @@ __device__ void epi_resid(const GemmEpi& ep, const float* __restrict__ part, con
   }
 }
 
-// SwiGLU epilogue of one (gate tile, up tile) pair.
+// SwiGLU epilogue of one (gate tile g, up tile g + ffn/128) pair; sm.inv was
+// filled during the mainloop.
 template <typename TX>
 __device__ void epi_swiglu(const GemmEpi& ep, const float* __restrict__ part, const GemmShape& s,
-                           int ncols, int t, int et, EpiSmem& sm) {
-  if (et < sm.nact)
-    sm.inv[et] = inv_rms_parts(ep.ssq_in, ep.ssq_tiles, ncols, sm.rows[et], ep.d, ep.eps);
-  drain_sync();
-  const int n = t * 128 + et;
+                           int ncols, int g, int seg, int et, EpiSmem& sm) {
+  const int n = g * 128 + et;
   if (n >= ep.ffn) return;
-  for (int k0 = 0; k0 < sm.nact; k0 += 2) {
-    float gv[2], uv[2];
+  const int4 tg = sm.ti[seg][0], tu = sm.ti[seg][1];
+  for (int k0 = 0; k0 < sm.nact; k0 += 4) {
+    const int nr = min(4, sm.nact - k0);
+    float gv[4], uv[4];
+    tile_sum4<4>(part, s, tg, ncols, sm.rows + k0, nr, n & 127, gv);
+    tile_sum4<4>(part, s, tu, ncols, sm.rows + k0, nr, n & 127, uv);
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int k = k0 + u;
-      gv[u] = k < sm.nact ? sk_reduce(part, s, ncols, sm.rows[k], n) : 0.f;
-      uv[u] = k < sm.nact ? sk_reduce(part, s, ncols, sm.rows[k], ep.ffn + n) : 0.f;
-    }
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int k = k0 + u;
-      if (k >= sm.nact) break;
-      const float r = sm.inv[k];
+    for (int u = 0; u < 4; ++u) {
+      if (u >= nr) break;
+      const float r = sm.inv[k0 + u];
       const float g = r * gv[u], up = r * uv[u];
-      store_x<TX>(reinterpret_cast<TX*>(ep.X), (size_t)sm.rows[k] * ep.ffn + n,
+      store_x<TX>(reinterpret_cast<TX*>(ep.X), (size_t)sm.rows[k0 + u] * ep.ffn + n,
                   g / (1.f + __expf(-g)) * up, ep.lo);
     }
   }
@@ -260,7 +255,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     k_gemm(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmWlo,
            const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmXlo,
            float* __restrict__ part, const GemmShape s, const int stages,
-           const int* __restrict__ run_flag, int* __restrict__ err, const GemmEpi ep) {
+           const int* __restrict__ run_flag, int* __restrict__ err, const GemmEpi ep,
+           const __grid_constant__ CUtensorMap tmNext, const GemmShape sNext) {
   using TX = typename std::conditional<MODE == 0, __nv_bfloat16, float>::type;
   __shared__ EpiSmem esm;
   constexpr bool TF32 = MODE != 0;
@@ -345,15 +341,25 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       if constexpr (NSPLIT == 2)
         tma_load_2d(a_base + g * SA + A_BYTES, &tmWlo, kx, t * GEMM_BM, full_bar(g), pol_w);
     }
-    // The rest of this CTA's weight range (up to GEMM_L2_PREFETCH_BYTES) goes to
-    // L2 now, so HBM keeps streaming this GEMM's weights while the kernels in
-    // front of it finish; the ring then refills from L2.
+    // The rest of this CTA's weight range goes to L2 now (often already there:
+    // the GEMM in front of this one requested it), and so does this CTA's
+    // slice of the NEXT GEMM's weights (sNext.units > 0), so HBM keeps
+    // streaming weights through this kernel's tail and the kernels that follow
+    // (attention, epilogues) until the next GEMM's ring is filled.
     const int nl2 = min(u1 - u0, npre + GEMM_L2_PREFETCH_BYTES / (int)SA);
     for (int g = npre; g < nl2; ++g) {
       const int uu = u0 + g, t = uu / s.kch;
       const int kx = (uu - t * s.kch) * BKE;
       tma_prefetch_l2(&tmW, kx, t * GEMM_BM);
       if constexpr (NSPLIT == 2) tma_prefetch_l2(&tmWlo, kx, t * GEMM_BM);
+    }
+    if (sNext.units > 0 && c < sNext.grid) {
+      const int v0 = sk_u0(c, sNext.units, sNext.grid), v1 = sk_u0(c + 1, sNext.units, sNext.grid);
+      const int vend = min(v1, v0 + GEMM_L2_PREFETCH_BYTES / (int)A_BYTES);
+      for (int uu = v0; uu < vend; ++uu) {
+        const int t = uu / sNext.kch;
+        tma_prefetch_l2(&tmNext, (uu - t * sNext.kch) * BKE, t * GEMM_BM);
+      }
     }
   }
   pdl_wait();
@@ -451,11 +457,30 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     // ---------------- drain: TMEM -> fp32 partials (+ group epilogue) ----------------
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     const int et = threadIdx.x - 64;  // 0..127 over the drain warps
-    if (ep.kind != EPI_NONE && et == 0) {
-      int na = 0;
-      for (int i = 0; i < NC; ++i)
-        if (ep.mask[i]) esm.rows[na++] = i;
-      esm.nact = na;
+    if (ep.kind != EPI_NONE) {
+      if (et == 0) {
+        int na = 0;
+        for (int i = 0; i < NC; ++i)
+          if (ep.mask[i]) esm.rows[na++] = i;
+        esm.nact = na;
+      }
+      // table entries of every group this CTA may complete (static tables)
+      const int t0 = u0 / s.kch, nseg = (u1 - 1) / s.kch - t0 + 1;
+      if (et < nseg && et < 8) {
+        const int t = t0 + et;
+        if (ep.kind == EPI_SWIGLU) {
+          const int groups = ep.ffn / GEMM_BM, g = t % groups;
+          esm.ti[et][0] = __ldg(s.tinfo + g);
+          esm.ti[et][1] = __ldg(s.tinfo + g + groups);
+        } else {
+          esm.ti[et][0] = __ldg(s.tinfo + t);
+        }
+      }
+      drain_sync();
+      // the SwiGLU's RMSNorm factors (sums of squares written by the GEMM in
+      // front of this one) are ready now, long before the first accumulator
+      if (ep.kind == EPI_SWIGLU && et < esm.nact)
+        esm.inv[et] = inv_rms_parts(ep.ssq_in, ep.ssq_tiles, NC, esm.rows[et], ep.d, ep.eps);
     }
     int seg = 0;
     for (int u = u0; u < u1; ++seg) {
@@ -475,21 +500,26 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 #pragma unroll
       for (int i = 0; i < NC; ++i) dst[(size_t)i * GEMM_BM] = __uint_as_float(r[i]);
       if (ep.kind != EPI_NONE) {
-        // publish this segment; the arrival that completes the group runs its epilogue
-        __threadfence();
+        // publish this segment; the arrival that completes the group runs its
+        // epilogue.  The barrier orders the drain threads' partial stores before
+        // thread 0's acq_rel atomic (cumulativity), whose acquire side makes the
+        // other CTAs' partials visible to the whole group after the next barrier.
         drain_sync();
         if (et == 0) {
           const int grp = ep.kind == EPI_SWIGLU ? t % (ep.ffn / GEMM_BM) : t;
-          const int old = atomicAdd(ep.counters + grp, 1);
+          int old;
+          asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], 1;"
+                       : "=r"(old)
+                       : "l"(ep.counters + grp)
+                       : "memory");
           esm.last = (old + 1 == ep.need[grp]) ? grp : -1;
           if (esm.last >= 0) ep.counters[grp] = 0;
         }
         drain_sync();
         const int grp = esm.last;
         if (grp >= 0) {
-          __threadfence();
-          if (ep.kind == EPI_RESID) epi_resid<TX>(ep, part, s, NC, grp, et, esm);
-          else epi_swiglu<TX>(ep, part, s, NC, grp, et, esm);
+          if (ep.kind == EPI_RESID) epi_resid<TX>(ep, part, s, NC, grp, seg, et, esm);
+          else epi_swiglu<TX>(ep, part, s, NC, grp, seg, et, esm);
         }
         drain_sync();
       }
@@ -625,7 +655,8 @@ template <int MODE, int NC>
 static cudaError_t launch_t(const CUtensorMap& tmW, const CUtensorMap& tmWlo,
                             const CUtensorMap& tmX, const CUtensorMap& tmXlo, float* part,
                             const GemmShape& s, const int* run_flag, int* err,
-                            cudaStream_t stream, bool pdl, const GemmEpi& ep) {
+                            cudaStream_t stream, bool pdl, const GemmEpi& ep,
+                            const CUtensorMap& tmN, const GemmShape& sN) {
   const int nsplit = MODE == 2 ? 2 : 1;
   const int stages = stages_for(NC, nsplit);
   const size_t smem = smem_bytes(NC, stages, nsplit);
@@ -647,21 +678,26 @@ static cudaError_t launch_t(const CUtensorMap& tmW, const CUtensorMap& tmWlo,
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
   return cudaLaunchKernelEx(&cfg, k_gemm<MODE, NC>, tmW, tmWlo, tmX, tmXlo, part, s, stages,
-                            run_flag, err, ep);
+                            run_flag, err, ep, tmN, sN);
 }
 
 cudaError_t gemm_launch(const CUtensorMap& tmW, const CUtensorMap& tmWlo, const CUtensorMap& tmX,
                         const CUtensorMap& tmXlo, float* part, const GemmShape& s, int ncols,
                         int mode, const int* run_flag, int* err, cudaStream_t stream, bool pdl,
-                        const GemmEpi* epi) {
+                        const GemmEpi* epi, const CUtensorMap* next_w,
+                        const GemmShape* next_s) {
   GemmEpi none = {};
   none.kind = EPI_NONE;
   const GemmEpi& ep = epi ? *epi : none;
+  GemmShape no_next = {};
+  const bool has_next = next_w && next_s && mode != 2;
+  const GemmShape& sN = has_next ? *next_s : no_next;
+  const CUtensorMap& tmN = has_next ? *next_w : tmW;
 #define LT_GEMM_CASE(N)                                                                      \
   case N:                                                                                    \
-    return mode == 2   ? launch_t<2, N>(tmW, tmWlo, tmX, tmXlo, part, s, run_flag, err, stream, pdl, ep) \
-           : mode == 1 ? launch_t<1, N>(tmW, tmWlo, tmX, tmXlo, part, s, run_flag, err, stream, pdl, ep) \
-                       : launch_t<0, N>(tmW, tmWlo, tmX, tmXlo, part, s, run_flag, err, stream, pdl, ep);
+    return mode == 2   ? launch_t<2, N>(tmW, tmWlo, tmX, tmXlo, part, s, run_flag, err, stream, pdl, ep, tmN, sN) \
+           : mode == 1 ? launch_t<1, N>(tmW, tmWlo, tmX, tmXlo, part, s, run_flag, err, stream, pdl, ep, tmN, sN) \
+                       : launch_t<0, N>(tmW, tmWlo, tmX, tmXlo, part, s, run_flag, err, stream, pdl, ep, tmN, sN);
   switch (ncols) {
     LT_GEMM_CASE(8)
     LT_GEMM_CASE(16)

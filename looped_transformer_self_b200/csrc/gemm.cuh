@@ -36,13 +36,15 @@ namespace lt {
 constexpr int GEMM_BM = 128;            // output features per tile (MMA M)
 constexpr int GEMM_CHUNK_BYTES = 128;   // K bytes per stage (one 128B-swizzle row)
 constexpr int GEMM_THREADS = 192;       // warp 0: TMA, warp 1: MMA, warps 2-5: drain
-// Shared memory per CTA for the TMA ring: ~100 KB keeps >= 4 stages (>= 64 KB of
-// weight tiles in flight per SM, well above what HBM latency x bandwidth needs)
-// and lets the next GEMM's CTA become resident, and prefetch, while this one drains.
+// Shared memory per CTA for the TMA ring (5 stages of 18 KB at 16 rows).  A
+// ring this size lets the next GEMM's CTA be resident on the same SM and fill
+// its own ring before its dependency wait, which measured better than a deeper
+// ring with one CTA per SM.
 constexpr int GEMM_SMEM_BUDGET = 104 * 1024;
-// Weight bytes per CTA requested into L2 ahead of the ring (148 CTAs: ~37 MB,
-// so two GEMMs in flight stay well inside the 126 MB L2).
-constexpr int GEMM_L2_PREFETCH_BYTES = 256 * 1024;
+// Weight bytes per CTA requested into L2 ahead of use, for this GEMM's range
+// beyond the ring and for the next GEMM's slice (148 CTAs: <= 47 MB each, well
+// inside the 126 MB L2).
+constexpr int GEMM_L2_PREFETCH_BYTES = 320 * 1024;
 
 // Plans the stream-K split of one weight matrix.  `grid_cap`: CTAs (#SMs).
 // Fills the host copies of the reducer tables: tile_c [2*tiles], cta_t0 [grid]
@@ -64,10 +66,13 @@ int make_tmap(CUtensorMap* map, const void* base, bool f32, uint64_t rows, uint6
 // (device, may be null): skip when *run_flag == 0.  pdl: launch with
 // programmatic stream serialization.
 // epi (may be null): in-GEMM epilogue run by the CTA completing each tile group.
+// next_w / next_s (may be null): the weights of the GEMM that follows, whose
+// slice each CTA requests into L2.
 cudaError_t gemm_launch(const CUtensorMap& tmW, const CUtensorMap& tmWlo, const CUtensorMap& tmX,
                         const CUtensorMap& tmXlo, float* part, const GemmShape& s, int ncols,
                         int mode, const int* run_flag, int* err, cudaStream_t stream, bool pdl,
-                        const GemmEpi* epi = nullptr);
+                        const GemmEpi* epi = nullptr, const CUtensorMap* next_w = nullptr,
+                        const GemmShape* next_s = nullptr);
 
 // Segments that complete each epilogue group (host).  group_tiles 0: one group
 // per tile; else groups = tiles / group_tiles and tile t belongs to t % groups

@@ -286,18 +286,43 @@ __global__ void __launch_bounds__(128) k_attn(
   __shared__ float hm[8], hl[8];
   __shared__ float hacc[8][HD];
   __shared__ int last;
-  const int i = blockIdx.x, h = blockIdx.y, sp = blockIdx.z;
-  // Row bookkeeping, slot lists and the cache rows of earlier positions were
-  // written by kernels that finished before this grid was launched, so they
-  // are read -- and the block's K/V rows are requested into L2 -- before the
-  // dependency wait, while the QKV GEMM in front of this kernel still runs.
-  const bool on = mask[i] != 0;
-  const int n = on ? r_pos[i] + 1 : 0;
+  __shared__ int s_item[3];
+  // Block (head h, item w): items are the active rows' splits, rows in order,
+  // so the work sits in the first blocks of the grid (blocks past the last
+  // item only wait and exit).  Row bookkeeping, slot lists, the cache rows of
+  // earlier positions and (fused) the RMSNorm sums of squares were written by
+  // kernels that finished before this grid was launched: they are read -- and
+  // the block's K/V rows are requested into L2 -- before the dependency wait,
+  // while the QKV GEMM in front of this kernel still runs.
+  const int h = blockIdx.x, w = blockIdx.y;
+  if (threadIdx.x == 0) {
+    int acc = 0, row = -1, spl = 0, nsr = 0;
+#pragma unroll 8
+    for (int k = 0; k < C; ++k) {
+      const int nk = mask[k] ? (r_pos[k] + ATT_CH) / ATT_CH : 0;
+      if (row < 0 && w < acc + nk) {
+        row = k;
+        spl = w - acc;
+        nsr = nk;
+      }
+      acc += nk;
+    }
+    s_item[0] = row;
+    s_item[1] = spl;
+    s_item[2] = nsr;
+  }
+  __syncthreads();
+  const int i = s_item[0], sp = s_item[1], ns = s_item[2];
+  if (i < 0) {
+    pdl_wait();
+    pdl_trigger();
+    return;
+  }
+  const int n = r_pos[i] + 1;
   const int start = sp * ATT_CH;
-  const int ns = (n + ATT_CH - 1) / ATT_CH;
-  const int cnt = start < n ? min(ATT_CH, n - start) : 0;
-  const int plane = plane_base + (on && tagsrc ? tagsrc[i] : 0) + tag_off;
-  if (cnt > 0) {
+  const int cnt = min(ATT_CH, n - start);
+  const int plane = plane_base + (tagsrc ? tagsrc[i] : 0) + tag_off;
+  {
     const int blen = r_blen[i], boff = r_boff[i];
     for (int t = threadIdx.x; t < cnt; t += blockDim.x) {
       const int j = start + t;
@@ -315,33 +340,50 @@ __global__ void __launch_bounds__(128) k_attn(
                    : "memory");
     }
   }
+  // fused prologue inputs that do not depend on the QKV GEMM
+  const int half = HD / 2;
+  const bool own = sp == ns - 1;  // this block holds the row's own position
+  float rr = 1.f;
+  float2 cs = make_float2(1.f, 0.f);
+  int4 tiA = make_int4(0, -1, 0, 0), tiB = tiA, tiV = tiA;
+  int nA = 0, nB = 0, nV = 0;
+  bool is_k = false;
+  if constexpr (FUSED) {
+    rr = inv_rms_parts(ssq, ssq_tiles, C, i, d, eps);
+    const int t = threadIdx.x;
+    if (t < 2 * half) {
+      const int e = t < half ? t : t - half;
+      is_k = t >= half;
+      nA = (is_k ? d : 0) + h * HD + e;
+      nB = nA + half;
+      tiA = __ldg(qs_shape.tinfo + (nA >> 7));
+      tiB = __ldg(qs_shape.tinfo + (nB >> 7));
+      cs = rope[(size_t)(n - 1) * half + e];
+    }
+    if (t < HD) {
+      nV = 2 * d + h * HD + t;
+      tiV = __ldg(qs_shape.tinfo + (nV >> 7));
+    }
+  }
   pdl_wait();
   pdl_trigger();
-  if (!on) {
-    if (sp == 0)
-      for (int e = threadIdx.x; e < HD; e += blockDim.x)
-        store_act<T>(X + (size_t)i * d + h * HD, e, 0.f, lo);
-    return;
-  }
-  if (cnt == 0) return;
   const int hw = threadIdx.x >> 4, l16 = threadIdx.x & 15;
   const float scale = rsqrtf((float)HD);
   float qv[EPL];
   if constexpr (FUSED) {
-    const int pos = n - 1, half = HD / 2;
-    const bool own = sp == ns - 1;  // this block holds the row's own position
-    const float rr = inv_rms_parts(ssq, ssq_tiles, C, i, d, eps);
     const int slot = r_slot[i];
     T* krow = kv + kv_off<T>(plane, slot, 0, S, d) + (size_t)h * HD;
     T* vrow = kv + kv_off<T>(plane, slot, 1, S, d) + (size_t)h * HD;
-    for (int t = threadIdx.x; t < 2 * half; t += blockDim.x) {
-      const int e = t < half ? t : t - half;  // q pairs on the first threads, k pairs on the next
-      const bool is_k = t >= half;
-      if (is_k && !own) continue;
-      const float2 cs = rope[(size_t)pos * half + e];
-      const int n1 = (is_k ? d : 0) + h * HD + e, n2 = n1 + half;
-      const float a1 = rr * sk_reduce(part, qs_shape, C, i, n1);
-      const float a2 = rr * sk_reduce(part, qs_shape, C, i, n2);
+    const int t = threadIdx.x;
+    float a1 = 0.f, a2 = 0.f, av = 0.f;
+    const bool do_pair = t < 2 * half && (!is_k || own);
+    if (do_pair) {
+      a1 = rr * sk_reduce_ti(part, qs_shape, tiA, C, i, nA);
+      a2 = rr * sk_reduce_ti(part, qs_shape, tiB, C, i, nB);
+    }
+    if (own && t < HD) av = rr * sk_reduce_ti(part, qs_shape, tiV, C, i, nV);
+    if (do_pair) {
+      const int e = t < half ? t : t - half;
       const float r1 = a1 * cs.x - a2 * cs.y, r2 = a2 * cs.x + a1 * cs.y;
       if (is_k) {
         krow[e] = from_f<T>(r1);
@@ -351,9 +393,7 @@ __global__ void __launch_bounds__(128) k_attn(
         qsm[e + half] = r2;
       }
     }
-    if (own)
-      for (int e = threadIdx.x; e < HD; e += blockDim.x)
-        vrow[e] = from_f<T>(rr * sk_reduce(part, qs_shape, C, i, 2 * d + h * HD + e));
+    if (own && t < HD) vrow[t] = from_f<T>(av);
     __syncthreads();  // the own cache row is complete and visible to this block
 #pragma unroll
     for (int e = 0; e < EPL; ++e) qv[e] = qsm[l16 * EPL + e] * scale;

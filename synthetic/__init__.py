@@ -113,7 +113,9 @@ DECODES: Dict[str, DecodeConfig] = {
     "ouro14_greedy": DecodeConfig(1, 2, 0.0, 1.0, 2, 1024),
     "ouro14_sample": DecodeConfig(1, 2, 1.0, 0.95, 2, 1024),
     "huginn35_greedy": DecodeConfig(8, 16, 0.0, 1.0, 2, 512),
+    "huginn35_sample": DecodeConfig(8, 16, 1.0, 0.95, 2, 512),
     "ouro26_greedy": DecodeConfig(1, 2, 0.0, 1.0, 2, 2048),
+    "ouro26_sample": DecodeConfig(1, 2, 1.0, 0.95, 2, 2048),
 }
 
 PROMPT_LEN = {"tiny": 32, "tiny16": 32, "ouro14": 512, "huginn35": 256, "ouro26": 4096}
