@@ -143,9 +143,14 @@ int lt_decode_step(lt_handle* h, int ar_mode, int32_t* h_tok, int* n_committed);
  *     freeing their KV slots; its parent forgets the child.
  *   lt_commit_branch: commit the token of `uid`, which must be a child of the
  *     root, WITHOUT full-depth verification (logged with source 3); every
- *     branch outside its subtree is pruned and it becomes the root.
- * Errors: LT_ERR_ARG for an unknown uid, the root, or (commit) a non-child;
- * LT_ERR_STATE when no decode is in progress.
+ *     branch outside its subtree is pruned and it becomes the root.  The old
+ *     root has not run all R loop iterations yet, and later rows attend to
+ *     its position at every depth, so it stays in the table as a retiring
+ *     entry (parent -2 in lt_read_branch_table): it keeps iterating with the
+ *     batch and taking its readouts (which write its coda cache rows), decides
+ *     nothing, and leaves after its R-th iteration.
+ * Errors: LT_ERR_ARG for an unknown uid, the root, a retiring entry, or
+ * (commit) a non-child; LT_ERR_STATE when no decode is in progress.
  */
 int lt_rollback_branch(lt_handle* h, int32_t uid);
 int lt_commit_branch(lt_handle* h, int32_t uid);
@@ -178,6 +183,7 @@ typedef struct {
   int gemm_core_launches;
   double gemm_other_ms;     /* prelude / coda / LM-head GEMMs */
   int gemm_other_launches;
+  double gemm_other_bytes;
   double attn_ms;           /* attention + split combine */
   int attn_launches;
   double kv_bytes;          /* KV read + written by the shared-block layers */

@@ -67,7 +67,8 @@ class ProfileC(ctypes.Structure):
     _fields_ = [("steps", _i), ("rows", _i), ("step_ms", ctypes.c_double),
                 ("gemm_core_ms", ctypes.c_double), ("gemm_core_bytes", ctypes.c_double),
                 ("gemm_core_launches", _i), ("gemm_other_ms", ctypes.c_double),
-                ("gemm_other_launches", _i), ("attn_ms", ctypes.c_double),
+                ("gemm_other_launches", _i), ("gemm_other_bytes", ctypes.c_double),
+                ("attn_ms", ctypes.c_double),
                 ("attn_launches", _i), ("kv_bytes", ctypes.c_double),
                 ("weight_bytes_core", ctypes.c_double)]
 
@@ -181,7 +182,10 @@ class Decoder:
     non-default CUDA stream, owned by this object."""
 
     def __init__(self, cfg, dec, weights=None, max_branches=16, max_ctx=None, trace_steps=0,
-                 second_mode=0, device="cuda"):
+                 second_mode=0, device="cuda", workspace_fill=None):
+        """workspace_fill: a byte value written over the whole workspace before
+        lt_create (tests use it to show that no state is read before it is
+        written); None leaves the allocation as it comes."""
         import numpy as np
         self.np = np
         self.cfg, self.dec = cfg, dec
@@ -195,6 +199,9 @@ class Decoder:
         check(lib().lt_workspace_bytes(ctypes.byref(self.mc), ctypes.byref(self.dc),
                                        ctypes.byref(need)), "lt_workspace_bytes")
         self.workspace = torch.empty(need.value, dtype=torch.uint8, device=self.device)
+        if workspace_fill is not None:
+            self.workspace.fill_(workspace_fill)
+            torch.cuda.synchronize(self.device)
         h = _vp()
         check(lib().lt_create(ctypes.byref(self.mc), ctypes.byref(self.dc),
                               self.workspace.data_ptr(), need.value, self.stream.cuda_stream,

@@ -31,8 +31,9 @@ using namespace lt;
 extern "C" int lt_gemm_scratch_bytes(int dtype, int n_out, int k, int ncols, size_t* bytes) {
   if (!bytes || n_out <= 0 || k <= 0) return LT_ERR_ARG;
   GemmShape s;
-  gemm_plan(n_out, k, dtype == LT_F32, sm_count(), &s, nullptr, nullptr);
-  *bytes = align256((size_t)gemm_table_ints(n_out, k, dtype == LT_F32, sm_count()) * sizeof(int)) +
+  gemm_plan(n_out, k, dtype == LT_F32, ncols, sm_count(), &s, nullptr, nullptr);
+  *bytes = align256((size_t)gemm_table_ints(n_out, k, dtype == LT_F32, ncols, sm_count()) *
+                    sizeof(int)) +
            align256(gemm_part_bytes(s, ncols));
   if (dtype == LT_F32) *bytes += 2 * align256((size_t)n_out * k * 4) + 2 * align256((size_t)ncols * k * 4);
   return LT_OK;
@@ -49,9 +50,9 @@ extern "C" int lt_gemm_rows(int dtype, const void* d_w, const void* d_x, float* 
   lt_gemm_scratch_bytes(dtype, n_out, k, ncols, &need);
   if (scratch_bytes < need) return LT_ERR_CAPACITY;
   GemmShape s;
-  gemm_plan(n_out, k, f32, sm_count(), &s, nullptr, nullptr);
-  std::vector<int> tab(gemm_table_ints(n_out, k, f32, sm_count()));
-  gemm_plan(n_out, k, f32, sm_count(), &s, tab.data(), tab.data() + 2 * s.tiles);
+  gemm_plan(n_out, k, f32, ncols, sm_count(), &s, nullptr, nullptr);
+  std::vector<int> tab(gemm_table_ints(n_out, k, f32, ncols, sm_count()));
+  gemm_plan(n_out, k, f32, ncols, sm_count(), &s, tab.data(), tab.data() + 2 * s.tiles);
   char* cur = (char*)d_scratch;
   int* d_tab = (int*)cur;
   cur += align256(tab.size() * sizeof(int));
@@ -64,7 +65,7 @@ extern "C" int lt_gemm_rows(int dtype, const void* d_w, const void* d_x, float* 
   s.tile_c = d_tab;
   s.cta_t0 = d_tab + 2 * s.tiles;
   s.tinfo = reinterpret_cast<const int4*>(d_tab + gemm_tinfo_offset(s));
-  CUtensorMap tw, tx, twl, txl;
+  GemmOperand tw, tx, twl, txl;
   const void* w_hi = d_w;
   const void* x_hi = d_x;
   if (f32) {  // fp32 operands run as split tf32 (hi + lo pairs)
@@ -80,11 +81,11 @@ extern "C" int lt_gemm_rows(int dtype, const void* d_w, const void* d_x, float* 
       return LT_ERR_CUDA;
     w_hi = wh;
     x_hi = xh;
-    if (make_tmap(&twl, wl, true, n_out, k, GEMM_BM) != 0) return LT_ERR_SHAPE;
-    if (make_tmap(&txl, xl, true, ncols, k, ncols) != 0) return LT_ERR_SHAPE;
+    if (make_operand(&twl, wl, true, n_out, k, GEMM_BM, s.kc) != 0) return LT_ERR_SHAPE;
+    if (make_operand(&txl, xl, true, ncols, k, ncols, s.kc) != 0) return LT_ERR_SHAPE;
   }
-  if (make_tmap(&tw, w_hi, f32, n_out, k, GEMM_BM) != 0) return LT_ERR_SHAPE;
-  if (make_tmap(&tx, x_hi, f32, ncols, k, ncols) != 0) return LT_ERR_SHAPE;
+  if (make_operand(&tw, w_hi, f32, n_out, k, GEMM_BM, s.kc) != 0) return LT_ERR_SHAPE;
+  if (make_operand(&tx, x_hi, f32, ncols, k, ncols, s.kc) != 0) return LT_ERR_SHAPE;
   if (!f32) {
     twl = tw;
     txl = tx;

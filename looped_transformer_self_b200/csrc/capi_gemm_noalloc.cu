@@ -66,9 +66,9 @@ extern "C" int lt_gemm_rows_noalloc(int dtype, const void* d_w, const void* d_x,
   }
   GemmShape s;
   const int grid_cap = sm_count_dev(dev);
-  gemm_plan(n_out, k, false, grid_cap, &s, nullptr, nullptr);
-  std::vector<int> tab(gemm_table_ints(n_out, k, false, grid_cap));
-  gemm_plan(n_out, k, false, grid_cap, &s, tab.data(), tab.data() + 2 * s.tiles);
+  gemm_plan(n_out, k, false, ncols, grid_cap, &s, nullptr, nullptr);
+  std::vector<int> tab(gemm_table_ints(n_out, k, false, ncols, grid_cap));
+  gemm_plan(n_out, k, false, ncols, grid_cap, &s, tab.data(), tab.data() + 2 * s.tiles);
   const size_t tab_bytes = align256(tab.size() * sizeof(int));
   const size_t need = tab_bytes + gemm_part_bytes(s, ncols);
   if (need > (size_t)LT_NOALLOC_SCRATCH_BYTES) return LT_ERR_CAPACITY;
@@ -83,9 +83,9 @@ extern "C" int lt_gemm_rows_noalloc(int dtype, const void* d_w, const void* d_x,
   s.tile_c = d_tab;
   s.cta_t0 = d_tab + 2 * s.tiles;
   s.tinfo = reinterpret_cast<const int4*>(d_tab + gemm_tinfo_offset(s));
-  CUtensorMap tw, tx;
-  if (make_tmap(&tw, d_w, false, n_out, k, GEMM_BM) != 0) return LT_ERR_SHAPE;
-  if (make_tmap(&tx, d_x, false, ncols, k, ncols) != 0) return LT_ERR_SHAPE;
+  GemmOperand tw, tx;
+  if (make_operand(&tw, d_w, false, n_out, k, GEMM_BM, s.kc) != 0) return LT_ERR_SHAPE;
+  if (make_operand(&tx, d_x, false, ncols, k, ncols, s.kc) != 0) return LT_ERR_SHAPE;
   if (gemm_launch(tw, tw, tx, tx, part, s, ncols, 0, nullptr, nullptr, st, false) != cudaSuccess)
     return LT_ERR_CUDA;
   dim3 grid((n_out + 255) / 256, ncols);

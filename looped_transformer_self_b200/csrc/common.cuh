@@ -135,7 +135,10 @@ __host__ __device__ __forceinline__ int sk_cta_of(int u, int U, int G) {
 struct GemmShape {
   int n_out;     // output features (MMA M side, tiled by 128)
   int k;         // reduction length
-  int kch;       // k-chunks of BK elements
+  int kch;       // stream-K units per tile (groups of kc k-chunks)
+  int kc;        // k-chunks (128 bytes of K each) per unit: one TMA request per operand
+  int nch;       // k-chunks per tile, ceil(K / chunk)
+  int nfull;     // k-chunks that lie wholly inside K (units within them load as one 3-D box)
   int tiles;     // ceil(n_out / 128)
   int units;     // tiles * kch
   int grid;      // CTAs (<= units)
@@ -233,7 +236,8 @@ enum EpiKind : int { EPI_NONE = 0, EPI_RESID = 1, EPI_SWIGLU = 2 };
 
 struct GemmEpi {
   int kind;
-  int* counters;       // [groups] arrivals, zero between launches (the last arrival resets)
+  unsigned long long* counters;  // [groups] segment arrivals, monotonic over launches (a
+                                // launch's arrivals take a group from k*need to (k+1)*need)
   const int* need;     // [groups] segments that complete a group
   const int* mask;     // [ncols] rows taking part
   // EPI_RESID (group = one tile of h's features):

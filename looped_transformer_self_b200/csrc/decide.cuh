@@ -299,6 +299,14 @@ __device__ __forceinline__ float residual_into(const float* __restrict__ mu,
   return Z;
 }
 
+// Parent value of a retiring entry: a former root left behind by an external
+// commit.  It keeps running one iteration per step and its readouts, so its
+// committed position gets its block and coda cache rows at every depth before
+// any later row reads them, but it decides nothing (k_decide skips it), is
+// never pruned, and leaves the table (keeping its slot, which holds a
+// committed position) after its R-th iteration.
+constexpr int BK_RETIRING = -2;
+
 __global__ void __launch_bounds__(1024) k_decide(Dev D) {
   __shared__ float sk[33];
   __shared__ int si[33];
@@ -307,7 +315,8 @@ __global__ void __launch_bounds__(1024) k_decide(Dev D) {
   pdl_trigger();
   Ctl* c = D.ctl;
   const int i = blockIdx.x;
-  if (c->finished || !D.m_ro[i]) return;
+  // rows without a readout, and retiring entries, decide nothing
+  if (c->finished || !D.m_ro[i] || D.b_parent[i] == BK_RETIRING) return;
   const int r = D.r_depth[i];
   const int uid = D.b_uid[i];
   const bool ar = c->ar_mode != 0;
@@ -531,7 +540,8 @@ __device__ void bk_logic(BookSmem& b, const Dev& D, Ctl& c, int mode, int arg) {
     int root = -1;
     for (int k = 0; k < C; ++k)
       if (b.alive[k] && b.pos[k] == c.L - 1) root = k;
-    if (e < 0 || root < 0 || e == root || (mode == 3 && b.parent[e] != b.uid[root])) {
+    if (e < 0 || root < 0 || e == root || b.parent[e] == BK_RETIRING ||
+        (mode == 3 && b.parent[e] != b.uid[root])) {
       set_err(&c.err, DEV_STATE);
       return;
     }
@@ -561,9 +571,15 @@ __device__ void bk_logic(BookSmem& b, const Dev& D, Ctl& c, int mode, int arg) {
     c.n_commit++;
     c.L++;
     for (int k = 0; k < C; ++k) {
-      if (!b.alive[k] || bk_in_subtree(b, k, e)) continue;
+      if (!b.alive[k] || bk_in_subtree(b, k, e) || b.parent[k] == BK_RETIRING) continue;
+      if (k == root) {  // it has iterations left: it retires instead
+        b.parent[k] = BK_RETIRING;
+        b.c1[k] = b.c2[k] = b.x1[k] = b.x2[k] = -1;
+        b.gate[k] = 0;
+        continue;
+      }
       b.alive[k] = 0;
-      if (k != root) bk_free_slot(b, b.slot[k]);
+      bk_free_slot(b, b.slot[k]);
     }
     b.parent[e] = -1;
     D.lists[c.L - 1] = b.slot[e];
@@ -575,6 +591,8 @@ __device__ void bk_logic(BookSmem& b, const Dev& D, Ctl& c, int mode, int arg) {
     c.steps++;
     c.rows_sum += c.rows_cur;
     c.rows_max = max(c.rows_max, c.rows_cur);
+    for (int k = 0; k < C; ++k)  // retiring entries that ran their R-th iteration
+      if (b.alive[k] && b.parent[k] == BK_RETIRING && b.depth[k] >= D.R) b.alive[k] = 0;
     int n = 0;
     for (int k = 0; k < C; ++k)
       if (b.alive[k]) b.order[n++] = k;
@@ -624,7 +642,7 @@ __device__ void bk_logic(BookSmem& b, const Dev& D, Ctl& c, int mode, int arg) {
       else c.n_fallback++;
       const int surv = bk_find_uid(b, C, src == 1 ? b.c1[root] : src == 2 ? b.c2[root] : -1);
       for (int k = 0; k < C; ++k) {
-        if (!b.alive[k]) continue;
+        if (!b.alive[k] || b.parent[k] == BK_RETIRING) continue;
         const bool keep = surv >= 0 && bk_in_subtree(b, k, surv);
         if (!keep) {
           b.alive[k] = 0;

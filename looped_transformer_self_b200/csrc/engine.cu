@@ -26,8 +26,8 @@ namespace lt {
 
 struct LayerW {
   const void *g1, *wqkv, *wo, *g2, *wgu, *wd;
-  CUtensorMap tm_qkv, tm_o, tm_gu, tm_d;          // hi parts (or the bf16 weights)
-  CUtensorMap tm_qkv_lo, tm_o_lo, tm_gu_lo, tm_d_lo;  // lo parts (split tf32 only)
+  GemmOperand tm_qkv, tm_o, tm_gu, tm_d;          // hi parts (or the bf16 weights)
+  GemmOperand tm_qkv_lo, tm_o_lo, tm_gu_lo, tm_d_lo;  // lo parts (split tf32 only)
 };
 
 struct Handle {
@@ -51,15 +51,15 @@ struct Handle {
   int pass_graph_rows = -1;
   float* ssq = nullptr;     // [ceil(d/128)][C] sum-of-squares parts of the pending RMSNorm
   int ssq_tiles = 0;
-  int *cnt_o = nullptr, *cnt_gu = nullptr, *cnt_d = nullptr;     // in-GEMM epilogue counters
+  unsigned long long *cnt_o = nullptr, *cnt_gu = nullptr, *cnt_d = nullptr;  // epilogue arrivals
   int *need_o = nullptr, *need_gu = nullptr, *need_d = nullptr;  // arrivals completing a group
   void *Xd = nullptr, *Xo = nullptr, *Xf = nullptr, *kv = nullptr;
   float2* rope = nullptr;
   int* gemm_tab = nullptr;
   std::vector<int> plane_base;
   GemmShape sh_qkv, sh_o, sh_gu, sh_d, sh_head;
-  CUtensorMap tm_Xd, tm_Xo, tm_Xf, tm_head;
-  CUtensorMap tm_Xd_lo, tm_Xo_lo, tm_Xf_lo, tm_head_lo;
+  GemmOperand tm_Xd, tm_Xo, tm_Xf, tm_head;
+  GemmOperand tm_Xd_lo, tm_Xo_lo, tm_Xf_lo, tm_head_lo;
   const void *embed = nullptr, *final_norm = nullptr, *head = nullptr;
   std::vector<LayerW> layers;
   bool loaded = false, prefilled = false, begun = false;
@@ -197,11 +197,11 @@ static size_t carve(Handle* H, char* base) {
   const int dims[5][2] = {{3 * d, d}, {d, d}, {2 * f, d}, {d, f}, {V, d}};
   int tab_ints = 0;
   for (int k = 0; k < 5; ++k)
-    tab_ints += (gemm_table_ints(dims[k][0], dims[k][1], H->f32, gc) + 3) / 4 * 4;
+    tab_ints += (gemm_table_ints(dims[k][0], dims[k][1], H->f32, C, gc) + 3) / 4 * 4;
   H->gemm_tab = cv.take<int>(tab_ints);
   size_t part_floats = 0;
   for (int k = 0; k < 5; ++k) {
-    gemm_plan(dims[k][0], dims[k][1], H->f32, gc, shapes[k], nullptr, nullptr);
+    gemm_plan(dims[k][0], dims[k][1], H->f32, C, gc, shapes[k], nullptr, nullptr);
     part_floats = std::max(part_floats, gemm_part_bytes(*shapes[k], C) / sizeof(float));
   }
   H->part = cv.take<float>(part_floats);
@@ -212,9 +212,9 @@ static size_t carve(Handle* H, char* base) {
   H->attn_cnt = cv.take<int>((size_t)C * m.n_heads);
   H->ssq_tiles = (d + 127) / 128;
   H->ssq = cv.take<float>((size_t)H->ssq_tiles * C);
-  H->cnt_o = cv.take<int>(H->ssq_tiles);
-  H->cnt_d = cv.take<int>(H->ssq_tiles);
-  H->cnt_gu = cv.take<int>(f / 128);
+  H->cnt_o = cv.take<unsigned long long>(H->ssq_tiles);
+  H->cnt_d = cv.take<unsigned long long>(H->ssq_tiles);
+  H->cnt_gu = cv.take<unsigned long long>(f / 128);
   H->need_o = cv.take<int>(H->ssq_tiles);
   H->need_d = cv.take<int>(H->ssq_tiles);
   H->need_gu = cv.take<int>(f / 128);
@@ -293,10 +293,10 @@ static void plan(Handle* H) {
   } while (0)
 
 template <typename T>
-static cudaError_t gemm(Handle* H, const CUtensorMap& tw, const CUtensorMap& twl,
-                        const CUtensorMap& tx, const CUtensorMap& txl, const GemmShape& s,
+static cudaError_t gemm(Handle* H, const GemmOperand& tw, const GemmOperand& twl,
+                        const GemmOperand& tx, const GemmOperand& txl, const GemmShape& s,
                         const int* flag, const GemmEpi* epi = nullptr,
-                        const CUtensorMap* next_w = nullptr, const GemmShape* next_s = nullptr) {
+                        const GemmOperand* next_w = nullptr, const GemmShape* next_s = nullptr) {
   const double esz = H->f32 ? 4.0 : 2.0, split = H->mode == 2 ? 2.0 : 1.0;
   // algorithmic bytes: the weight matrix (both tf32 halves when split), the
   // activation rows and the fp32 result rows
@@ -315,8 +315,15 @@ static cudaError_t attention(Handle* H, int gl, const int* tagsrc, int tag_off, 
   Dev& D = H->D;
   const int C = H->C, Hn = H->m.n_heads;
   auto kern = fused ? k_attn<T, HD, true> : k_attn<T, HD, false>;
-  // grid: (head, work item); items = active rows' 128-position splits
-  return launch(H->use_pdl, kern, dim3(Hn, C * H->max_splits), dim3(128), H->stream,
+  // grid: (head, y); block y takes work items y, y + gy, ... (items = active
+  // rows' 128-position splits); gy: one resident wave of blocks
+  static int per_sm[2] = {0, 0};
+  int& nb = per_sm[fused ? 1 : 0];
+  if (nb == 0 && (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kern, 128, 0) != cudaSuccess ||
+                  nb < 1))
+    nb = 1;
+  const int gy = std::max(1, std::min(C * H->max_splits, nb * sm_count() / Hn));
+  return launch(H->use_pdl, kern, dim3(Hn, gy), dim3(128), H->stream,
                 (const float*)H->q, (T*)H->kv, H->plane_base[gl], tagsrc, tag_off, H->S,
                 H->m.d_model, Hn, mask, (const int*)D.r_pos, (const int*)D.r_blen,
                 (const int*)D.r_boff, H->lists_override ? H->lists_override : (const int*)D.lists,
@@ -389,7 +396,7 @@ static cudaError_t run_layers(Handle* H, int gl0, int n, int kind, const int* ma
     LT_CK(gemm<T>(H, L.tm_gu, L.tm_gu_lo, H->tm_Xd, H->tm_Xd_lo, H->sh_gu, flag, &egu, &L.tm_d,
                   &H->sh_d));
     ed.g = (l + 1 < n) ? H->layers[gl + 1].g1 : nullptr;  // next layer's g1 (.) h
-    const CUtensorMap* nw = (l + 1 < n) ? &H->layers[gl + 1].tm_qkv : (fused ? &H->tm_head : nullptr);
+    const GemmOperand* nw = (l + 1 < n) ? &H->layers[gl + 1].tm_qkv : (fused ? &H->tm_head : nullptr);
     const GemmShape* ns = (l + 1 < n) ? &H->sh_qkv : (fused ? &H->sh_head : nullptr);
     LT_CK(gemm<T>(H, L.tm_d, L.tm_d_lo, H->tm_Xf, H->tm_Xf_lo, H->sh_d, flag, &ed, nw, ns));
   }
@@ -526,12 +533,18 @@ extern "C" int lt_create(const lt_model_config* m, const lt_decode_config* dc, v
   std::vector<int> tab;
   std::vector<int> offs;
   for (int k = 0; k < 5; ++k) {
-    const int n = (gemm_table_ints(dims[k][0], dims[k][1], H->f32, gc) + 3) / 4 * 4;
+    const int n = (gemm_table_ints(dims[k][0], dims[k][1], H->f32, H->C, gc) + 3) / 4 * 4;
     std::vector<int> t(n, 0);
-    gemm_plan(dims[k][0], dims[k][1], H->f32, gc, shapes[k], t.data(),
+    gemm_plan(dims[k][0], dims[k][1], H->f32, H->C, gc, shapes[k], t.data(),
               t.data() + 2 * shapes[k]->tiles);
     offs.push_back((int)tab.size());
     tab.insert(tab.end(), t.begin(), t.end());
+  }
+  // a CTA of an epilogue GEMM keeps one arrival target per tile it touches
+  if (H->sh_o.jmax > GEMM_MAX_SEGS || H->sh_gu.jmax > GEMM_MAX_SEGS ||
+      H->sh_d.jmax > GEMM_MAX_SEGS) {
+    delete hd;
+    return LT_ERR_SHAPE;
   }
   cudaError_t e = cudaMemcpy(H->gemm_tab, tab.data(), tab.size() * sizeof(int), cudaMemcpyHostToDevice);
   if (e != cudaSuccess) {
@@ -556,8 +569,8 @@ extern "C" int lt_create(const lt_model_config* m, const lt_decode_config* dc, v
     if (cudaMemcpy(H->need_o, need_o.data(), need_o.size() * 4, cudaMemcpyHostToDevice) ||
         cudaMemcpy(H->need_d, need_d.data(), need_d.size() * 4, cudaMemcpyHostToDevice) ||
         cudaMemcpy(H->need_gu, need_gu.data(), need_gu.size() * 4, cudaMemcpyHostToDevice) ||
-        cudaMemset(H->cnt_o, 0, need_o.size() * 4) || cudaMemset(H->cnt_d, 0, need_d.size() * 4) ||
-        cudaMemset(H->cnt_gu, 0, need_gu.size() * 4) ||
+        cudaMemset(H->cnt_o, 0, need_o.size() * 8) || cudaMemset(H->cnt_d, 0, need_d.size() * 8) ||
+        cudaMemset(H->cnt_gu, 0, need_gu.size() * 8) ||
         cudaMemset(H->Xd, 0, px * H->C * d * esz) || cudaMemset(H->Xo, 0, px * H->C * d * esz) ||
         cudaMemset(H->Xf, 0, px * H->C * f * esz) ||
         cudaMemset(H->ssq, 0, (size_t)H->ssq_tiles * H->C * 4)) {
@@ -567,12 +580,13 @@ extern "C" int lt_create(const lt_model_config* m, const lt_decode_config* dc, v
   }
   // activation tensor maps (B operands)
   const size_t esz = H->f32 ? 4 : 2;
-  if (make_tmap(&H->tm_Xd, H->Xd, H->f32, H->C, d, H->C) ||
-      make_tmap(&H->tm_Xo, H->Xo, H->f32, H->C, d, H->C) ||
-      make_tmap(&H->tm_Xf, H->Xf, H->f32, H->C, f, H->C) ||
-      make_tmap(&H->tm_Xd_lo, (char*)H->Xd + H->lo_d * esz, H->f32, H->C, d, H->C) ||
-      make_tmap(&H->tm_Xo_lo, (char*)H->Xo + H->lo_d * esz, H->f32, H->C, d, H->C) ||
-      make_tmap(&H->tm_Xf_lo, (char*)H->Xf + H->lo_f * esz, H->f32, H->C, f, H->C)) {
+  const int kc = gemm_kc(H->C, H->f32);
+  if (make_operand(&H->tm_Xd, H->Xd, H->f32, H->C, d, H->C, kc) ||
+      make_operand(&H->tm_Xo, H->Xo, H->f32, H->C, d, H->C, kc) ||
+      make_operand(&H->tm_Xf, H->Xf, H->f32, H->C, f, H->C, kc) ||
+      make_operand(&H->tm_Xd_lo, (char*)H->Xd + H->lo_d * esz, H->f32, H->C, d, H->C, kc) ||
+      make_operand(&H->tm_Xo_lo, (char*)H->Xo + H->lo_d * esz, H->f32, H->C, d, H->C, kc) ||
+      make_operand(&H->tm_Xf_lo, (char*)H->Xf + H->lo_f * esz, H->f32, H->C, f, H->C, kc)) {
     delete hd;
     return LT_ERR_SHAPE;
   }
@@ -601,9 +615,10 @@ extern "C" int lt_load_weights(lt_handle* hd, const void* d_embed, const void* d
   size_t wofs = 0;
   // A weight matrix's tensor maps: bf16 -> the caller's tensor; fp32 -> hi / lo
   // tf32 copies in the workspace (split once here, at load time).
-  auto maps = [&](const void* w, int rows, int k, CUtensorMap* hi, CUtensorMap* lo) -> int {
+  const int kc = gemm_kc(H->C, H->f32);
+  auto maps = [&](const void* w, int rows, int k, GemmOperand* hi, GemmOperand* lo) -> int {
     if (!H->f32) {
-      if (make_tmap(hi, w, false, rows, k, GEMM_BM)) return -1;
+      if (make_operand(hi, w, false, rows, k, GEMM_BM, kc)) return -1;
       *lo = *hi;
       return 0;
     }
@@ -613,7 +628,8 @@ extern "C" int lt_load_weights(lt_handle* hd, const void* d_embed, const void* d
     wofs += n;
     if (wofs > H->wsplit_elems) return -2;
     if (split_tf32((const float*)w, wh, wl, n, H->stream) != cudaSuccess) return -3;
-    if (make_tmap(hi, wh, true, rows, k, GEMM_BM) || make_tmap(lo, wl, true, rows, k, GEMM_BM))
+    if (make_operand(hi, wh, true, rows, k, GEMM_BM, kc) ||
+        make_operand(lo, wl, true, rows, k, GEMM_BM, kc))
       return -1;
     return 0;
   };
@@ -1023,6 +1039,7 @@ extern "C" int lt_profile_steps(lt_handle* hd, int ar_mode, int n_steps, lt_prof
       } else if (ev.kind == 1) {
         out->gemm_other_ms += t;
         out->gemm_other_launches += 1;
+        out->gemm_other_bytes += ev.bytes;
       } else {
         out->attn_ms += t;
         out->attn_launches += 1;

@@ -1,5 +1,7 @@
 // tcgen05 / TMEM / TMA weight-streaming GEMM (see gemm.cuh for the design).
 #include <stdio.h>
+#include <stdlib.h>
+#include <string.h>
 
 #include <algorithm>
 #include <type_traits>
@@ -63,6 +65,21 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       ".L2::cache_hint [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar), "l"(policy)
       : "memory");
+}
+// 3-D box (128-byte rows x rows x chunks): a k-group of kc swizzled tiles.
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int y, int z,
+                                            uint32_t bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      ".L2::cache_hint [%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(0), "r"(y), "r"(z), "r"(bar), "l"(policy)
+      : "memory");
+}
+__device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap* map, int y, int z) {
+  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(0), "r"(y), "r"(z)
+               : "memory");
 }
 // Pulls one weight tile into L2 (no shared memory, no barrier).
 __device__ __forceinline__ void tma_prefetch_l2(const CUtensorMap* map, int x, int y) {
@@ -177,18 +194,19 @@ struct EpiSmem {
   float inv[64];     // per active row: 1 / rms (SwiGLU)
   float wsum[4][64]; // per warp, per active row: partial sum of squares
   int4 ti[8][2];     // per segment of this CTA: table entries of its group's tiles
+  unsigned long long target[GEMM_MAX_SEGS];  // per segment: arrival count completing its group
 };
 
-// Residual epilogue of one tile: h += scale * y; X = g (.) h; sum-of-squares part.
+// Residual epilogue of one tile for active rows r0 .. r1-1 (indices into
+// sm.rows): h += scale * y; X = g (.) h; sum-of-squares part of those rows.
 template <typename TX>
 __device__ void epi_resid(const GemmEpi& ep, const float* __restrict__ part, const GemmShape& s,
-                          int ncols, int t, int seg, int et, EpiSmem& sm) {
+                          int ncols, int t, int4 ti, int r0, int r1, int et, EpiSmem& sm) {
   const int n = t * 128 + et;
   const bool valid = n < s.n_out;
   const int lane = et & 31, w = et >> 5;
-  const int4 ti = sm.ti[seg][0];
-  for (int k0 = 0; k0 < sm.nact; k0 += 4) {
-    const int nr = min(4, sm.nact - k0);
+  for (int k0 = r0; k0 < r1; k0 += 4) {
+    const int nr = min(4, r1 - k0);
     float y[4], h0[4];
 #pragma unroll
     for (int u = 0; u < 4; ++u)  // h rows first: their loads overlap the partials'
@@ -213,22 +231,22 @@ __device__ void epi_resid(const GemmEpi& ep, const float* __restrict__ part, con
     }
   }
   drain_sync();
-  if (et < sm.nact) {
+  if (et >= r0 && et < r1) {
     const float v = sm.wsum[0][et] + sm.wsum[1][et] + sm.wsum[2][et] + sm.wsum[3][et];
     ep.ssq_out[(size_t)t * ncols + sm.rows[et]] = v;
   }
 }
 
-// SwiGLU epilogue of one (gate tile g, up tile g + ffn/128) pair; sm.inv was
-// filled during the mainloop.
+// SwiGLU epilogue of one (gate tile g, up tile g + ffn/128) pair for active
+// rows r0 .. r1-1; sm.inv was filled during the mainloop.
 template <typename TX>
 __device__ void epi_swiglu(const GemmEpi& ep, const float* __restrict__ part, const GemmShape& s,
-                           int ncols, int g, int seg, int et, EpiSmem& sm) {
+                           int ncols, int g, int4 tg, int4 tu, int r0, int r1, int et,
+                           EpiSmem& sm) {
   const int n = g * 128 + et;
   if (n >= ep.ffn) return;
-  const int4 tg = sm.ti[seg][0], tu = sm.ti[seg][1];
-  for (int k0 = 0; k0 < sm.nact; k0 += 4) {
-    const int nr = min(4, sm.nact - k0);
+  for (int k0 = r0; k0 < r1; k0 += 4) {
+    const int nr = min(4, r1 - k0);
     float gv[4], uv[4];
     tile_sum4<4>(part, s, tg, ncols, sm.rows + k0, nr, n & 127, gv);
     tile_sum4<4>(part, s, tu, ncols, sm.rows + k0, nr, n & 127, uv);
@@ -252,19 +270,21 @@ __device__ void epi_swiglu(const GemmEpi& ep, const float* __restrict__ part, co
 // the products to ~2^-21 relative error (fp32-grade) on the tensor cores.
 template <int MODE, int NC>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
-    k_gemm(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmWlo,
-           const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmXlo,
+    k_gemm(const __grid_constant__ GemmOperand W, const __grid_constant__ GemmOperand Wlo,
+           const __grid_constant__ GemmOperand X, const __grid_constant__ GemmOperand Xlo,
            float* __restrict__ part, const GemmShape s, const int stages,
            const int* __restrict__ run_flag, int* __restrict__ err, const GemmEpi ep,
-           const __grid_constant__ CUtensorMap tmNext, const GemmShape sNext) {
+           const __grid_constant__ GemmOperand Next, const GemmShape sNext) {
   using TX = typename std::conditional<MODE == 0, __nv_bfloat16, float>::type;
   __shared__ EpiSmem esm;
   constexpr bool TF32 = MODE != 0;
   constexpr int NSPLIT = MODE == 2 ? 2 : 1;
-  constexpr uint32_t A_BYTES = GEMM_BM * GEMM_CHUNK_BYTES;
+  constexpr uint32_t A_BYTES = GEMM_BM * GEMM_CHUNK_BYTES;  // one chunk of one tile
   constexpr uint32_t B_BYTES = NC * GEMM_CHUNK_BYTES;
-  constexpr uint32_t SA = NSPLIT * A_BYTES, SB = NSPLIT * B_BYTES;  // per-stage bytes
   constexpr int BKE = TF32 ? 32 : 64;  // elements per k-chunk
+  // stage layout: W [hi chunks 0..kc-1][lo chunks], X [hi chunks][lo chunks]
+  const int KC = s.kc;
+  const uint32_t SA = NSPLIT * KC * A_BYTES, SB = NSPLIT * KC * B_BYTES;  // per-stage bytes
   constexpr int TCOLS = tmem_cols<NC>();
   constexpr uint32_t IDESC = instr_desc<TF32, NC>();
 
@@ -305,11 +325,13 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmW)) : "memory");
-    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmX)) : "memory");
-    if constexpr (NSPLIT == 2) {
-      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmWlo)) : "memory");
-      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmXlo)) : "memory");
+    const GemmOperand* ops[4] = {&W, &X, &Wlo, &Xlo};
+    for (int o = 0; o < 2 * NSPLIT; ++o) {
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&ops[o]->chunk))
+                   : "memory");
+      if (KC > 1 && s.nfull >= KC)  // the 3-D view exists
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&ops[o]->group))
+                     : "memory");
     }
   }
   if (warp == 1) {
@@ -324,6 +346,54 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  // Unit uu = (tile t, k-group j): chunks c0 .. c0 + n - 1 of tile t.  A group
+  // of kc whole chunks is one 3-D request per operand; a group that reaches
+  // the end of K is one 2-D request per chunk (the ragged chunk zero-filled).
+  auto unit_of = [&](int uu, int& t, int& c0) -> int {
+    t = uu / s.kch;
+    c0 = (uu - t * s.kch) * KC;
+    return (KC > 1 && c0 + KC <= s.nfull) ? 0 : min(KC, s.nch - c0);  // 0: one 3-D box
+  };
+  auto load_w = [&](int uu, uint32_t dst, uint32_t bar, uint64_t pol) -> uint32_t {
+    int t, c0;
+    const int n = unit_of(uu, t, c0);
+    if (n == 0) {
+      tma_load_3d(dst, &W.group, t * GEMM_BM, c0, bar, pol);
+      if constexpr (NSPLIT == 2) tma_load_3d(dst + KC * A_BYTES, &Wlo.group, t * GEMM_BM, c0, bar, pol);
+      return NSPLIT * KC * A_BYTES;
+    }
+    for (int j = 0; j < n; ++j) {
+      tma_load_2d(dst + j * A_BYTES, &W.chunk, (c0 + j) * BKE, t * GEMM_BM, bar, pol);
+      if constexpr (NSPLIT == 2)
+        tma_load_2d(dst + (KC + j) * A_BYTES, &Wlo.chunk, (c0 + j) * BKE, t * GEMM_BM, bar, pol);
+    }
+    return NSPLIT * n * A_BYTES;
+  };
+  auto w_bytes = [&](int uu) -> uint32_t {
+    int t, c0;
+    const int n = unit_of(uu, t, c0);
+    return NSPLIT * (n == 0 ? KC : n) * A_BYTES;
+  };
+  auto load_x = [&](int uu, uint32_t dst, uint32_t bar, uint64_t pol) {
+    int t, c0;
+    const int n = unit_of(uu, t, c0);
+    if (n == 0) {
+      tma_load_3d(dst, &X.group, 0, c0, bar, pol);
+      if constexpr (NSPLIT == 2) tma_load_3d(dst + KC * B_BYTES, &Xlo.group, 0, c0, bar, pol);
+      return;
+    }
+    for (int j = 0; j < n; ++j) {
+      tma_load_2d(dst + j * B_BYTES, &X.chunk, (c0 + j) * BKE, 0, bar, pol);
+      if constexpr (NSPLIT == 2)
+        tma_load_2d(dst + (KC + j) * B_BYTES, &Xlo.chunk, (c0 + j) * BKE, 0, bar, pol);
+    }
+  };
+  auto x_bytes = [&](int uu) -> uint32_t {
+    int t, c0;
+    const int n = unit_of(uu, t, c0);
+    return NSPLIT * (n == 0 ? KC : n) * B_BYTES;
+  };
+
   // Weights do not depend on earlier kernels: the first `npre` stages of
   // weight tiles are requested before waiting on the preceding grid, so with
   // programmatic dependent launch this CTA's prologue and pipeline fill overlap
@@ -334,31 +404,39 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   const uint64_t pol_w = policy_evict_first(), pol_x = policy_evict_last();
   if (warp == 0 && lane == 0) {
     for (int g = 0; g < npre; ++g) {
-      const int uu = u0 + g, t = uu / s.kch;
-      const int kx = (uu - t * s.kch) * BKE;
-      mbar_expect_tx_only(full_bar(g), SA);
-      tma_load_2d(a_base + g * SA, &tmW, kx, t * GEMM_BM, full_bar(g), pol_w);
-      if constexpr (NSPLIT == 2)
-        tma_load_2d(a_base + g * SA + A_BYTES, &tmWlo, kx, t * GEMM_BM, full_bar(g), pol_w);
+      mbar_expect_tx_only(full_bar(g), w_bytes(u0 + g));
+      load_w(u0 + g, a_base + g * SA, full_bar(g), pol_w);
     }
     // The rest of this CTA's weight range goes to L2 now (often already there:
     // the GEMM in front of this one requested it), and so does this CTA's
     // slice of the NEXT GEMM's weights (sNext.units > 0), so HBM keeps
     // streaming weights through this kernel's tail and the kernels that follow
     // (attention, epilogues) until the next GEMM's ring is filled.
-    const int nl2 = min(u1 - u0, npre + GEMM_L2_PREFETCH_BYTES / (int)SA);
+    const int nl2 = min(u1 - u0, npre + GEMM_L2_PREFETCH_BYTES / (int)(KC * A_BYTES));
     for (int g = npre; g < nl2; ++g) {
-      const int uu = u0 + g, t = uu / s.kch;
-      const int kx = (uu - t * s.kch) * BKE;
-      tma_prefetch_l2(&tmW, kx, t * GEMM_BM);
-      if constexpr (NSPLIT == 2) tma_prefetch_l2(&tmWlo, kx, t * GEMM_BM);
+      int t, c0;
+      const int n = unit_of(u0 + g, t, c0);
+      if (n == 0) {
+        tma_prefetch_l2_3d(&W.group, t * GEMM_BM, c0);
+        if constexpr (NSPLIT == 2) tma_prefetch_l2_3d(&Wlo.group, t * GEMM_BM, c0);
+      } else {
+        for (int j = 0; j < n; ++j) {
+          tma_prefetch_l2(&W.chunk, (c0 + j) * BKE, t * GEMM_BM);
+          if constexpr (NSPLIT == 2) tma_prefetch_l2(&Wlo.chunk, (c0 + j) * BKE, t * GEMM_BM);
+        }
+      }
     }
     if (sNext.units > 0 && c < sNext.grid) {
       const int v0 = sk_u0(c, sNext.units, sNext.grid), v1 = sk_u0(c + 1, sNext.units, sNext.grid);
-      const int vend = min(v1, v0 + GEMM_L2_PREFETCH_BYTES / (int)A_BYTES);
+      const int vend = min(v1, v0 + GEMM_L2_PREFETCH_BYTES / (int)(sNext.kc * A_BYTES));
       for (int uu = v0; uu < vend; ++uu) {
-        const int t = uu / sNext.kch;
-        tma_prefetch_l2(&tmNext, (uu - t * sNext.kch) * BKE, t * GEMM_BM);
+        const int t = uu / sNext.kch, c0 = (uu - t * sNext.kch) * sNext.kc;
+        if (sNext.kc > 1 && c0 + sNext.kc <= sNext.nfull) {
+          tma_prefetch_l2_3d(&Next.group, t * GEMM_BM, c0);
+        } else {
+          for (int j = 0; j < min(sNext.kc, sNext.nch - c0); ++j)
+            tma_prefetch_l2(&Next.chunk, (c0 + j) * BKE, t * GEMM_BM);
+        }
       }
     }
   }
@@ -380,27 +458,16 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     if (lane == 0) {
       // ---------------- TMA producer ----------------
       int g = 0;
-      for (int u = u0; u < u1 && !*abort_flag;) {
-        const int t = u / s.kch;
-        const int seg_end = min(u1, (t + 1) * s.kch);
-        for (int uu = u; uu < seg_end; ++uu, ++g) {
-          const int st = g % stages, n = g / stages;
-          const int kx = (uu - t * s.kch) * BKE;
-          if (g < npre) {  // weights already requested
-            mbar_expect_tx(full_bar(st), SB);
-          } else {
-            if (!mbar_wait(empty_bar(st), (n & 1) ^ 1, abort_flag)) break;
-            mbar_expect_tx(full_bar(st), SA + SB);
-            tma_load_2d(a_base + st * SA, &tmW, kx, t * GEMM_BM, full_bar(st), pol_w);
-            if constexpr (NSPLIT == 2)
-              tma_load_2d(a_base + st * SA + A_BYTES, &tmWlo, kx, t * GEMM_BM, full_bar(st),
-                          pol_w);
-          }
-          tma_load_2d(b_base + st * SB, &tmX, kx, 0, full_bar(st), pol_x);
-          if constexpr (NSPLIT == 2)
-            tma_load_2d(b_base + st * SB + B_BYTES, &tmXlo, kx, 0, full_bar(st), pol_x);
+      for (int uu = u0; uu < u1; ++uu, ++g) {
+        const int st = g % stages, n = g / stages;
+        if (g < npre) {  // weights already requested
+          mbar_expect_tx(full_bar(st), x_bytes(uu));
+        } else {
+          if (!mbar_wait(empty_bar(st), (n & 1) ^ 1, abort_flag)) break;
+          mbar_expect_tx(full_bar(st), w_bytes(uu) + x_bytes(uu));
+          load_w(uu, a_base + st * SA, full_bar(st), pol_w);
         }
-        u = seg_end;
+        load_x(uu, b_base + st * SB, full_bar(st), pol_x);
       }
       // on abort: arrive on prefetched stages never reached so their loads can land
       for (int gg = g; gg < npre; ++gg) mbar_arrive(full_bar(gg));
@@ -422,24 +489,32 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         const uint32_t d_tmem = tmem + (uint32_t)(b * NC);
         for (int uu = u; uu < seg_end; ++uu, ++g) {
           const int st = g % stages, n = g / stages;
+          int tt, c0;
+          const int nc = unit_of(uu, tt, c0);
+          const int nchunk = nc == 0 ? KC : nc;
           if (!mbar_wait(full_bar(st), n & 1, abort_flag)) {
             ok = false;
             break;
           }
           tc_fence_after();
           const uint32_t a0 = a_base + st * SA, b0 = b_base + st * SB;
+          for (int j = 0; j < nchunk; ++j) {
+            const uint32_t aj = a0 + j * A_BYTES, bj = b0 + j * B_BYTES;
 #pragma unroll
-          for (int kk = 0; kk < GEMM_CHUNK_BYTES / 32; ++kk) {
-            const uint32_t acc = (uu > u || kk > 0) ? 1u : 0u;
-            if constexpr (NSPLIT == 2) {
-              // small cross terms first, then the leading product
-              tc_mma<TF32>(d_tmem, smem_desc(a0 + A_BYTES + 32u * kk), smem_desc(b0 + 32u * kk),
-                           IDESC, acc);
-              tc_mma<TF32>(d_tmem, smem_desc(a0 + 32u * kk), smem_desc(b0 + B_BYTES + 32u * kk),
-                           IDESC, 1u);
-              tc_mma<TF32>(d_tmem, smem_desc(a0 + 32u * kk), smem_desc(b0 + 32u * kk), IDESC, 1u);
-            } else {
-              tc_mma<TF32>(d_tmem, smem_desc(a0 + 32u * kk), smem_desc(b0 + 32u * kk), IDESC, acc);
+            for (int kk = 0; kk < GEMM_CHUNK_BYTES / 32; ++kk) {
+              const uint32_t acc = (uu > u || j > 0 || kk > 0) ? 1u : 0u;
+              if constexpr (NSPLIT == 2) {
+                // small cross terms first, then the leading product
+                tc_mma<TF32>(d_tmem, smem_desc(aj + KC * A_BYTES + 32u * kk),
+                             smem_desc(bj + 32u * kk), IDESC, acc);
+                tc_mma<TF32>(d_tmem, smem_desc(aj + 32u * kk),
+                             smem_desc(bj + KC * B_BYTES + 32u * kk), IDESC, 1u);
+                tc_mma<TF32>(d_tmem, smem_desc(aj + 32u * kk), smem_desc(bj + 32u * kk), IDESC,
+                             1u);
+              } else {
+                tc_mma<TF32>(d_tmem, smem_desc(aj + 32u * kk), smem_desc(bj + 32u * kk), IDESC,
+                             acc);
+              }
             }
           }
           tc_commit(empty_bar(st));
@@ -500,30 +575,66 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 #pragma unroll
       for (int i = 0; i < NC; ++i) dst[(size_t)i * GEMM_BM] = __uint_as_float(r[i]);
       if (ep.kind != EPI_NONE) {
-        // publish this segment; the arrival that completes the group runs its
-        // epilogue.  The barrier orders the drain threads' partial stores before
-        // thread 0's acq_rel atomic (cumulativity), whose acquire side makes the
-        // other CTAs' partials visible to the whole group after the next barrier.
+        // publish this segment: the barrier orders the drain threads' partial
+        // stores before thread 0's release atomic (cumulativity)
         drain_sync();
         if (et == 0) {
           const int grp = ep.kind == EPI_SWIGLU ? t % (ep.ffn / GEMM_BM) : t;
-          int old;
-          asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], 1;"
-                       : "=r"(old)
+          unsigned long long old;
+          asm volatile("atom.release.gpu.global.add.u64 %0, [%1], 1;"
+                       : "=l"(old)
                        : "l"(ep.counters + grp)
                        : "memory");
-          esm.last = (old + 1 == ep.need[grp]) ? grp : -1;
-          if (esm.last >= 0) ep.counters[grp] = 0;
+          // earlier launches left the counter at a multiple of need
+          const unsigned long long need = (unsigned long long)__ldg(ep.need + grp);
+          if (seg < GEMM_MAX_SEGS) esm.target[seg] = (old / need + 1) * need;
+        }
+      }
+      u = seg_end;
+    }
+    // Group epilogues.  Every segment of a group takes a share of its active
+    // rows (share k of n: rows [k*nact/n, (k+1)*nact/n)), so a group's
+    // partials are read by all of its contributors at once rather than by the
+    // last to arrive.  Shares start only after this CTA published all of its
+    // segments; a CTA that waits has published everything, and the grid (<= one
+    // CTA per SM) is wholly resident before any dependent grid launches, so the
+    // waits form no cycle.
+    if (ep.kind != EPI_NONE && !*abort_flag) {
+      const int t0 = u0 / s.kch, nseg = min((u1 - 1) / s.kch - t0 + 1, GEMM_MAX_SEGS);
+      const bool sw = ep.kind == EPI_SWIGLU;
+      const int groups = sw ? ep.ffn / GEMM_BM : s.tiles;
+      for (int sg = 0; sg < nseg; ++sg) {
+        const int t = t0 + sg;
+        const int grp = sw ? t % groups : t;
+        const int4 ta = sg < 8 ? esm.ti[sg][0] : __ldg(s.tinfo + grp);
+        const int4 tb = !sw ? ta : (sg < 8 ? esm.ti[sg][1] : __ldg(s.tinfo + grp + groups));
+        const int need = __ldg(ep.need + grp);
+        const int share = !sw ? c - ta.x : (t < groups ? c - ta.x : (ta.y - ta.x + 1) + c - tb.x);
+        if (et == 0) {
+          const unsigned long long target = esm.target[sg];
+          const long long w0 = clock64();
+          unsigned long long seen = 0;
+          while (true) {
+            asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(seen) : "l"(ep.counters + grp)
+                         : "memory");
+            if (seen >= target) break;
+            // give up on a timeout here or in another CTA (whose group may never complete)
+            if ((err && *reinterpret_cast<volatile int*>(err) == DEV_TIMEOUT) ||
+                clock64() - w0 > WAIT_LIMIT_CYCLES) {
+              *abort_flag = 1;
+              break;
+            }
+          }
         }
         drain_sync();
-        const int grp = esm.last;
-        if (grp >= 0) {
-          if (ep.kind == EPI_RESID) epi_resid<TX>(ep, part, s, NC, grp, seg, et, esm);
-          else epi_swiglu<TX>(ep, part, s, NC, grp, seg, et, esm);
+        if (*abort_flag) break;
+        const int r0 = share * esm.nact / need, r1 = (share + 1) * esm.nact / need;
+        if (r1 > r0) {
+          if (!sw) epi_resid<TX>(ep, part, s, NC, t, ta, r0, r1, et, esm);
+          else epi_swiglu<TX>(ep, part, s, NC, grp, ta, tb, r0, r1, et, esm);
         }
         drain_sync();
       }
-      u = seg_end;
     }
   }
   tc_fence_before();
@@ -548,19 +659,40 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
-static int stages_for(int ncols, int nsplit) {
-  const int stage = nsplit * (GEMM_BM * GEMM_CHUNK_BYTES + ncols * GEMM_CHUNK_BYTES);
-  int st = (GEMM_SMEM_BUDGET - 1024 - 256) / stage;
+GemmTuning gemm_tuning() {
+  static GemmTuning t = [] {
+    GemmTuning v;
+    const char* e = getenv("LT_GEMM_KC");
+    const int kc = e ? atoi(e) : 4;
+    v.kc = (kc == 1 || kc == 2 || kc == 4) ? kc : 4;
+    e = getenv("LT_GEMM_SMEM_KB");
+    const int kb = e ? atoi(e) : (v.kc <= 2 ? 112 : 220);
+    v.smem_budget = std::min(std::max(kb, 48), 224) * 1024;
+    return v;
+  }();
+  return t;
+}
+
+static int stages_for(int ncols, int nsplit, int kc) {
+  const int stage = nsplit * kc * (GEMM_BM + ncols) * GEMM_CHUNK_BYTES;
+  const int st = (gemm_tuning().smem_budget - 1024 - 512) / stage;
   return std::min(st, 16);
 }
-static size_t smem_bytes(int ncols, int stages, int nsplit) {
-  return 1024 + (size_t)stages * nsplit * (GEMM_BM + ncols) * GEMM_CHUNK_BYTES +
+static size_t smem_bytes(int ncols, int stages, int nsplit, int kc) {
+  return 1024 + (size_t)stages * nsplit * kc * (GEMM_BM + ncols) * GEMM_CHUNK_BYTES +
          8 * (2 * stages + 5) + 16;
 }
 
-int gemm_table_ints(int n_out, int k, bool f32, int grid_cap) {
+int gemm_kc(int ncols, bool f32) {
+  const int nsplit = f32 ? 2 : 1;
+  int kc = gemm_tuning().kc;
+  while (kc > 1 && stages_for(ncols, nsplit, kc) < 2) kc /= 2;
+  return kc;
+}
+
+int gemm_table_ints(int n_out, int k, bool f32, int ncols, int grid_cap) {
   GemmShape s;
-  gemm_plan(n_out, k, f32, grid_cap, &s, nullptr, nullptr);
+  gemm_plan(n_out, k, f32, ncols, grid_cap, &s, nullptr, nullptr);
   return 2 * s.tiles + s.grid + 4 * s.tiles + 4;  // tile_c, cta_t0, (pad to 16 B), tinfo
 }
 
@@ -568,12 +700,15 @@ int gemm_tinfo_offset(const GemmShape& s) {  // int offset of tinfo within the t
   return ((2 * s.tiles + s.grid + 3) / 4) * 4;
 }
 
-void gemm_plan(int n_out, int k, bool f32, int grid_cap, GemmShape* s, int* tile_c,
+void gemm_plan(int n_out, int k, bool f32, int ncols, int grid_cap, GemmShape* s, int* tile_c,
                int* cta_t0) {
   const int bke = f32 ? 32 : 64;
   s->n_out = n_out;
   s->k = k;
-  s->kch = (k + bke - 1) / bke;
+  s->kc = gemm_kc(ncols, f32);
+  s->nch = (k + bke - 1) / bke;
+  s->nfull = k / bke;
+  s->kch = (s->nch + s->kc - 1) / s->kc;
   s->tiles = (n_out + GEMM_BM - 1) / GEMM_BM;
   s->units = s->tiles * s->kch;
   s->grid = std::min(grid_cap, s->units);
@@ -651,21 +786,51 @@ int make_tmap(CUtensorMap* map, const void* base, bool f32, uint64_t rows, uint6
   return r == CUDA_SUCCESS ? 0 : -3;
 }
 
+// 3-D view of a K-major operand: (128-byte row piece, row, chunk), the chunk
+// dimension stepping 128 bytes along K.  Only whole chunks are mapped, so a
+// box never reads past a row's end.
+static int make_group_map(CUtensorMap* map, const void* base, bool f32, uint64_t rows,
+                          uint64_t k, uint32_t box_rows, int kc) {
+  EncodeTiledFn enc = get_encode();
+  if (!enc) return -1;
+  const uint32_t esz = f32 ? 4 : 2, bke = GEMM_CHUNK_BYTES / esz;
+  if (((uintptr_t)base & 15) || ((k * esz) & 15) || box_rows == 0 || box_rows > 256) return -2;
+  cuuint64_t dims[3] = {bke, rows, k / bke};
+  cuuint64_t strides[2] = {k * esz, GEMM_CHUNK_BYTES};
+  cuuint32_t box[3] = {bke, box_rows, (cuuint32_t)kc};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                   const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? 0 : -3;
+}
+
+int make_operand(GemmOperand* op, const void* base, bool f32, uint64_t rows, uint64_t k,
+                 uint32_t box_rows, int kc) {
+  memset(op, 0, sizeof(*op));
+  if (int e = make_tmap(&op->chunk, base, f32, rows, k, box_rows)) return e;
+  const uint64_t bke = GEMM_CHUNK_BYTES / (f32 ? 4 : 2);
+  if (kc > 1 && k / bke >= (uint64_t)kc)
+    return make_group_map(&op->group, base, f32, rows, k, box_rows, kc);
+  return 0;
+}
+
 template <int MODE, int NC>
-static cudaError_t launch_t(const CUtensorMap& tmW, const CUtensorMap& tmWlo,
-                            const CUtensorMap& tmX, const CUtensorMap& tmXlo, float* part,
-                            const GemmShape& s, const int* run_flag, int* err,
-                            cudaStream_t stream, bool pdl, const GemmEpi& ep,
-                            const CUtensorMap& tmN, const GemmShape& sN) {
+static cudaError_t launch_t(const GemmOperand& W, const GemmOperand& Wlo, const GemmOperand& X,
+                            const GemmOperand& Xlo, float* part, const GemmShape& s,
+                            const int* run_flag, int* err, cudaStream_t stream, bool pdl,
+                            const GemmEpi& ep, const GemmOperand& N, const GemmShape& sN) {
   const int nsplit = MODE == 2 ? 2 : 1;
-  const int stages = stages_for(NC, nsplit);
-  const size_t smem = smem_bytes(NC, stages, nsplit);
-  static bool attr_set = false;
-  if (!attr_set) {
+  const int stages = stages_for(NC, nsplit, s.kc);
+  if (stages < 1) return cudaErrorInvalidValue;
+  const size_t smem = smem_bytes(NC, stages, nsplit, s.kc);
+  static size_t attr_bytes = 0;
+  if (smem > attr_bytes) {
     cudaError_t e = cudaFuncSetAttribute(k_gemm<MODE, NC>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    attr_set = true;
+    attr_bytes = smem;
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(s.grid);
@@ -677,14 +842,14 @@ static cudaError_t launch_t(const CUtensorMap& tmW, const CUtensorMap& tmWlo,
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, k_gemm<MODE, NC>, tmW, tmWlo, tmX, tmXlo, part, s, stages,
-                            run_flag, err, ep, tmN, sN);
+  return cudaLaunchKernelEx(&cfg, k_gemm<MODE, NC>, W, Wlo, X, Xlo, part, s, stages, run_flag, err,
+                            ep, N, sN);
 }
 
-cudaError_t gemm_launch(const CUtensorMap& tmW, const CUtensorMap& tmWlo, const CUtensorMap& tmX,
-                        const CUtensorMap& tmXlo, float* part, const GemmShape& s, int ncols,
+cudaError_t gemm_launch(const GemmOperand& W, const GemmOperand& Wlo, const GemmOperand& X,
+                        const GemmOperand& Xlo, float* part, const GemmShape& s, int ncols,
                         int mode, const int* run_flag, int* err, cudaStream_t stream, bool pdl,
-                        const GemmEpi* epi, const CUtensorMap* next_w,
+                        const GemmEpi* epi, const GemmOperand* next_w,
                         const GemmShape* next_s) {
   GemmEpi none = {};
   none.kind = EPI_NONE;
@@ -692,12 +857,12 @@ cudaError_t gemm_launch(const CUtensorMap& tmW, const CUtensorMap& tmWlo, const 
   GemmShape no_next = {};
   const bool has_next = next_w && next_s && mode != 2;
   const GemmShape& sN = has_next ? *next_s : no_next;
-  const CUtensorMap& tmN = has_next ? *next_w : tmW;
-#define LT_GEMM_CASE(N)                                                                      \
-  case N:                                                                                    \
-    return mode == 2   ? launch_t<2, N>(tmW, tmWlo, tmX, tmXlo, part, s, run_flag, err, stream, pdl, ep, tmN, sN) \
-           : mode == 1 ? launch_t<1, N>(tmW, tmWlo, tmX, tmXlo, part, s, run_flag, err, stream, pdl, ep, tmN, sN) \
-                       : launch_t<0, N>(tmW, tmWlo, tmX, tmXlo, part, s, run_flag, err, stream, pdl, ep, tmN, sN);
+  const GemmOperand& N = has_next ? *next_w : W;
+#define LT_GEMM_CASE(C)                                                                           \
+  case C:                                                                                         \
+    return mode == 2   ? launch_t<2, C>(W, Wlo, X, Xlo, part, s, run_flag, err, stream, pdl, ep, N, sN) \
+           : mode == 1 ? launch_t<1, C>(W, Wlo, X, Xlo, part, s, run_flag, err, stream, pdl, ep, N, sN) \
+                       : launch_t<0, C>(W, Wlo, X, Xlo, part, s, run_flag, err, stream, pdl, ep, N, sN);
   switch (ncols) {
     LT_GEMM_CASE(8)
     LT_GEMM_CASE(16)

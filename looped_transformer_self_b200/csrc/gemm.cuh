@@ -15,13 +15,20 @@
 //    runs all ncols columns, so a row's result never depends on how many other
 //    rows are active (batch invariance: the speculative and full-depth paths
 //    give bit-identical rows).
-//  * stream-K: the (tile, 128-byte k-chunk) units are split evenly over one CTA
-//    per SM; each CTA streams its contiguous unit range through a TMA ring of
-//    up to ~200 KB of shared memory, issues tcgen05.mma from one thread into
-//    double-buffered TMEM accumulators, and drains each finished tile segment
-//    (tcgen05.ld) as an fp32 partial.  The consumer kernel adds a tile's
-//    partials in CTA order (fixed order: deterministic).  The partition depends
-//    only on (n_out, K, #SMs), never on the active row count.
+//  * stream-K: the (tile, k-group) units are split evenly over one CTA per SM;
+//    each CTA streams its contiguous unit range through a TMA ring in shared
+//    memory, issues tcgen05.mma from one thread into double-buffered TMEM
+//    accumulators, and drains each finished tile segment (tcgen05.ld) as an
+//    fp32 partial.  The consumer adds a tile's partials in CTA order (fixed
+//    order: deterministic).  The partition depends only on (n_out, K, kc,
+//    #SMs), never on the active row count.
+//  * one TMA request per operand per stage.  A k-group is kc consecutive
+//    128-byte k-chunks of a 128-row tile; a 3-D view of W (128-byte rows x
+//    rows x chunks) loads the whole group as kc standard 128B-swizzled tiles
+//    in one request.  On B200 an SM's TMA completes roughly one request per
+//    ~0.6 us whatever its size up to 32 KB, so 16 KB requests cap an SM near
+//    27 GB/s (~4 TB/s for the GPU) while 64 KB requests reach the HBM rate.
+//    Groups that reach a ragged K tail fall back to one 2-D request per chunk.
 //  * bf16 operands: kind::f16 with fp32 accumulate; fp32 operands: kind::tf32,
 //    either one pass or split hi + lo (three MMAs per k-step, fp32-grade).
 //  * K tails and n_out tails are zero-filled by TMA.
@@ -34,44 +41,62 @@
 namespace lt {
 
 constexpr int GEMM_BM = 128;            // output features per tile (MMA M)
-constexpr int GEMM_CHUNK_BYTES = 128;   // K bytes per stage (one 128B-swizzle row)
+constexpr int GEMM_CHUNK_BYTES = 128;   // K bytes per k-chunk (one 128B-swizzle row)
 constexpr int GEMM_THREADS = 192;       // warp 0: TMA, warp 1: MMA, warps 2-5: drain
-// Shared memory per CTA for the TMA ring (5 stages of 18 KB at 16 rows).  A
-// ring this size lets the next GEMM's CTA be resident on the same SM and fill
-// its own ring before its dependency wait, which measured better than a deeper
-// ring with one CTA per SM.
-constexpr int GEMM_SMEM_BUDGET = 104 * 1024;
+constexpr int GEMM_MAX_SEGS = 16;       // tiles one CTA may touch in a GEMM with an epilogue
 // Weight bytes per CTA requested into L2 ahead of use, for this GEMM's range
 // beyond the ring and for the next GEMM's slice (148 CTAs: <= 47 MB each, well
 // inside the 126 MB L2).
 constexpr int GEMM_L2_PREFETCH_BYTES = 320 * 1024;
 
-// Plans the stream-K split of one weight matrix.  `grid_cap`: CTAs (#SMs).
+// Ring geometry: k-chunks per stage (kc in {1, 2, 4}) and the shared-memory
+// budget of the ring.  Default: kc 4 in ~218 KB (three 72 KB stages at 16
+// rows, one CTA per SM).  kc 2 in ~109 KB lets the next GEMM's CTA be resident
+// beside this one, but measured slower on the Ouro-1.4B decode step (1.70 vs
+// 1.56 ms).  LT_GEMM_KC and LT_GEMM_SMEM_KB override them (read once per
+// process).
+struct GemmTuning {
+  int kc;
+  int smem_budget;
+};
+GemmTuning gemm_tuning();
+// Chunks per unit for this operand width (kc reduced until two stages fit).
+int gemm_kc(int ncols, bool f32);
+
+// Plans the stream-K split of one weight matrix.  `grid_cap`: CTAs (#SMs);
+// `ncols`: the activation width the GEMM will run with (sets kc).
 // Fills the host copies of the reducer tables: tile_c [2*tiles], cta_t0 [grid]
 // and, when tile_c_host is given, the tinfo block after them (see gemm_table_ints;
 // the caller sizes tile_c_host with gemm_table_ints).
-void gemm_plan(int n_out, int k, bool f32, int grid_cap, GemmShape* s, int* tile_c_host,
-               int* cta_t0_host);
+void gemm_plan(int n_out, int k, bool f32, int ncols, int grid_cap, GemmShape* s,
+               int* tile_c_host, int* cta_t0_host);
 // Table block of one shape: tile_c [2*tiles], cta_t0 [grid], pad, tinfo [4*tiles]
 // (int4, 16-byte aligned when the block is).  gemm_plan fills it from tile_c_host.
-int gemm_table_ints(int n_out, int k, bool f32, int grid_cap);
+int gemm_table_ints(int n_out, int k, bool f32, int ncols, int grid_cap);
 int gemm_tinfo_offset(const GemmShape& s);
 
-// Encodes a K-major 2-D tensor map (rows x k, box box_rows x 128 bytes, 128B swizzle).
-int make_tmap(CUtensorMap* map, const void* base, bool f32, uint64_t rows, uint64_t k,
-              uint32_t box_rows);
+// The two TMA views of one K-major operand (rows x k, 128B swizzle): `chunk`
+// is 2-D with a box of box_rows x 128 bytes; `group` is 3-D (128-byte rows,
+// rows, whole chunks) with a box of box_rows x kc chunks, present when
+// kc > 1 and K holds at least kc whole chunks.
+struct GemmOperand {
+  CUtensorMap chunk;
+  CUtensorMap group;
+};
+int make_operand(GemmOperand* op, const void* base, bool f32, uint64_t rows, uint64_t k,
+                 uint32_t box_rows, int kc);
 
 // Launches the GEMM.  ncols in {8, 16, 32, 64}.  mode: 0 bf16, 1 tf32, 2 fp32 as
-// split tf32 (tmWlo / tmXlo map the low parts; ignored otherwise).  run_flag
+// split tf32 (Wlo / Xlo view the low parts; ignored otherwise).  run_flag
 // (device, may be null): skip when *run_flag == 0.  pdl: launch with
 // programmatic stream serialization.
 // epi (may be null): in-GEMM epilogue run by the CTA completing each tile group.
 // next_w / next_s (may be null): the weights of the GEMM that follows, whose
 // slice each CTA requests into L2.
-cudaError_t gemm_launch(const CUtensorMap& tmW, const CUtensorMap& tmWlo, const CUtensorMap& tmX,
-                        const CUtensorMap& tmXlo, float* part, const GemmShape& s, int ncols,
+cudaError_t gemm_launch(const GemmOperand& W, const GemmOperand& Wlo, const GemmOperand& X,
+                        const GemmOperand& Xlo, float* part, const GemmShape& s, int ncols,
                         int mode, const int* run_flag, int* err, cudaStream_t stream, bool pdl,
-                        const GemmEpi* epi = nullptr, const CUtensorMap* next_w = nullptr,
+                        const GemmEpi* epi = nullptr, const GemmOperand* next_w = nullptr,
                         const GemmShape* next_s = nullptr);
 
 // Segments that complete each epilogue group (host).  group_tiles 0: one group

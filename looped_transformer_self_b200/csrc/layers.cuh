@@ -253,9 +253,9 @@ struct RawVec {
 // Block (row i, head h, split sp) covers positions [sp*CH, min(sp*CH+CH, pos+1)) of
 // the row's own prefix (committed slots, then the ancestors' and its own slot),
 // all read from the row's depth plane.  16 lanes share one cache row (HD/16
-// elements each, vector loads); each half-warp keeps ATT_U positions' K and V
-// loads in flight and folds them into an online softmax (one pass over the
-// cache).  The 8 half-warps merge in fixed order; the split's (max, sum,
+// elements each, vector loads); each half-warp keeps att_u<T>() positions' K and
+// V loads in flight (16 for bf16 caches: a 128-position split is one round of
+// loads) and folds them into an online softmax (one pass over the cache).  The 8 half-warps merge in fixed order; the split's (max, sum,
 // unnormalised acc) goes to `opart`, and the last block of the (row, head) to
 // finish merges all splits in split order and writes the O-GEMM input row
 // (deterministic whichever block comes last).
@@ -268,7 +268,10 @@ struct RawVec {
 // (planes differ) and siblings never hold each other's positions.  Prefill
 // rows of one chunk do read each other's rows, so prefill runs the separate
 // QKV epilogue first (FUSED = false) and reads q from `q`.
-constexpr int ATT_U = 8;  // positions per half-warp in flight
+template <typename T>
+__host__ __device__ constexpr int att_u() {  // positions per half-warp in flight
+  return sizeof(T) == 2 ? 16 : 8;
+}
 
 template <typename T, int HD, bool FUSED>
 __global__ void __launch_bounds__(128) k_attn(
@@ -287,22 +290,25 @@ __global__ void __launch_bounds__(128) k_attn(
   __shared__ float hacc[8][HD];
   __shared__ int last;
   __shared__ int s_item[3];
-  // Block (head h, item w): items are the active rows' splits, rows in order,
-  // so the work sits in the first blocks of the grid (blocks past the last
-  // item only wait and exit).  Row bookkeeping, slot lists, the cache rows of
-  // earlier positions and (fused) the RMSNorm sums of squares were written by
-  // kernels that finished before this grid was launched: they are read -- and
-  // the block's K/V rows are requested into L2 -- before the dependency wait,
-  // while the QKV GEMM in front of this kernel still runs.
-  const int h = blockIdx.x, w = blockIdx.y;
+  // Block (head h, y): items are the active rows' splits, rows in order; block y
+  // takes items y, y + gridDim.y, ...  The grid holds about one resident wave
+  // (a grid of every possible item would be mostly empty blocks, each still
+  // scheduled and retired before the O GEMM may start).  Row bookkeeping, slot
+  // lists, the cache rows of earlier positions and (fused) the RMSNorm sums of
+  // squares were written by kernels that finished before this grid was
+  // launched: for the first item they are read -- and the block's K/V rows are
+  // requested into L2 -- before the dependency wait, while the QKV GEMM in
+  // front of this kernel still runs.
+  const int h = blockIdx.x;
+  for (int item = blockIdx.y, it = 0;; item += gridDim.y, ++it) {
   if (threadIdx.x == 0) {
     int acc = 0, row = -1, spl = 0, nsr = 0;
 #pragma unroll 8
     for (int k = 0; k < C; ++k) {
       const int nk = mask[k] ? (r_pos[k] + ATT_CH) / ATT_CH : 0;
-      if (row < 0 && w < acc + nk) {
+      if (row < 0 && item < acc + nk) {
         row = k;
-        spl = w - acc;
+        spl = item - acc;
         nsr = nk;
       }
       acc += nk;
@@ -314,9 +320,11 @@ __global__ void __launch_bounds__(128) k_attn(
   __syncthreads();
   const int i = s_item[0], sp = s_item[1], ns = s_item[2];
   if (i < 0) {
-    pdl_wait();
-    pdl_trigger();
-    return;
+    if (it == 0) {
+      pdl_wait();
+      pdl_trigger();
+    }
+    break;
   }
   const int n = r_pos[i] + 1;
   const int start = sp * ATT_CH;
@@ -365,8 +373,10 @@ __global__ void __launch_bounds__(128) k_attn(
       tiV = __ldg(qs_shape.tinfo + (nV >> 7));
     }
   }
-  pdl_wait();
-  pdl_trigger();
+  if (it == 0) {
+    pdl_wait();
+    pdl_trigger();
+  }
   const int hw = threadIdx.x >> 4, l16 = threadIdx.x & 15;
   const float scale = rsqrtf((float)HD);
   float qv[EPL];
@@ -411,6 +421,7 @@ __global__ void __launch_bounds__(128) k_attn(
 #pragma unroll
   for (int e = 0; e < EPL; ++e) acc[e] = 0.f;
   // both half-warps of a warp run the same trip count (the shuffles need the warp)
+  constexpr int ATT_U = att_u<T>();
   for (int tb = (hw & ~1) * ATT_U; tb < cnt; tb += 8 * ATT_U) {
     const int t0 = tb + (hw & 1) * ATT_U;
     RawVec<T, EPL> kx[ATT_U], vx[ATT_U];
@@ -494,20 +505,47 @@ __global__ void __launch_bounds__(128) k_attn(
     if (last) counters[i * H + h] = 0;
   }
   __syncthreads();
-  if (!last) return;
+  if (last) {
   __threadfence();
+  // Merge all splits in split order.  One round of independent loads: thread s
+  // fetches split s's (max, sum) into shared memory while every thread fetches
+  // its accumulator element of the first ATT_MB splits; then the weights
+  // exp(max_s - M) come from shared memory.
   const float* base = opart + (size_t)(i * H + h) * max_splits * (HD + 2);
+  constexpr int ATT_MB = 16;
+  constexpr int CAP = 4 * HD;  // splits whose (max, sum) fit in hacc
+  float* sM = &hacc[0][0];
+  float* sL = sM + CAP;
+  const int e = threadIdx.x;  // element of the head (blockDim >= HD)
+  float av[ATT_MB];
+#pragma unroll
+  for (int k = 0; k < ATT_MB; ++k)
+    av[k] = (e < HD && k < ns) ? __ldcg(base + (size_t)k * (HD + 2) + 2 + e) : 0.f;
+  if (ns <= CAP) {
+    for (int s2 = threadIdx.x; s2 < ns; s2 += blockDim.x) {
+      sM[s2] = __ldcg(base + (size_t)s2 * (HD + 2));
+      sL[s2] = __ldcg(base + (size_t)s2 * (HD + 2) + 1);
+    }
+  }
+  __syncthreads();
+  auto mx_of = [&](int s2) { return ns <= CAP ? sM[s2] : __ldcg(base + (size_t)s2 * (HD + 2)); };
+  auto l_of = [&](int s2) { return ns <= CAP ? sL[s2] : __ldcg(base + (size_t)s2 * (HD + 2) + 1); };
   float Mx = -INFINITY;
-  for (int s2 = 0; s2 < ns; ++s2) Mx = fmaxf(Mx, __ldcg(base + (size_t)s2 * (HD + 2)));
+  for (int s2 = 0; s2 < ns; ++s2) Mx = fmaxf(Mx, mx_of(s2));
   float Lx = 0.f;
-  for (int s2 = 0; s2 < ns; ++s2)
-    Lx += __ldcg(base + (size_t)s2 * (HD + 2) + 1) * __expf(__ldcg(base + (size_t)s2 * (HD + 2)) - Mx);
-  for (int e = threadIdx.x; e < HD; e += blockDim.x) {
+  for (int s2 = 0; s2 < ns; ++s2) Lx += l_of(s2) * __expf(mx_of(s2) - Mx);
+  if (e < HD) {
     float o = 0.f;
-    for (int s2 = 0; s2 < ns; ++s2)
-      o += __ldcg(base + (size_t)s2 * (HD + 2) + 2 + e) * __expf(__ldcg(base + (size_t)s2 * (HD + 2)) - Mx);
+#pragma unroll
+    for (int k = 0; k < ATT_MB; ++k)
+      if (k < ns) o += av[k] * __expf(mx_of(k) - Mx);
+    for (int s2 = ATT_MB; s2 < ns; ++s2)
+      o += __ldcg(base + (size_t)s2 * (HD + 2) + 2 + e) * __expf(mx_of(s2) - Mx);
     store_act<T>(X + (size_t)i * d + h * HD, e, o / Lx, lo);
   }
+  }  // last
+  __syncthreads();  // shared memory is reused by the next item
+  }  // items
 }
 
 // ---- RoPE table: (cos, sin) of pos * theta^(-2e/hd), computed in double ------------

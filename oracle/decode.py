@@ -222,6 +222,12 @@ class Branch:
     q2: Optional[np.ndarray] = None
     child1: int = -1
     child2: int = -1
+    # A former root left behind by an external commit: it keeps iterating and
+    # taking its readouts (so its committed position gets its block and coda
+    # cache rows at every depth) but decides nothing -- no proposal, no
+    # verification -- is never pruned, and leaves the table once it has run
+    # all R iterations.
+    retiring: bool = False
 
 
 class SpecDecoder:
@@ -335,9 +341,16 @@ class SpecDecoder:
                 b.p = S.process(z, self.T, self.top_p)
         self.step_margin.append(margin)
         self.step_gap.append(gap)
+        # retiring rows that ran their last iteration leave (their slots hold
+        # committed positions)
+        for u in order:
+            if self.branches[u].retiring and self.branches[u].depth >= self.R:
+                del self.branches[u]
         # 4. proposals
         for u in order:
-            b = self.branches[u]
+            b = self.branches.get(u)
+            if b is None or b.retiring:
+                continue
             spawn = b.pos + 1 < self.pos_limit  # is a child at pos+1 still needed?
             if b.depth == self.d1:
                 b.q1 = b.p
@@ -387,7 +400,7 @@ class SpecDecoder:
                 if x_ is not None:
                     keep.add(u)
         for u in sorted(self.branches):
-            if u in keep:
+            if u in keep or self.branches[u].retiring:
                 continue
             b = self.branches.pop(u)
             if u != root.uid:  # the root's slot holds a committed position
@@ -415,7 +428,7 @@ class SpecDecoder:
         """Prune branch `uid` and all its descendants (not the root); their slots
         are freed and the parent forgets the child."""
         b = self.branches[uid]
-        assert uid != self.root().uid
+        assert uid != self.root().uid and not b.retiring
         for u in self._subtree(uid):
             self.free.add(self.branches.pop(u).slot)
         p = self.branches.get(b.parent)
@@ -428,7 +441,10 @@ class SpecDecoder:
     def commit_branch(self, uid: int) -> None:
         """Commit a child of the root without full-depth verification (an
         external acceptance, source 3): its token is appended, every branch
-        outside its subtree is pruned and it becomes the root."""
+        outside its subtree is pruned and it becomes the root.  The old root
+        has not run all R iterations yet, and later rows read its position's
+        cache rows at every depth, so it stays in the table as a retiring row
+        until it has (see Branch.retiring)."""
         root = self.root()
         b = self.branches[uid]
         assert b.parent == root.uid
@@ -437,11 +453,17 @@ class SpecDecoder:
         self.cstep.append(self.stats.steps)
         keep = set(self._subtree(uid))
         for u in sorted(self.branches):
-            if u in keep:
+            x = self.branches[u]
+            if u in keep or x.retiring:
                 continue
-            x = self.branches.pop(u)
-            if u != root.uid:
-                self.free.add(x.slot)
+            if u == root.uid:
+                x.retiring = True
+                x.child1 = x.child2 = x.x1 = x.x2 = -1
+                x.gate = False
+                x.q1 = x.q2 = None
+                continue
+            self.branches.pop(u)
+            self.free.add(x.slot)
         b.parent = -1
         self.cslots.append(b.slot)
 

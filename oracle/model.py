@@ -58,10 +58,14 @@ class LoopedModel:
     models carry their bf16-rounded values).
     """
 
-    def __init__(self, cfg, weights: Dict[str, np.ndarray], n_slots: int):
+    def __init__(self, cfg, weights: Dict[str, np.ndarray], n_slots: int,
+                 unwritten: float = 0.0):
+        """``unwritten``: value of cache rows no position has written (NaN makes
+        any read of a row that was never computed poison the result)."""
         self.cfg = cfg
         self.w = {k: np.ascontiguousarray(v, dtype=np.float32) for k, v in weights.items()}
         self.n_slots = n_slots
+        self.unwritten = unwritten
         self.caches: Dict[Tuple[str, int], Tuple[np.ndarray, np.ndarray]] = {}
         self.lib = lib()
 
@@ -70,7 +74,8 @@ class LoopedModel:
         key = (layer, tag)
         if key not in self.caches:
             d = self.cfg.d_model
-            self.caches[key] = (np.zeros((self.n_slots, d)), np.zeros((self.n_slots, d)))
+            self.caches[key] = (np.full((self.n_slots, d), self.unwritten),
+                                np.full((self.n_slots, d), self.unwritten))
         return self.caches[key]
 
     # -- one layer -----------------------------------------------------------

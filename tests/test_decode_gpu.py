@@ -229,15 +229,19 @@ def test_bf16_greedy_spec_equals_ar_long_context(cfg):
     assert st["n_first"] + st["n_second"] + st["n_fallback"] == dec.max_new
 
 
-def test_tree_edits_match_oracle(tiny):
+@pytest.mark.parametrize("fill", [None, 0x3F, 0xFF])
+def test_tree_edits_match_oracle(tiny, fill):
     """lt_rollback_branch / lt_commit_branch between single steps: the GPU's
     branch rows, slots and commits stay bit-identical to the oracle doing the
-    same edits."""
+    same edits -- also when the workspace starts out as garbage (0x3F: finite
+    values, 0xFF: NaN and -1), so nothing is read before it is written (an
+    external commit leaves the old root retiring until its cache rows exist at
+    every depth)."""
     from oracle import decode as D
     from oracle.model import LoopedModel
     cfg, w, prompt = tiny
     dec = syn.DECODES["tiny_greedy"].replace(d1=1, d2=2, max_new=24)
-    g = _decoder(cfg, dec, w, max_branches=16)
+    g = _decoder(cfg, dec, w, max_branches=16, workspace_fill=fill)
     first, _, _ = g.prefill(prompt)
     sd = D.SpecDecoder(D.OracleRows(LoopedModel(cfg, w, 256)), prompt, cfg.R, dec.d1, dec.d2,
                        dec.max_new, 0.0, 1.0, dec.seed, 256)

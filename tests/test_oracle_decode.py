@@ -156,7 +156,51 @@ def test_rollback_keeps_output_lossless_and_commit_branch_edits_tree():
     assert sd.root().uid == child.uid and sd.src[-1] == 3
     assert sd.cslots[-1] == child.slot and root.slot in sd.cslots
     for b in sd.branches.values():
-        assert b.uid == child.uid or child.uid in _ancestors(sd, b)
+        if not b.retiring:
+            assert b.uid == child.uid or child.uid in _ancestors(sd, b)
+    # the old root had iterations left: it retires (stays until its R-th)
+    assert [b.uid for b in sd.branches.values() if b.retiring] == [root.uid]
+    assert root.depth < cfg.R and root.slot not in sd.free
+
+
+def test_no_row_reads_a_cache_row_that_was_never_written():
+    """Every cache row a row attends to was computed first, also around
+    external commits (whose old root has not run all R iterations) and
+    rollbacks: with unwritten rows set to NaN, every readout stays finite and
+    the tokens equal those of the zero-filled run; a retiring root leaves the
+    table right after its R-th iteration."""
+    cfg, w = _tiny()
+    prompt = syn.prompt_for("tiny", 16)
+
+    def run(unwritten):
+        sd = D.SpecDecoder(D.OracleRows(LoopedModel(cfg, w, 128, unwritten=unwritten)), prompt,
+                           cfg.R, 1, 2, 14, 0.0, 1.0, 2, 128, keep_logits=True)
+        commits, leave = 0, {}
+        while not sd.done():
+            sd.step()
+            for u, s in list(leave.items()):
+                if sd.stats.steps == s:
+                    assert u not in sd.branches
+                    del leave[u]
+                else:
+                    assert u in sd.branches and sd.branches[u].retiring
+            if sd.done():
+                break
+            root = sd.root()
+            if sd.stats.steps >= (3, 8, 1 << 30)[commits] and root.child1 in sd.branches:
+                sd.commit_branch(root.child1)
+                commits += 1
+                leave[root.uid] = sd.stats.steps + cfg.R - root.depth
+            elif sd.stats.steps == 6:
+                others = [u for u, b in sd.branches.items() if u != root.uid and not b.retiring]
+                if others:
+                    sd.rollback(max(others))
+        assert commits == 2 and not leave
+        return sd
+
+    a, b = run(np.nan), run(0.0)
+    assert all(np.isfinite(z).all() for z in a.logits.values())
+    assert a.committed == b.committed and a.src == b.src
 
 
 def _ancestors(sd, b):
