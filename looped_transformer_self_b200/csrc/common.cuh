@@ -137,6 +137,9 @@ struct GemmShape {
   int k;         // reduction length
   int kch;       // stream-K units per tile (groups of kc k-chunks)
   int kc;        // k-chunks (128 bytes of K each) per unit: one TMA request per operand
+  int l2_own;    // weight bytes per CTA of its own range requested into L2 beyond the ring
+  int l2_next;   // weight bytes per CTA of the next GEMM's slice requested into L2
+  int prewait;   // ring stages of weights requested before the dependency wait
   int nch;       // k-chunks per tile, ceil(K / chunk)
   int nfull;     // k-chunks that lie wholly inside K (units within them load as one 3-D box)
   int tiles;     // ceil(n_out / 128)

@@ -400,7 +400,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   // the kernels in front of it.  Their barriers get the weight bytes now
   // (expect_tx without arrival) and the activation bytes plus the arrival once
   // the activations may be read.
-  const int npre = min(stages, u1 - u0);
+  const int npre = min(min(stages, s.prewait), u1 - u0);
   const uint64_t pol_w = policy_evict_first(), pol_x = policy_evict_last();
   if (warp == 0 && lane == 0) {
     for (int g = 0; g < npre; ++g) {
@@ -412,7 +412,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     // slice of the NEXT GEMM's weights (sNext.units > 0), so HBM keeps
     // streaming weights through this kernel's tail and the kernels that follow
     // (attention, epilogues) until the next GEMM's ring is filled.
-    const int nl2 = min(u1 - u0, npre + GEMM_L2_PREFETCH_BYTES / (int)(KC * A_BYTES));
+    const int nl2 = min(u1 - u0, npre + s.l2_own / (int)(KC * A_BYTES));
     for (int g = npre; g < nl2; ++g) {
       int t, c0;
       const int n = unit_of(u0 + g, t, c0);
@@ -428,7 +428,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     }
     if (sNext.units > 0 && c < sNext.grid) {
       const int v0 = sk_u0(c, sNext.units, sNext.grid), v1 = sk_u0(c + 1, sNext.units, sNext.grid);
-      const int vend = min(v1, v0 + GEMM_L2_PREFETCH_BYTES / (int)(sNext.kc * A_BYTES));
+      const int vend = min(v1, v0 + s.l2_next / (int)(sNext.kc * A_BYTES));
       for (int uu = v0; uu < vend; ++uu) {
         const int t = uu / sNext.kch, c0 = (uu - t * sNext.kch) * sNext.kc;
         if (sNext.kc > 1 && c0 + sNext.kc <= sNext.nfull) {
@@ -668,6 +668,12 @@ GemmTuning gemm_tuning() {
     e = getenv("LT_GEMM_SMEM_KB");
     const int kb = e ? atoi(e) : (v.kc <= 2 ? 112 : 220);
     v.smem_budget = std::min(std::max(kb, 48), 224) * 1024;
+    e = getenv("LT_GEMM_L2_OWN_KB");
+    v.l2_own = std::max(0, e ? atoi(e) : 0) * 1024;
+    e = getenv("LT_GEMM_L2_NEXT_KB");
+    v.l2_next = std::max(0, e ? atoi(e) : 0) * 1024;
+    e = getenv("LT_GEMM_PREWAIT");
+    v.prewait = e ? std::max(0, atoi(e)) : 16;
     return v;
   }();
   return t;
@@ -706,6 +712,9 @@ void gemm_plan(int n_out, int k, bool f32, int ncols, int grid_cap, GemmShape* s
   s->n_out = n_out;
   s->k = k;
   s->kc = gemm_kc(ncols, f32);
+  s->l2_own = gemm_tuning().l2_own;
+  s->l2_next = gemm_tuning().l2_next;
+  s->prewait = gemm_tuning().prewait;
   s->nch = (k + bke - 1) / bke;
   s->nfull = k / bke;
   s->kch = (s->nch + s->kc - 1) / s->kc;

@@ -44,10 +44,6 @@ constexpr int GEMM_BM = 128;            // output features per tile (MMA M)
 constexpr int GEMM_CHUNK_BYTES = 128;   // K bytes per k-chunk (one 128B-swizzle row)
 constexpr int GEMM_THREADS = 192;       // warp 0: TMA, warp 1: MMA, warps 2-5: drain
 constexpr int GEMM_MAX_SEGS = 16;       // tiles one CTA may touch in a GEMM with an epilogue
-// Weight bytes per CTA requested into L2 ahead of use, for this GEMM's range
-// beyond the ring and for the next GEMM's slice (148 CTAs: <= 47 MB each, well
-// inside the 126 MB L2).
-constexpr int GEMM_L2_PREFETCH_BYTES = 320 * 1024;
 
 // Ring geometry: k-chunks per stage (kc in {1, 2, 4}) and the shared-memory
 // budget of the ring.  Default: kc 4 in ~218 KB (three 72 KB stages at 16
@@ -55,9 +51,16 @@ constexpr int GEMM_L2_PREFETCH_BYTES = 320 * 1024;
 // beside this one, but measured slower on the Ouro-1.4B decode step (1.70 vs
 // 1.56 ms).  LT_GEMM_KC and LT_GEMM_SMEM_KB override them (read once per
 // process).
+// Weight bytes per CTA requested into L2 ahead of use: l2_own for this GEMM's
+// range beyond the ring, l2_next for the next GEMM's slice (default 0: with
+// 64 KB stages the ring requested before the dependency wait already keeps
+// HBM busy; LT_GEMM_L2_OWN_KB / LT_GEMM_L2_NEXT_KB override).
 struct GemmTuning {
   int kc;
   int smem_budget;
+  int l2_own;
+  int l2_next;
+  int prewait;  // ring stages of weights requested before the dependency wait (LT_GEMM_PREWAIT)
 };
 GemmTuning gemm_tuning();
 // Chunks per unit for this operand width (kc reduced until two stages fit).
