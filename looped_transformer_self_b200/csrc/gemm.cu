@@ -7,259 +7,10 @@
 #include <type_traits>
 
 #include "gemm.cuh"
+#include "gemm_epi.cuh"
+#include "tc.cuh"
 
 namespace lt {
-
-// ---------------------------------------------------------------------------
-// PTX wrappers
-// ---------------------------------------------------------------------------
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return (uint32_t)__cvta_generic_to_shared(p);
-}
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
-               : "memory");
-}
-// Adds expected transaction bytes to the current phase without arriving.
-__device__ __forceinline__ void mbar_expect_tx_only(uint32_t bar, uint32_t bytes) {
-  asm volatile("mbarrier.expect_tx.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}\n"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-constexpr long long WAIT_LIMIT_CYCLES = 2000000000LL;  // ~1 s at 1.9 GHz
-
-// Bounded wait on an mbarrier phase; false when it gave up (or another role did).
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const long long t0 = clock64();
-  while (!mbar_try_wait(bar, parity)) {
-    if (*abort_flag) return false;
-    if (clock64() - t0 > WAIT_LIMIT_CYCLES) {
-      *abort_flag = 1;
-      return false;
-    }
-  }
-  return true;
-}
-
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y,
-                                            uint32_t bar, uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      ".L2::cache_hint [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar), "l"(policy)
-      : "memory");
-}
-// 3-D box (128-byte rows x rows x chunks): a k-group of kc swizzled tiles.
-__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int y, int z,
-                                            uint32_t bar, uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      ".L2::cache_hint [%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(0), "r"(y), "r"(z), "r"(bar), "l"(policy)
-      : "memory");
-}
-__device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap* map, int y, int z) {
-  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
-                   reinterpret_cast<uint64_t>(map)),
-               "r"(0), "r"(y), "r"(z)
-               : "memory");
-}
-// Pulls one weight tile into L2 (no shared memory, no barrier).
-__device__ __forceinline__ void tma_prefetch_l2(const CUtensorMap* map, int x, int y) {
-  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
-                   reinterpret_cast<uint64_t>(map)),
-               "r"(x), "r"(y)
-               : "memory");
-}
-__device__ __forceinline__ uint64_t policy_evict_first() {
-  uint64_t p;
-  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
-  return p;
-}
-__device__ __forceinline__ uint64_t policy_evict_last() {
-  uint64_t p;
-  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
-  return p;
-}
-
-__device__ __forceinline__ void tc_fence_before() {
-  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_after() {
-  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_commit(uint32_t bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                   bar)
-               : "memory");
-}
-template <bool TF32>
-__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
-                                       uint32_t idesc, uint32_t accumulate) {
-  if constexpr (TF32) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-        : "memory");
-  } else {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-        : "memory");
-  }
-}
-// 32 lanes x 32 bits, 8 consecutive columns.
-__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t* r) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7])
-      : "r"(taddr)
-      : "memory");
-}
-__device__ __forceinline__ void tmem_wait_ld() {
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
-
-// Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, 8-row
-// atoms of 1024 bytes (stride byte offset 1024), sm100 descriptor version 1.
-__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr) {
-  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) |
-         ((uint64_t)(1024 >> 4) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
-}
-
-// Instruction descriptor: D fp32, A/B bf16 (kind::f16) or tf32 (kind::tf32),
-// both K-major, N = ncols, M = 128.
-template <bool TF32, int NC>
-__device__ __forceinline__ constexpr uint32_t instr_desc() {
-  return (1u << 4) | ((TF32 ? 2u : 1u) << 7) | ((TF32 ? 2u : 1u) << 10) |
-         ((uint32_t)(NC >> 3) << 17) | ((uint32_t)(GEMM_BM >> 4) << 24);
-}
-
-template <int NC>
-constexpr int tmem_cols() {
-  return (2 * NC) <= 32 ? 32 : (2 * NC) <= 64 ? 64 : (2 * NC) <= 128 ? 128 : 256;
-}
-
-// ---------------------------------------------------------------------------
-// in-GEMM epilogues (run by the 4 drain warps of the CTA completing a group)
-// ---------------------------------------------------------------------------
-__device__ __forceinline__ void drain_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
-
-template <typename TX>
-__device__ __forceinline__ void store_x(TX* X, size_t idx, float v, size_t lo);
-template <>
-__device__ __forceinline__ void store_x<__nv_bfloat16>(__nv_bfloat16* X, size_t idx, float v,
-                                                       size_t) {
-  X[idx] = __float2bfloat16_rn(v);
-}
-template <>
-__device__ __forceinline__ void store_x<float>(float* X, size_t idx, float v, size_t lo) {
-  if (lo) {  // split tf32 pair
-    const float hi = __uint_as_float(__float_as_uint(v) & 0xFFFFE000u);
-    X[idx] = hi;
-    X[lo + idx] = v - hi;
-  } else {
-    X[idx] = v;
-  }
-}
-template <typename TX>
-__device__ __forceinline__ float load_g(const void* g, int n) {
-  return (float)(reinterpret_cast<const TX*>(g)[n]);
-}
-
-struct EpiSmem {
-  int rows[64];      // active rows of this launch
-  int nact;
-  int last;          // group completed by this CTA, or -1
-  float inv[64];     // per active row: 1 / rms (SwiGLU)
-  float wsum[4][64]; // per warp, per active row: partial sum of squares
-  int4 ti[8][2];     // per segment of this CTA: table entries of its group's tiles
-  unsigned long long target[GEMM_MAX_SEGS];  // per segment: arrival count completing its group
-};
-
-// Residual epilogue of one tile for active rows r0 .. r1-1 (indices into
-// sm.rows): h += scale * y; X = g (.) h; sum-of-squares part of those rows.
-template <typename TX>
-__device__ void epi_resid(const GemmEpi& ep, const float* __restrict__ part, const GemmShape& s,
-                          int ncols, int t, int4 ti, int r0, int r1, int et, EpiSmem& sm) {
-  const int n = t * 128 + et;
-  const bool valid = n < s.n_out;
-  const int lane = et & 31, w = et >> 5;
-  for (int k0 = r0; k0 < r1; k0 += 4) {
-    const int nr = min(4, r1 - k0);
-    float y[4], h0[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u)  // h rows first: their loads overlap the partials'
-      h0[u] = (valid && u < nr) ? __ldcg(ep.h + (size_t)sm.rows[k0 + u] * ep.d + n) : 0.f;
-    tile_sum4<12>(part, s, ti, ncols, sm.rows + k0, nr, n & 127, y);
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      if (u >= nr) break;
-      const int i = sm.rows[k0 + u];
-      float hv = 0.f;
-      if (valid) {
-        hv = h0[u] + ep.scale * y[u];
-        ep.h[(size_t)i * ep.d + n] = hv;
-        if (ep.g)
-          store_x<TX>(reinterpret_cast<TX*>(ep.X), (size_t)i * ep.d + n, load_g<TX>(ep.g, n) * hv,
-                      ep.lo);
-      }
-      float sq = hv * hv;
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
-      if (lane == 0) sm.wsum[w][k0 + u] = sq;
-    }
-  }
-  drain_sync();
-  if (et >= r0 && et < r1) {
-    const float v = sm.wsum[0][et] + sm.wsum[1][et] + sm.wsum[2][et] + sm.wsum[3][et];
-    ep.ssq_out[(size_t)t * ncols + sm.rows[et]] = v;
-  }
-}
-
-// SwiGLU epilogue of one (gate tile g, up tile g + ffn/128) pair for active
-// rows r0 .. r1-1; sm.inv was filled during the mainloop.
-template <typename TX>
-__device__ void epi_swiglu(const GemmEpi& ep, const float* __restrict__ part, const GemmShape& s,
-                           int ncols, int g, int4 tg, int4 tu, int r0, int r1, int et,
-                           EpiSmem& sm) {
-  const int n = g * 128 + et;
-  if (n >= ep.ffn) return;
-  for (int k0 = r0; k0 < r1; k0 += 4) {
-    const int nr = min(4, r1 - k0);
-    float gv[4], uv[4];
-    tile_sum4<4>(part, s, tg, ncols, sm.rows + k0, nr, n & 127, gv);
-    tile_sum4<4>(part, s, tu, ncols, sm.rows + k0, nr, n & 127, uv);
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      if (u >= nr) break;
-      const float r = sm.inv[k0 + u];
-      const float g = r * gv[u], up = r * uv[u];
-      store_x<TX>(reinterpret_cast<TX*>(ep.X), (size_t)sm.rows[k0 + u] * ep.ffn + n,
-                  g / (1.f + __expf(-g)) * up, ep.lo);
-    }
-  }
-}
 
 // ---------------------------------------------------------------------------
 // kernel
@@ -557,12 +308,23 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       if (ep.kind == EPI_SWIGLU && et < esm.nact)
         esm.inv[et] = inv_rms_parts(ep.ssq_in, ep.ssq_tiles, NC, esm.rows[et], ep.d, ep.eps);
     }
+    // Thread 0 takes every continue / stop decision and shares it through
+    // esm.okb / esm.ok after a drain barrier, so the 128 drain threads always reach the
+    // same barriers (an abort seen by some threads only would strand the rest).
+    bool dead = false;
     int seg = 0;
     for (int u = u0; u < u1; ++seg) {
       const int t = u / s.kch;
       const int seg_end = min(u1, (t + 1) * s.kch);
       const int b = seg & 1, use = seg >> 1;
-      if (!mbar_wait(accf_bar(b), use & 1, abort_flag)) break;
+      // (two slots: a slot is rewritten only after the next barrier, which every
+      // thread passes after reading it)
+      if (et == 0) esm.okb[seg & 1] = mbar_wait(accf_bar(b), use & 1, abort_flag) ? 1 : 0;
+      drain_sync();
+      if (!esm.okb[seg & 1]) {
+        dead = true;
+        break;
+      }
       tc_fence_after();
       uint32_t r[NC];
       const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * NC);
@@ -599,7 +361,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     // segments; a CTA that waits has published everything, and the grid (<= one
     // CTA per SM) is wholly resident before any dependent grid launches, so the
     // waits form no cycle.
-    if (ep.kind != EPI_NONE && !*abort_flag) {
+    if (ep.kind != EPI_NONE && !dead) {
       const int t0 = u0 / s.kch, nseg = min((u1 - 1) / s.kch - t0 + 1, GEMM_MAX_SEGS);
       const bool sw = ep.kind == EPI_SWIGLU;
       const int groups = sw ? ep.ffn / GEMM_BM : s.tiles;
@@ -625,9 +387,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
               break;
             }
           }
+          esm.ok = *abort_flag ? 0 : 1;
         }
         drain_sync();
-        if (*abort_flag) break;
+        if (!esm.ok) break;
         const int r0 = share * esm.nact / need, r1 = (share + 1) * esm.nact / need;
         if (r1 > r0) {
           if (!sw) epi_resid<TX>(ep, part, s, NC, t, ta, r0, r1, et, esm);

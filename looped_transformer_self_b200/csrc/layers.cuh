@@ -253,9 +253,8 @@ struct RawVec {
 // Block (row i, head h, split sp) covers positions [sp*CH, min(sp*CH+CH, pos+1)) of
 // the row's own prefix (committed slots, then the ancestors' and its own slot),
 // all read from the row's depth plane.  16 lanes share one cache row (HD/16
-// elements each, vector loads); each half-warp keeps att_u<T>() positions' K and
-// V loads in flight (16 for bf16 caches: a 128-position split is one round of
-// loads) and folds them into an online softmax (one pass over the cache).  The 8 half-warps merge in fixed order; the split's (max, sum,
+// elements each, vector loads); each half-warp keeps 8 positions' K and V loads
+// in flight and folds them into an online softmax (one pass over the cache).  The 8 half-warps merge in fixed order; the split's (max, sum,
 // unnormalised acc) goes to `opart`, and the last block of the (row, head) to
 // finish merges all splits in split order and writes the O-GEMM input row
 // (deterministic whichever block comes last).
@@ -270,82 +269,85 @@ struct RawVec {
 // QKV epilogue first (FUSED = false) and reads q from `q`.
 template <typename T>
 __host__ __device__ constexpr int att_u() {  // positions per half-warp in flight
-  return sizeof(T) == 2 ? 16 : 8;
+  return 8;
 }
 
-template <typename T, int HD, bool FUSED>
-__global__ void __launch_bounds__(128) k_attn(
-    const float* __restrict__ q, T* __restrict__ kv, int plane_base,
-    const int* __restrict__ tagsrc, int tag_off, int S, int d, int H,
-    const int* __restrict__ mask, const int* __restrict__ r_pos, const int* __restrict__ r_blen,
-    const int* __restrict__ r_boff, const int* __restrict__ lists, const int* __restrict__ chain,
-    int W, int max_splits, float* __restrict__ opart, int* __restrict__ counters,
-    T* __restrict__ X, size_t lo, const float* __restrict__ part, const GemmShape qs_shape, int C,
-    const int* __restrict__ r_slot, const float2* __restrict__ rope,
-    const float* __restrict__ ssq, int ssq_tiles, float eps, int* err) {
+// Everything one attention work item reads or writes (device pointers).
+struct AttnArgs {
+  const float* q;            // [C][d] queries (prefill; FUSED reads the QKV partials)
+  void* kv;                  // cache pool (T)
+  int plane_base;            // first plane of this layer
+  const int* tagsrc;         // per row: plane offset (depth or readout tag), or null
+  int tag_off;
+  int S, d, H;               // slots, model width, heads
+  const int* r_pos;
+  const int* r_blen;
+  const int* r_boff;
+  const int* lists;
+  const int* chain;
+  int W, max_splits;
+  float* opart;              // [C][H][max_splits][HD + 2] split partials
+  int* counters;             // [C][H] split tickets (the last block resets)
+  void* X;                   // [C][d] O-GEMM operand rows (T)
+  size_t lo;                 // fp32 models: offset of the low tf32 plane
+  const float* part;         // QKV GEMM partials (FUSED)
+  GemmShape qs_shape;
+  int C;
+  const int* r_slot;
+  const float2* rope;
+  const float* ssq;          // RMSNorm sum-of-squares tile parts of the rows (FUSED)
+  int ssq_tiles;
+  float eps;
+  int* err;
+  int kv_prefetch;           // 1: request the item's K/V rows into L2 before the dependency wait
+};
+
+template <int HD>
+struct AttnSmem {
+  float qsm[HD];
+  int sl[ATT_CH];
+  float hm[8], hl[8];
+  float hacc[8][HD];
+  int last;
+};
+
+// One work item: (row i, head h, 128-position split sp of ns).  Run by 128
+// threads (tid 0..127); `bar` synchronises them, `dep` returns once the
+// inputs written by the preceding phase may be read (the QKV partials, the
+// rows' sums of squares).  Work that does not need them -- the slot list, L2
+// requests for the K/V rows and (RR_EARLY) the row's RMSNorm factor -- comes
+// first.  Returns true in the block that merged the row's splits (written X).
+template <typename T, int HD, bool FUSED, bool RR_EARLY, class Bar, class Dep>
+__device__ bool attn_item(const AttnArgs& a, AttnSmem<HD>& sm, int h, int i, int sp, int ns,
+                          int tid, Bar bar, Dep dep) {
   constexpr int EPL = HD / 16;
-  __shared__ float qsm[HD];
-  __shared__ int sl[ATT_CH];
-  __shared__ float hm[8], hl[8];
-  __shared__ float hacc[8][HD];
-  __shared__ int last;
-  __shared__ int s_item[3];
-  // Block (head h, y): items are the active rows' splits, rows in order; block y
-  // takes items y, y + gridDim.y, ...  The grid holds about one resident wave
-  // (a grid of every possible item would be mostly empty blocks, each still
-  // scheduled and retired before the O GEMM may start).  Row bookkeeping, slot
-  // lists, the cache rows of earlier positions and (fused) the RMSNorm sums of
-  // squares were written by kernels that finished before this grid was
-  // launched: for the first item they are read -- and the block's K/V rows are
-  // requested into L2 -- before the dependency wait, while the QKV GEMM in
-  // front of this kernel still runs.
-  const int h = blockIdx.x;
-  for (int item = blockIdx.y, it = 0;; item += gridDim.y, ++it) {
-  if (threadIdx.x == 0) {
-    int acc = 0, row = -1, spl = 0, nsr = 0;
-#pragma unroll 8
-    for (int k = 0; k < C; ++k) {
-      const int nk = mask[k] ? (r_pos[k] + ATT_CH) / ATT_CH : 0;
-      if (row < 0 && item < acc + nk) {
-        row = k;
-        spl = item - acc;
-        nsr = nk;
-      }
-      acc += nk;
-    }
-    s_item[0] = row;
-    s_item[1] = spl;
-    s_item[2] = nsr;
-  }
-  __syncthreads();
-  const int i = s_item[0], sp = s_item[1], ns = s_item[2];
-  if (i < 0) {
-    if (it == 0) {
-      pdl_wait();
-      pdl_trigger();
-    }
-    break;
-  }
-  const int n = r_pos[i] + 1;
+  constexpr int NT = 128;
+  T* const kv = reinterpret_cast<T*>(a.kv);
+  const int S = a.S, d = a.d, H = a.H, C = a.C;
+  const int n = a.r_pos[i] + 1;
   const int start = sp * ATT_CH;
   const int cnt = min(ATT_CH, n - start);
-  const int plane = plane_base + (tagsrc ? tagsrc[i] : 0) + tag_off;
+  const int plane = a.plane_base + (a.tagsrc ? a.tagsrc[i] : 0) + a.tag_off;
   {
-    const int blen = r_blen[i], boff = r_boff[i];
-    for (int t = threadIdx.x; t < cnt; t += blockDim.x) {
+    const int blen = a.r_blen[i], boff = a.r_boff[i];
+    for (int t = tid; t < cnt; t += NT) {
       const int j = start + t;
-      int s = j < blen ? lists[boff + j] : chain[i * W + (j % W)];
+      int s = j < blen ? a.lists[boff + j] : a.chain[i * a.W + (j % a.W)];
       if (s < 0 || s >= S) {
-        set_err(err, DEV_BAD_INDEX);
+        set_err(a.err, DEV_BAD_INDEX);
         s = 0;
       }
-      sl[t] = s;
-      const T* kr = kv + kv_off<T>(plane, s, 0, S, d) + (size_t)h * HD;
-      const T* vr = kv + kv_off<T>(plane, s, 1, S, d) + (size_t)h * HD;
-      asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(kr), "r"((int)(HD * sizeof(T)))
-                   : "memory");
-      asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(vr), "r"((int)(HD * sizeof(T)))
-                   : "memory");
+      sm.sl[t] = s;
+      if (a.kv_prefetch) {
+        const T* kr = kv + kv_off<T>(plane, s, 0, S, d) + (size_t)h * HD;
+        const T* vr = kv + kv_off<T>(plane, s, 1, S, d) + (size_t)h * HD;
+        asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(kr),
+                     "r"((int)(HD * sizeof(T)))
+                     : "memory");
+        asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(vr),
+                     "r"((int)(HD * sizeof(T)))
+                     : "memory");
+      }
     }
   }
   // fused prologue inputs that do not depend on the QKV GEMM
@@ -357,41 +359,39 @@ __global__ void __launch_bounds__(128) k_attn(
   int nA = 0, nB = 0, nV = 0;
   bool is_k = false;
   if constexpr (FUSED) {
-    rr = inv_rms_parts(ssq, ssq_tiles, C, i, d, eps);
-    const int t = threadIdx.x;
+    if constexpr (RR_EARLY) rr = inv_rms_parts(a.ssq, a.ssq_tiles, C, i, d, a.eps);
+    const int t = tid;
     if (t < 2 * half) {
       const int e = t < half ? t : t - half;
       is_k = t >= half;
       nA = (is_k ? d : 0) + h * HD + e;
       nB = nA + half;
-      tiA = __ldg(qs_shape.tinfo + (nA >> 7));
-      tiB = __ldg(qs_shape.tinfo + (nB >> 7));
-      cs = rope[(size_t)(n - 1) * half + e];
+      tiA = __ldg(a.qs_shape.tinfo + (nA >> 7));
+      tiB = __ldg(a.qs_shape.tinfo + (nB >> 7));
+      cs = a.rope[(size_t)(n - 1) * half + e];
     }
     if (t < HD) {
       nV = 2 * d + h * HD + t;
-      tiV = __ldg(qs_shape.tinfo + (nV >> 7));
+      tiV = __ldg(a.qs_shape.tinfo + (nV >> 7));
     }
   }
-  if (it == 0) {
-    pdl_wait();
-    pdl_trigger();
-  }
-  const int hw = threadIdx.x >> 4, l16 = threadIdx.x & 15;
+  dep();
+  if constexpr (FUSED && !RR_EARLY) rr = inv_rms_parts(a.ssq, a.ssq_tiles, C, i, d, a.eps);
+  const int hw = tid >> 4, l16 = tid & 15;
   const float scale = rsqrtf((float)HD);
   float qv[EPL];
   if constexpr (FUSED) {
-    const int slot = r_slot[i];
+    const int slot = a.r_slot[i];
     T* krow = kv + kv_off<T>(plane, slot, 0, S, d) + (size_t)h * HD;
     T* vrow = kv + kv_off<T>(plane, slot, 1, S, d) + (size_t)h * HD;
-    const int t = threadIdx.x;
+    const int t = tid;
     float a1 = 0.f, a2 = 0.f, av = 0.f;
     const bool do_pair = t < 2 * half && (!is_k || own);
     if (do_pair) {
-      a1 = rr * sk_reduce_ti(part, qs_shape, tiA, C, i, nA);
-      a2 = rr * sk_reduce_ti(part, qs_shape, tiB, C, i, nB);
+      a1 = rr * sk_reduce_ti(a.part, a.qs_shape, tiA, C, i, nA);
+      a2 = rr * sk_reduce_ti(a.part, a.qs_shape, tiB, C, i, nB);
     }
-    if (own && t < HD) av = rr * sk_reduce_ti(part, qs_shape, tiV, C, i, nV);
+    if (own && t < HD) av = rr * sk_reduce_ti(a.part, a.qs_shape, tiV, C, i, nV);
     if (do_pair) {
       const int e = t < half ? t : t - half;
       const float r1 = a1 * cs.x - a2 * cs.y, r2 = a2 * cs.x + a1 * cs.y;
@@ -399,19 +399,19 @@ __global__ void __launch_bounds__(128) k_attn(
         krow[e] = from_f<T>(r1);
         krow[e + half] = from_f<T>(r2);
       } else {
-        qsm[e] = r1;
-        qsm[e + half] = r2;
+        sm.qsm[e] = r1;
+        sm.qsm[e + half] = r2;
       }
     }
     if (own && t < HD) vrow[t] = from_f<T>(av);
-    __syncthreads();  // the own cache row is complete and visible to this block
+    bar();  // the own cache row is complete and visible to these threads
 #pragma unroll
-    for (int e = 0; e < EPL; ++e) qv[e] = qsm[l16 * EPL + e] * scale;
+    for (int e = 0; e < EPL; ++e) qv[e] = sm.qsm[l16 * EPL + e] * scale;
   } else {
-    load_vec<float, EPL>(q + (size_t)i * d + h * HD + l16 * EPL, qv);
+    load_vec<float, EPL>(a.q + (size_t)i * d + h * HD + l16 * EPL, qv);
 #pragma unroll
     for (int e = 0; e < EPL; ++e) qv[e] *= scale;
-    __syncthreads();
+    bar();
   }
   const size_t head_off = (size_t)h * HD + l16 * EPL;
   const T* kbase = kv + kv_off<T>(plane, 0, 0, S, d) + head_off;
@@ -429,7 +429,7 @@ __global__ void __launch_bounds__(128) k_attn(
     for (int u = 0; u < ATT_U; ++u) {
       const int t = t0 + u;
       if (t < cnt) {
-        const size_t off = (size_t)sl[t] * slot_stride;
+        const size_t off = (size_t)sm.sl[t] * slot_stride;
         kx[u].load(kbase + off);
         vx[u].load(vbase + off);
       } else {
@@ -471,85 +471,146 @@ __global__ void __launch_bounds__(128) k_attn(
     m = mnew;
   }
   if (l16 == 0) {
-    hm[hw] = m;
-    hl[hw] = l;
+    sm.hm[hw] = m;
+    sm.hl[hw] = l;
   }
 #pragma unroll
-  for (int e = 0; e < EPL; ++e) hacc[hw][l16 * EPL + e] = acc[e];
-  __syncthreads();
+  for (int e = 0; e < EPL; ++e) sm.hacc[hw][l16 * EPL + e] = acc[e];
+  bar();
   float M = -INFINITY;
 #pragma unroll
-  for (int w = 0; w < 8; ++w) M = fmaxf(M, hm[w]);
-  float* out = opart + ((size_t)(i * H + h) * max_splits + sp) * (HD + 2);
-  for (int e = threadIdx.x; e < HD; e += blockDim.x) {
-    float a = 0.f;
+  for (int w = 0; w < 8; ++w) M = fmaxf(M, sm.hm[w]);
+  float* out = a.opart + ((size_t)(i * H + h) * a.max_splits + sp) * (HD + 2);
+  for (int e = tid; e < HD; e += NT) {
+    float v = 0.f;
 #pragma unroll
     for (int w = 0; w < 8; ++w)
-      if (hm[w] != -INFINITY) a += hacc[w][e] * __expf(hm[w] - M);
-    out[2 + e] = a;
+      if (sm.hm[w] != -INFINITY) v += sm.hacc[w][e] * __expf(sm.hm[w] - M);
+    out[2 + e] = v;
   }
-  if (threadIdx.x == 0) {
+  if (tid == 0) {
     float L = 0.f;
 #pragma unroll
     for (int w = 0; w < 8; ++w)
-      if (hm[w] != -INFINITY) L += hl[w] * __expf(hm[w] - M);
+      if (sm.hm[w] != -INFINITY) L += sm.hl[w] * __expf(sm.hm[w] - M);
     out[0] = M;
     out[1] = L;
   }
-  // the last split block of this (row, head) combines all splits in order
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    const int ticket = atomicAdd(&counters[i * H + h], 1);
-    last = ticket == ns - 1;
-    if (last) counters[i * H + h] = 0;
+  // the last split block of this (row, head) combines all splits in order;
+  // release: the split's stores before the ticket (acq_rel, not a full
+  // sequentially consistent fence)
+  asm volatile("fence.acq_rel.gpu;" ::: "memory");
+  bar();
+  if (tid == 0) {
+    const int ticket = atomicAdd(&a.counters[i * H + h], 1);
+    sm.last = ticket == ns - 1;
+    if (sm.last) a.counters[i * H + h] = 0;
   }
-  __syncthreads();
+  bar();
+  const bool last = sm.last;
   if (last) {
-  __threadfence();
-  // Merge all splits in split order.  One round of independent loads: thread s
-  // fetches split s's (max, sum) into shared memory while every thread fetches
-  // its accumulator element of the first ATT_MB splits; then the weights
-  // exp(max_s - M) come from shared memory.
-  const float* base = opart + (size_t)(i * H + h) * max_splits * (HD + 2);
-  constexpr int ATT_MB = 16;
-  constexpr int CAP = 4 * HD;  // splits whose (max, sum) fit in hacc
-  float* sM = &hacc[0][0];
-  float* sL = sM + CAP;
-  const int e = threadIdx.x;  // element of the head (blockDim >= HD)
-  float av[ATT_MB];
-#pragma unroll
-  for (int k = 0; k < ATT_MB; ++k)
-    av[k] = (e < HD && k < ns) ? __ldcg(base + (size_t)k * (HD + 2) + 2 + e) : 0.f;
-  if (ns <= CAP) {
-    for (int s2 = threadIdx.x; s2 < ns; s2 += blockDim.x) {
-      sM[s2] = __ldcg(base + (size_t)s2 * (HD + 2));
-      sL[s2] = __ldcg(base + (size_t)s2 * (HD + 2) + 1);
-    }
-  }
-  __syncthreads();
-  auto mx_of = [&](int s2) { return ns <= CAP ? sM[s2] : __ldcg(base + (size_t)s2 * (HD + 2)); };
-  auto l_of = [&](int s2) { return ns <= CAP ? sL[s2] : __ldcg(base + (size_t)s2 * (HD + 2) + 1); };
-  float Mx = -INFINITY;
-  for (int s2 = 0; s2 < ns; ++s2) Mx = fmaxf(Mx, mx_of(s2));
-  float Lx = 0.f;
-  for (int s2 = 0; s2 < ns; ++s2) Lx += l_of(s2) * __expf(mx_of(s2) - Mx);
-  if (e < HD) {
-    float o = 0.f;
+    asm volatile("fence.acq_rel.gpu;" ::: "memory");  // acquire: the other splits' stores
+    // Merge all splits in split order.  One round of independent loads: thread s
+    // fetches split s's (max, sum) into shared memory while every thread fetches
+    // its accumulator element of the first ATT_MB splits; then the weights
+    // exp(max_s - M) come from shared memory.
+    const float* base = a.opart + (size_t)(i * H + h) * a.max_splits * (HD + 2);
+    constexpr int ATT_MB = 16;
+    constexpr int CAP = 4 * HD;  // splits whose (max, sum) fit in hacc
+    float* sM = &sm.hacc[0][0];
+    float* sL = sM + CAP;
+    const int e = tid;  // element of the head (128 threads >= HD)
+    float av[ATT_MB];
 #pragma unroll
     for (int k = 0; k < ATT_MB; ++k)
-      if (k < ns) o += av[k] * __expf(mx_of(k) - Mx);
-    for (int s2 = ATT_MB; s2 < ns; ++s2)
-      o += __ldcg(base + (size_t)s2 * (HD + 2) + 2 + e) * __expf(mx_of(s2) - Mx);
-    store_act<T>(X + (size_t)i * d + h * HD, e, o / Lx, lo);
+      av[k] = (e < HD && k < ns) ? __ldcg(base + (size_t)k * (HD + 2) + 2 + e) : 0.f;
+    if (ns <= CAP) {
+      for (int s2 = tid; s2 < ns; s2 += NT) {
+        sM[s2] = __ldcg(base + (size_t)s2 * (HD + 2));
+        sL[s2] = __ldcg(base + (size_t)s2 * (HD + 2) + 1);
+      }
+    }
+    bar();
+    auto mx_of = [&](int s2) { return ns <= CAP ? sM[s2] : __ldcg(base + (size_t)s2 * (HD + 2)); };
+    auto l_of = [&](int s2) { return ns <= CAP ? sL[s2] : __ldcg(base + (size_t)s2 * (HD + 2) + 1); };
+    float Mx = -INFINITY;
+    for (int s2 = 0; s2 < ns; ++s2) Mx = fmaxf(Mx, mx_of(s2));
+    float Lx = 0.f;
+    for (int s2 = 0; s2 < ns; ++s2) Lx += l_of(s2) * __expf(mx_of(s2) - Mx);
+    if (e < HD) {
+      float o = 0.f;
+#pragma unroll
+      for (int k = 0; k < ATT_MB; ++k)
+        if (k < ns) o += av[k] * __expf(mx_of(k) - Mx);
+      for (int s2 = ATT_MB; s2 < ns; ++s2)
+        o += __ldcg(base + (size_t)s2 * (HD + 2) + 2 + e) * __expf(mx_of(s2) - Mx);
+      store_act<T>(reinterpret_cast<T*>(a.X) + (size_t)i * d + h * HD, e, o / Lx, a.lo);
+    }
   }
-  }  // last
-  __syncthreads();  // shared memory is reused by the next item
-  }  // items
+  bar();  // shared memory is reused by the next item
+  return last;
+}
+
+// Items of the active rows in row order: item -> (row, split, the row's
+// split count); row = -1 past the last item.  One thread.
+__device__ __forceinline__ int3 attn_resolve(const int* __restrict__ mask,
+                                             const int* __restrict__ r_pos, int C, int item) {
+  int acc = 0, row = -1, spl = 0, nsr = 0;
+#pragma unroll 8
+  for (int k = 0; k < C; ++k) {
+    const int nk = mask[k] ? (r_pos[k] + ATT_CH) / ATT_CH : 0;
+    if (row < 0 && item < acc + nk) {
+      row = k;
+      spl = item - acc;
+      nsr = nk;
+    }
+    acc += nk;
+  }
+  return make_int3(row, spl, nsr);
+}
+
+// Block (head h, y): block y takes items y, y + gridDim.y, ...  The grid holds
+// about one resident wave (a grid of every possible item would be mostly empty
+// blocks, each still scheduled and retired before the O GEMM may start).  Row
+// bookkeeping, slot lists, the cache rows of earlier positions and (fused) the
+// RMSNorm sums of squares were written by kernels that finished before this
+// grid was launched: for the first item they are read -- and the block's K/V
+// rows are requested into L2 -- before the dependency wait, while the QKV GEMM
+// in front of this kernel still runs.
+template <typename T, int HD, bool FUSED>
+__global__ void __launch_bounds__(128) k_attn(const AttnArgs a, const int* __restrict__ mask) {
+  __shared__ AttnSmem<HD> sm;
+  __shared__ int s_item[3];
+  const int h = blockIdx.x;
+  for (int item = blockIdx.y, it = 0;; item += gridDim.y, ++it) {
+    if (threadIdx.x == 0) {
+      const int3 r = attn_resolve(mask, a.r_pos, a.C, item);
+      s_item[0] = r.x;
+      s_item[1] = r.y;
+      s_item[2] = r.z;
+    }
+    __syncthreads();
+    const int i = s_item[0], sp = s_item[1], ns = s_item[2];
+    if (i < 0) {
+      if (it == 0) {
+        pdl_wait();
+        pdl_trigger();
+      }
+      break;
+    }
+    attn_item<T, HD, FUSED, true>(
+        a, sm, h, i, sp, ns, threadIdx.x, [] { __syncthreads(); },
+        [it] {
+          if (it == 0) {
+            pdl_wait();
+            pdl_trigger();
+          }
+        });
+  }
 }
 
 // ---- RoPE table: (cos, sin) of pos * theta^(-2e/hd), computed in double ------------
-__global__ void k_rope_table(float2* __restrict__ rope, int max_pos, int hd, double theta) {
+static __global__ void k_rope_table(float2* __restrict__ rope, int max_pos, int hd, double theta) {
   const int half = hd / 2;
   const int idx = blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= max_pos * half) return;
