@@ -371,14 +371,13 @@ static AttnArgs attn_args(Handle* H, int gl, const int* tagsrc, int tag_off, voi
   return a;
 }
 
+// Long contexts: one block per (head, work item) slot, blocks looping over items
+// (k_attn; the same bits as k_attn2).
 template <typename T, int HD>
-static cudaError_t attention(Handle* H, int gl, const int* tagsrc, int tag_off, const int* mask,
-                             T* Xo, bool fused) {
-  ProfScope ps(H, 2, 0.0);
+static cudaError_t attention_items(Handle* H, int gl, const int* tagsrc, int tag_off,
+                                   const int* mask, T* Xo, bool fused) {
   const int C = H->C, Hn = H->m.n_heads;
   auto kern = fused ? k_attn<T, HD, true> : k_attn<T, HD, false>;
-  // grid: (head, y); block y takes work items y, y + gy, ... (items = active
-  // rows' 128-position splits); gy: one resident wave of blocks
   static int per_sm[2] = {0, 0};
   int& nb = per_sm[fused ? 1 : 0];
   if (nb == 0 && (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kern, 128, 0) != cudaSuccess ||
@@ -387,6 +386,37 @@ static cudaError_t attention(Handle* H, int gl, const int* tagsrc, int tag_off, 
   const int gy = std::max(1, std::min(C * H->max_splits, nb * sm_count() / Hn));
   return launch(H->use_pdl, kern, dim3(Hn, gy), dim3(128), H->stream,
                 attn_args(H, gl, tagsrc, tag_off, (void*)Xo), mask);
+}
+
+template <typename T, int HD>
+static cudaError_t attention(Handle* H, int gl, const int* tagsrc, int tag_off, const int* mask,
+                             T* Xo, bool fused) {
+  ProfScope ps(H, 2, 0.0);
+  if (H->dc.max_ctx > ATT_RING_MAX_CTX) return attention_items<T, HD>(H, gl, tagsrc, tag_off, mask, Xo, fused);
+  auto kern = fused ? k_attn2<T, HD, true> : k_attn2<T, HD, false>;
+  // one resident wave of ring blocks (items are spread over them)
+  const size_t smem = a2_smem_bytes<T, HD>();
+  static int per_sm[2] = {0, 0};
+  int& nb = per_sm[fused ? 1 : 0];
+  if (nb == 0) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess)
+      return cudaErrorInvalidValue;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kern, 128, smem) != cudaSuccess || nb < 1)
+      nb = 1;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(nb * sm_count());
+  cfg.blockDim = dim3(128);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = H->stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = H->use_pdl ? 1 : 0;
+  if (H->counting) H->kernels_per_step++;
+  return cudaLaunchKernelEx(&cfg, kern, attn_args(H, gl, tagsrc, tag_off, (void*)Xo), mask);
 }
 
 // kind: 0 prelude (one cache), 1 shared block (cache of the row's depth), 2 coda
