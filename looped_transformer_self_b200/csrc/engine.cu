@@ -84,6 +84,7 @@ struct Handle {
   int prof_cat = 0;  // 0: shared-block layer, 1: prelude / coda / head
   struct Ev {
     int kind;  // 0 gemm core, 1 gemm other, 2 attention
+    int gate;  // device flag that lets the launch work: 0 none, 1 run, 2 new rows, 3 readouts
     double bytes;
     cudaEvent_t a, b;
   };
@@ -95,10 +96,11 @@ struct Handle {
 struct ProfScope {
   Handle* H;
   int idx = -1;
-  ProfScope(Handle* h, int kind, double bytes) : H(h) {
+  ProfScope(Handle* h, int kind, double bytes, int gate = 0) : H(h) {
     if (!H->profiling) return;
     Handle::Ev e;
     e.kind = kind;
+    e.gate = gate;
     e.bytes = bytes;
     cudaEventCreate(&e.a);
     cudaEventCreate(&e.b);
@@ -328,7 +330,9 @@ static cudaError_t gemm(Handle* H, const GemmOperand& tw, const GemmOperand& twl
   // activation rows and the fp32 result rows
   const double bytes = split * esz * ((double)s.n_out * s.k + (double)H->C * s.k) +
                        4.0 * H->C * s.n_out;
-  ProfScope ps(H, H->prof_cat, bytes);
+  const Ctl* ctl = H->D.ctl;
+  const int gate = flag == &ctl->flag_run ? 1 : flag == &ctl->flag_new ? 2 : flag == &ctl->flag_ro ? 3 : 0;
+  ProfScope ps(H, H->prof_cat, bytes, gate);
   if (H->counting) H->kernels_per_step++;
   return gemm_launch(tw, twl, tx, txl, H->part, s, H->C, H->mode, flag, &H->D.ctl->err,
                      H->stream, H->use_pdl, epi, next_w, next_s);
@@ -605,7 +609,7 @@ static cudaError_t run_pass(Handle* H) {
   double bytes = 0;
   for (const GemmShape* s : {&H->sh_qkv, &H->sh_o, &H->sh_gu, &H->sh_d})
     bytes += 2.0 * ((double)s->n_out * s->k + (double)C * s->k) + 4.0 * C * s->n_out;
-  ProfScope ps(H, 0, bytes * m.n_core);
+  ProfScope ps(H, 0, bytes * m.n_core, 1);
   if (H->counting) H->kernels_per_step++;
   return pass_launch(H->pp, C, m.head_dim, H->stream);
 }
@@ -1232,6 +1236,10 @@ extern "C" int lt_profile_steps(lt_handle* hd, int ar_mode, int n_steps, lt_prof
     for (auto& ev : H->evs) {
       float t = 0.f;
       cudaEventElapsedTime(&t, ev.a, ev.b);
+      // a GEMM whose flag was clear this step exited without reading its weights
+      const int live = ev.gate == 0 || (ev.gate == 1 && c.flag_run) ||
+                       (ev.gate == 2 && c.flag_new) || (ev.gate == 3 && c.flag_ro);
+      if (!live) ev.bytes = 0.0;
       if (ev.kind == 0) {
         out->gemm_core_ms += t;
         out->gemm_core_launches += 1;
