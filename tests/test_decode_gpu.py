@@ -178,6 +178,32 @@ def test_tiny_sampled_spec_matches_oracle(tiny):
     assert st["gate_opens"] == sp_o.stats.gate_opens
 
 
+@pytest.mark.parametrize("mode,name", [(1, "ungated"), (2, "masked")])
+def test_tiny_sampled_ablation_modes_match_oracle(tiny, mode, name):
+    """The ablation modes of the second proposal (LoopSpec section 3.4): the
+    residual without the gate (second_mode 1) and the non-residual draft from
+    p_d2 with x1 masked out (second_mode 2) -- tokens, commit sources, steps,
+    branch rows and gate-open counts match the oracle's same mode."""
+    from oracle import decode as D
+    from oracle.model import LoopedModel
+    cfg, w, prompt = tiny
+    dec = syn.DECODES["tiny_sample"]
+    n = 32
+    sp_o = D.decode_spec(D.OracleRows(LoopedModel(cfg, w, 256)), prompt, cfg.R, dec.d1, dec.d2, n,
+                         dec.temperature, dec.top_p, dec.seed, 256, second=name)
+    g = _decoder(cfg, dec, w, second_mode=mode)
+    first, _, _ = g.prefill(prompt)
+    toks, st = g.generate(n)
+    gpu = [first] + toks
+    same = next((i for i, (a, b) in enumerate(zip(gpu, sp_o.tokens)) if a != b), None)
+    assert same is None, (same, gpu, sp_o.tokens)
+    _, src, step = g.read_log(n)
+    assert src == sp_o.src and step == sp_o.commit_step
+    assert g.read_trace(st["steps"]) == sp_o.trace
+    assert st["gate_opens"] == sp_o.stats.gate_opens
+    assert st["gate_checks"] == sp_o.stats.gate_checks
+
+
 # ---------------------------------------------------------------------------
 # shapes the tiny model does not reach
 # ---------------------------------------------------------------------------

@@ -20,13 +20,13 @@ SMALL_BF16_96 = syn.ModelConfig("bf16_hd96", "bf16", 192, 2, 96, 384, 700, 1, 2,
                                 resid_scale=0.5, head_gain=4.0, seed=8)
 
 
-def _run(cfg, dec, w, prompt, use_pass, max_branches, n):
+def _run(cfg, dec, w, prompt, use_pass, max_branches, n, max_ctx=None):
     from looped_transformer_self_b200.binding import Decoder
     old = os.environ.get("LT_PASS")
     os.environ["LT_PASS"] = "1" if use_pass else "0"
     try:
-        g = Decoder(cfg, dec, w, max_branches=max_branches, max_ctx=len(prompt) + n + 16,
-                    trace_steps=8 * n)
+        g = Decoder(cfg, dec, w, max_branches=max_branches,
+                    max_ctx=max_ctx or len(prompt) + n + 16, trace_steps=8 * n)
     finally:
         if old is None:
             del os.environ["LT_PASS"]
@@ -65,3 +65,19 @@ def test_pass_kernel_sampled_matches_multi_kernel():
     a = _run(cfg, dec, w, prompt, True, 16, n)
     b = _run(cfg, dec, w, prompt, False, 16, n)
     assert a[0] == b[0] and a[1] == b[1] and a[2] == b[2]
+
+
+def test_pass_kernel_matches_register_attention_path():
+    """Caches sized beyond the ring-buffered attention's limit send the
+    multi-kernel pass to the register attention kernel; the pass kernel runs
+    the same attention item, so the bits still agree."""
+    cfg = SMALL_BF16_128
+    n = 24
+    dec = syn.DecodeConfig(1, 2, 0.0, 1.0, 3, n)
+    w = syn.make_weights(cfg)
+    prompt = syn.uniform_prompt(120, cfg.vocab, seed=13)
+    a = _run(cfg, dec, w, prompt, True, 16, n, max_ctx=4096)
+    b = _run(cfg, dec, w, prompt, False, 16, n, max_ctx=4096)
+    assert a[0] == b[0] and a[1] == b[1] and a[2] == b[2]
+    for x, y in zip(a[3], b[3]):
+        np.testing.assert_array_equal(np.asarray(x), np.asarray(y))
