@@ -227,6 +227,25 @@ const char* lt_last_error(const lt_handle* h);
 void lt_destroy(lt_handle* h);
 
 /*
+ * Total variation between two readouts of the same positions (depth
+ * selection, LoopSpec page, section 2.4, Eq. 7 and section 3.1, Fig. 3:
+ * E_X[TV(p_r, p_R)] over positions, fitted by a power law, sets d1 and d2
+ * through Eq. 8).  Row i of each input holds raw readout logits (e.g. the
+ * d_logits of lt_prefill at depths r and R); both rows get the readout
+ * processing of a decode step (temperature T, top-p, normalisation; section
+ * 2.1) and d_tv[i] = 1/2 sum_j |p_a(j) - p_b(j)|.  T = 0: one-hot argmax
+ * readouts, so d_tv[i] = 1 where the argmaxes differ, else 0.
+ *   d_za, d_zb  device fp32, row i at d_za + i * stride_a (elements), V entries;
+ *               OVERWRITTEN with the processed distributions when T > 0;
+ *               the two inputs must not overlap.
+ *   d_tv        device fp32 [n].
+ * Asynchronous on `stream`.  Errors: LT_ERR_ARG (null pointer with n > 0,
+ * V <= 0, T < 0, top_p <= 0, a stride below V), LT_ERR_CUDA (launch).
+ */
+int lt_readout_tv(float* d_za, long long stride_a, float* d_zb, long long stride_b, int n, int V,
+                  float T, float top_p, float* d_tv, void* stream);
+
+/*
  * Stand-alone weight-streaming GEMM of the shared block (tcgen05 + TMEM + TMA):
  *   d_y[i][n] = sum_k d_x[i][k] * d_w[n][k],  i < ncols, n < n_out.
  * This is the contraction every shared-block layer runs once per decode step

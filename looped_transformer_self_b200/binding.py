@@ -93,6 +93,8 @@ def _declare(L):
     L.lt_gemm_scratch_bytes.argtypes = [_i, _i, _i, _i, ctypes.POINTER(_sz)]
     L.lt_gemm_rows.argtypes = [_i, _vp, _vp, _vp, _i, _i, _i, _vp, _sz, _vp]
     L.lt_gemm_rows_noalloc.argtypes = [_i, _vp, _vp, _vp, _i, _i, _i, _vp]
+    L.lt_readout_tv.argtypes = [_vp, ctypes.c_longlong, _vp, ctypes.c_longlong, _i, _i,
+                                ctypes.c_float, ctypes.c_float, _vp, _vp]
     L.lt_workspace_bytes.argtypes = [ctypes.POINTER(ModelConfigC), ctypes.POINTER(DecodeConfigC),
                                      ctypes.POINTER(_sz)]
     L.lt_create.argtypes = [ctypes.POINTER(ModelConfigC), ctypes.POINTER(DecodeConfigC), _vp, _sz,
@@ -161,6 +163,23 @@ def gemm_rows_noalloc(w: torch.Tensor, x: torch.Tensor, stream=None) -> torch.Te
     check(lib().lt_gemm_rows_noalloc(LT_BF16, _ptr(w), _ptr(x), _ptr(y), n_out, k, ncols,
                                      _stream(stream)), "lt_gemm_rows_noalloc")
     return y
+
+
+def readout_tv(za: torch.Tensor, zb: torch.Tensor, temperature: float, top_p: float,
+               stream=None) -> torch.Tensor:
+    """Per-row total variation between the readout distributions of two fp32
+    logit matrices [n][V] (row stride free, unit column stride) through
+    lt_readout_tv.  With temperature > 0 both inputs are overwritten with the
+    processed distributions."""
+    assert za.is_cuda and zb.is_cuda and za.dtype == zb.dtype == torch.float32
+    assert za.dim() == zb.dim() == 2 and za.shape == zb.shape
+    assert za.stride(1) == 1 and zb.stride(1) == 1
+    n, V = za.shape
+    tv = torch.empty(n, dtype=torch.float32, device=za.device)
+    check(lib().lt_readout_tv(_ptr(za), za.stride(0), _ptr(zb), zb.stride(0), n, V,
+                              float(temperature), float(top_p), _ptr(tv), _stream(stream)),
+          "lt_readout_tv")
+    return tv
 
 
 # ---------------------------------------------------------------------------

@@ -23,6 +23,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "readout.cuh"
 
 namespace lt {
 
@@ -69,52 +70,8 @@ struct Dev {
 };
 
 // ---------------------------------------------------------------------------
-// block helpers
+// block helpers (arg-min / arg-max, suffix scan and readout processing: readout.cuh)
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ bool better_min(float k, int i, float bk, int bi) {
-  return k < bk || (k == bk && i < bi);
-}
-__device__ __forceinline__ bool better_max(float k, int i, float bk, int bi) {
-  return k > bk || (k == bk && i < bi);
-}
-
-// Block-wide arg-min (MIN=true) or arg-max of (key, index), lowest index on ties.
-template <bool MIN>
-__device__ __forceinline__ int block_arg(float k, int idx, float* sk, int* si) {
-  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    const float k2 = __shfl_xor_sync(0xffffffffu, k, o);
-    const int i2 = __shfl_xor_sync(0xffffffffu, idx, o);
-    if (MIN ? better_min(k2, i2, k, idx) : better_max(k2, i2, k, idx)) {
-      k = k2;
-      idx = i2;
-    }
-  }
-  __syncthreads();
-  if (lane == 0) {
-    sk[w] = k;
-    si[w] = idx;
-  }
-  __syncthreads();
-  if (w == 0) {
-    k = lane < nw ? sk[lane] : (MIN ? INFINITY : -INFINITY);
-    idx = lane < nw ? si[lane] : 0x7fffffff;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float k2 = __shfl_xor_sync(0xffffffffu, k, o);
-      const int i2 = __shfl_xor_sync(0xffffffffu, idx, o);
-      if (MIN ? better_min(k2, i2, k, idx) : better_max(k2, i2, k, idx)) {
-        k = k2;
-        idx = i2;
-      }
-    }
-    if (lane == 0) si[32] = idx;
-  }
-  __syncthreads();
-  return si[32];
-}
-
 // Exponential race over weights w[0..V) (w_j <= 0 never chosen).
 __device__ __forceinline__ int block_race(const float* __restrict__ w, int V,
                                           unsigned long long seed, uint32_t stream,
@@ -134,32 +91,6 @@ __device__ __forceinline__ int block_race(const float* __restrict__ w, int V,
   return block_arg<true>(best, bi, sk, si);
 }
 
-// Inclusive suffix sums of 1024 u64 bins held one per thread (blockDim 1024).
-__device__ __forceinline__ unsigned long long suffix_scan_1024(unsigned long long v,
-                                                              unsigned long long* wsum) {
-  // prefix scan over reversed order: thread t holds bin 1023 - t
-  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const unsigned long long t = __shfl_up_sync(0xffffffffu, v, o);
-    if (lane >= o) v += t;
-  }
-  __syncthreads();
-  if (lane == 31) wsum[w] = v;
-  __syncthreads();
-  if (w == 0) {
-    unsigned long long s = wsum[lane];
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const unsigned long long t = __shfl_up_sync(0xffffffffu, s, o);
-      if (lane >= o) s += t;
-    }
-    wsum[lane] = s;
-  }
-  __syncthreads();
-  return v + (w > 0 ? wsum[w - 1] : 0ull);
-}
-
 // ---------------------------------------------------------------------------
 // K4: readout processing of LM-head partials (one block of 1024 per readout row)
 // ---------------------------------------------------------------------------
@@ -170,11 +101,7 @@ __global__ void __launch_bounds__(1024)
               const float* __restrict__ ssq, int ssq_tiles, int d, float eps) {
   __shared__ float sk[33];
   __shared__ int si[33];
-  __shared__ float red[33];
-  __shared__ unsigned long long hist[1024];
-  __shared__ unsigned long long wsum[32];
-  __shared__ int sel[2];
-  __shared__ unsigned long long sel_above[1];
+  __shared__ DistSmem ds;
   pdl_wait();
   pdl_trigger();
   const int i = blockIdx.x;
@@ -207,73 +134,7 @@ __global__ void __launch_bounds__(1024)
   const int a = block_arg<false>(best, bi, sk, si);
   if (threadIdx.x == 0) arg[i] = a;
   if (greedy) return;
-  // softmax(z / T)
-  const float zmax = z[a];  // same thread may not have written it: reread after the barrier
-  const float invT = 1.f / T;
-  float ssum = 0.f;
-  for (int j = threadIdx.x; j < V; j += blockDim.x) {
-    const float e = expf((z[j] - zmax) * invT);
-    p[j] = e;
-    ssum += e;
-  }
-  const float Z = block_sum(ssum, red);
-  const float invZ = 1.f / Z;
-  if (!(top_p < 1.f)) {
-    for (int j = threadIdx.x; j < V; j += blockDim.x) p[j] *= invZ;
-    return;
-  }
-  // exact top-p threshold: 3-level radix select over the float bits of p with
-  // integer (2^-40) mass, so the sums do not depend on thread order
-  const double SCALE = 1099511627776.0;  // 2^40
-  const unsigned long long target = (unsigned long long)((double)top_p * SCALE + 0.5);
-  unsigned long long above = 0ull;
-  uint32_t prefix = 0u;
-  const int shifts[3] = {20, 10, 0};
-  bool all = false;
-  for (int lvl = 0; lvl < 3; ++lvl) {
-    hist[threadIdx.x] = 0ull;
-    __syncthreads();
-    const int sh = shifts[lvl];
-    for (int j = threadIdx.x; j < V; j += blockDim.x) {
-      const float pj = (lvl == 0) ? p[j] * invZ : p[j];
-      if (lvl == 0) p[j] = pj;
-      const uint32_t b = __float_as_uint(pj);
-      if (lvl == 0 || (b >> (sh + 10)) == prefix) {
-        const unsigned long long m = (unsigned long long)((double)pj * SCALE + 0.5);
-        atomicAdd(&hist[(b >> sh) & 1023u], m);
-      }
-    }
-    __syncthreads();
-    const int bin = 1023 - threadIdx.x;
-    const unsigned long long hv = hist[bin];
-    const unsigned long long cum = suffix_scan_1024(hv, wsum);  // mass of bins >= bin
-    if (threadIdx.x == 0) sel[0] = -1;
-    __syncthreads();
-    if (above + cum >= target && above + cum - hv < target) {
-      sel[0] = bin;
-      sel_above[0] = above + cum - hv;
-    }
-    __syncthreads();
-    if (sel[0] < 0) {
-      all = true;
-      break;
-    }
-    above = sel_above[0];
-    prefix = (prefix << 10) | (uint32_t)sel[0];
-    __syncthreads();
-  }
-  const uint32_t theta = all ? 0u : prefix;
-  float ks = 0.f;
-  for (int j = threadIdx.x; j < V; j += blockDim.x) {
-    const float pj = p[j];
-    if (__float_as_uint(pj) >= theta) ks += pj;
-  }
-  const float Z2 = block_sum(ks, red);
-  const float inv2 = 1.f / Z2;
-  for (int j = threadIdx.x; j < V; j += blockDim.x) {
-    const float pj = p[j];
-    p[j] = __float_as_uint(pj) >= theta ? pj * inv2 : 0.f;
-  }
+  readout_dist(z, p, V, a, T, top_p, ds);
 }
 
 // ---------------------------------------------------------------------------
