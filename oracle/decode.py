@@ -35,6 +35,27 @@ engine bit for bit):
      child becomes the root and its slot is appended to the committed slots;
      with no kept child a new root (depth 0) is created after the frees
      (unless that commit was the last one).
+
+Context-copy proposals (CopyLoop card, kongchang.com; oracle/copy.py has the
+lookup and the readings), when enabled, change steps 4-6 as follows:
+  4a. a branch at depth d1 whose first proposal is a copied token (it has a
+      copy child) is screened: if the token's depth-d1 score is below tau the
+      copy child's subtree is pruned and the branch proposes normally;
+  4b. a branch at depth d1 without a copy child looks up a copy proposal when
+      no copy row outside its own ancestors is alive; if the first copied
+      token passes the screen, x1 is that token (q1 one-hot) and the proposal
+      opens at once as a chain of rows, each the child of the previous one,
+      all at depth 0 -- they advance together, so each attends to its
+      ancestors' cache rows written earlier in the same pass.  The chain is
+      cut to the free table rows beyond a reserve for the ordinary tree, to
+      the uncommitted window and to the token budget.  A branch whose first
+      proposal is copied opens no second proposal;
+  5'. verification repeats while the new root reached R in this step (chain
+      rows reach R together), so one step can commit several tokens; a copied
+      x1 is verified with q1 one-hot: accepted with probability p_R(x1), else
+      the token is drawn from p_R with x1 removed.
+A child is never created at a position that would leave the uncommitted
+window (32 positions past the last committed one).
 """
 from __future__ import annotations
 
@@ -43,7 +64,10 @@ from typing import Any, Dict, List, Optional, Sequence, Tuple
 
 import numpy as np
 
+from . import copy as CP
 from . import sampling as S
+
+WIN = 32  # uncommitted window: a child's position minus the last committed one is < WIN
 
 
 # ----------------------------------------------------------------------------
@@ -86,6 +110,10 @@ class Stats:
     branches_created: int = 0
     resid_fallback: int = 0
     table_peak: int = 0  # most branches alive at once (children exist before the same step's prune)
+    copy_chains: int = 0  # copy proposals opened
+    copy_rows: int = 0  # rows they opened
+    copy_cut: int = 0  # copied rows pruned by the depth-d1 screen
+    n_copy: int = 0  # commits of a copied token
 
     def gamma(self, d1: int, d2: int, R: int) -> float:
         """Mean acceptance length, Eq. 9 (section 3.2)."""
@@ -228,6 +256,20 @@ class Branch:
     # verification -- is never pruned, and leaves the table once it has run
     # all R iterations.
     retiring: bool = False
+    z: Optional[np.ndarray] = None  # this step's readout logits (copy screening)
+    copy_row: bool = False  # its token was copied from the context
+    copy_child: bool = False  # x1 is a copied token and child1 the next copy row
+
+
+@dataclasses.dataclass
+class CopyConfig:
+    """Context-copy proposals (readings in oracle/copy.py)."""
+    tau: float
+    k: int = 4
+    max_len: int = 16
+    match_cap: int = 64
+    table: int = 64  # branch-table capacity the chain must fit in
+    reserve: int = 8  # rows kept free for the ordinary tree
 
 
 class SpecDecoder:
@@ -238,8 +280,10 @@ class SpecDecoder:
     def __init__(self, rows, prompt: Sequence[int], R: int, d1: int, d2: int, max_new: int,
                  temperature: float, top_p: float, seed: int, n_slots: int,
                  second: str = "gated", keep_trace: bool = True, keep_logits: bool = False,
-                 skip_prefill: bool = False, first: Optional[int] = None):
+                 skip_prefill: bool = False, first: Optional[int] = None,
+                 copy: Optional[CopyConfig] = None):
         assert 1 <= d1 < R and (d2 == 0 or d1 < d2 < R)
+        self.copy = copy
         self.rows, self.R, self.d1, self.d2 = rows, R, d1, d2
         self.T, self.top_p, self.seed = temperature, top_p, seed
         self.second = second
@@ -339,6 +383,7 @@ class SpecDecoder:
                 margin = min(margin, top2_margin(z))
                 gap = min(gap, top2_gap(z))
                 b.p = S.process(z, self.T, self.top_p)
+                b.z = z
         self.step_margin.append(margin)
         self.step_gap.append(gap)
         # retiring rows that ran their last iteration leave (their slots hold
@@ -347,17 +392,29 @@ class SpecDecoder:
             if self.branches[u].retiring and self.branches[u].depth >= self.R:
                 del self.branches[u]
         # 4. proposals
+        L = len(self.committed)
         for u in order:
             b = self.branches.get(u)
             if b is None or b.retiring:
                 continue
-            spawn = b.pos + 1 < self.pos_limit  # is a child at pos+1 still needed?
+            # is a child at pos+1 still needed, and inside the uncommitted window?
+            spawn = b.pos + 1 < self.pos_limit and b.pos + 1 - (L - 1) < WIN
             if b.depth == self.d1:
+                if b.copy_child:
+                    if CP.screen_score(b.z, b.x1) >= self.copy.tau:
+                        continue  # the copied token goes on
+                    st.copy_cut += len(self._subtree(b.child1))
+                    for v in self._subtree(b.child1):
+                        self.free.add(self.branches.pop(v).slot)
+                    b.child1, b.copy_child = -1, False
                 b.q1 = b.p
                 b.x1 = S.race(b.q1, self.seed, b.uid, S.PROP1)
+                if spawn and self.copy is not None and self._copy_allowed(b):
+                    if self._open_copy(b, L):
+                        continue
                 if spawn:
                     b.child1 = self._new_branch(b.uid, b.pos + 1, b.x1, b.chain).uid
-            elif self.d2 and b.depth == self.d2 and b.x1 >= 0:
+            elif self.d2 and b.depth == self.d2 and b.x1 >= 0 and not b.copy_child:
                 st.gate_checks += 1
                 if self.second == "gated":
                     b.gate = S.gate_open(b.p, b.q1, b.x1)
@@ -373,11 +430,56 @@ class SpecDecoder:
                     b.x2 = S.race(q2, self.seed, b.uid, S.PROP2)
                     if spawn:
                         b.child2 = self._new_branch(b.uid, b.pos + 1, b.x2, b.chain).uid
-        # 5. verify at full depth
-        root = self.root()
-        if root.depth < self.R:
-            return
-        x, src, fb = S.verify(root.p, root.x1, root.q1, root.gate, root.x2, root.q2,
+        # 5-6. verify at full depth, commit, prune / reroot; repeated while the
+        # new root also reached R in this step (copied chains)
+        while not self.done():
+            root = self.root()
+            if root.depth < self.R:
+                return
+            self._verify_commit(root)
+
+    def _copy_allowed(self, b: Branch) -> bool:
+        """No copy row alive outside b's own ancestors (b included)."""
+        for x in self.branches.values():
+            if x.copy_row and not x.retiring and x.uid != b.uid and b.uid not in self._subtree(x.uid):
+                return False
+        return True
+
+    def _open_copy(self, b: Branch, L: int) -> bool:
+        """Copy proposal for b (at depth d1, x1 already drawn): screen its first
+        token and open the chain.  Returns whether a chain was opened."""
+        cp = self.copy
+        seq = self.prefix_of(b)
+        _, _, prop = CP.lookup(seq, L, cp.k, cp.max_len, cp.match_cap)
+        if not prop or CP.screen_score(b.z, prop[0]) < cp.tau:
+            return False
+        m = min(len(prop),
+                cp.table - len(self.branches) - cp.reserve,  # free table rows beyond the reserve
+                # window: the last copied row at b.pos + m stays WIN - 2 - ceil(R / d1)
+                # or less past the last committed position (room for the tail's children)
+                WIN - 2 - (b.pos - (L - 1)) - -(-self.R // self.d1),
+                self.pos_limit - 1 - b.pos)  # token budget
+        if m < 1:
+            return False
+        self.stats.copy_chains += 1
+        self.stats.copy_rows += m
+        b.x1, b.q1, b.copy_child = prop[0], S.one_hot(prop[0], len(b.p)), True
+        parent = b
+        for j in range(m):
+            c = self._new_branch(parent.uid, parent.pos + 1, prop[j], parent.chain)
+            c.copy_row = True
+            if parent is b:
+                b.child1 = c.uid
+            else:
+                parent.x1, parent.copy_child, parent.child1 = prop[j], True, c.uid
+                parent.q1 = None  # set to one-hot once the row has a readout width
+            parent = c
+        return True
+
+    def _verify_commit(self, root: Branch) -> None:
+        st = self.stats
+        q1 = S.one_hot(root.x1, len(root.p)) if root.copy_child else root.q1
+        x, src, fb = S.verify(root.p, root.x1, q1, root.gate, root.x2, root.q2,
                               self.seed, root.uid)
         st.resid_fallback += fb
         self.committed.append(x)
@@ -385,20 +487,13 @@ class SpecDecoder:
         self.cstep.append(st.steps)
         if src == S.SRC_FIRST:
             st.n_first += 1
+            st.n_copy += int(root.copy_child)
         elif src == S.SRC_SECOND:
             st.n_second += 1
         else:
             st.n_fallback += 1
-        # 6. prune / reroot
         keep_uid = root.child1 if src == S.SRC_FIRST else root.child2 if src == S.SRC_SECOND else -1
-        keep = set()
-        if keep_uid >= 0:
-            for u in sorted(self.branches):
-                x_ = self.branches[u]
-                while x_ is not None and x_.uid != keep_uid:
-                    x_ = self.branches.get(x_.parent)
-                if x_ is not None:
-                    keep.add(u)
+        keep = set(self._subtree(keep_uid)) if keep_uid >= 0 else set()
         for u in sorted(self.branches):
             if u in keep or self.branches[u].retiring:
                 continue

@@ -126,6 +126,13 @@ def residual(mu: np.ndarray, nu: np.ndarray) -> Optional[np.ndarray]:
     return pos / z
 
 
+def one_hot(x: int, V: int) -> np.ndarray:
+    """The proposal distribution of a token that was not drawn (a copied token)."""
+    q = np.zeros(V, dtype=np.float64)
+    q[x] = 1.0
+    return q
+
+
 def gate_open(p_d2: np.ndarray, q1: np.ndarray, x1: int) -> bool:
     """Eq. 6: open iff the deeper readout lowers the first candidate's probability."""
     return bool(p_d2[x1] < q1[x1])
