@@ -71,6 +71,19 @@ typedef struct {
   int second_mode;     /* 0: gated residual (the method); 1: residual, no gate;
                           2: p_d2 with x1 masked, no gate (ablations, section 3.4) */
   int trace_steps;     /* steps whose branch rows are logged (0: none) */
+  /* Context-copy proposals (CopyLoop card, kongchang.com: copied continuations
+   * screened at a shallow depth before the full-depth verify).  copy_k = 0
+   * disables them.  A branch at depth d1 whose prefix ends with the longest
+   * earlier match (>= copy_k tokens, backward match capped at copy_match_cap)
+   * of the committed context proposes the committed tokens that followed it
+   * (<= copy_max_len <= 32) as a chain of rows opened together; a copied token
+   * goes on only while its depth-d1 softmax probability (T = 1) is >= copy_tau;
+   * copy_reserve table rows stay free for the ordinary tree.  Copied tokens are
+   * verified with a one-hot proposal (accepted with probability p_R(x), else a
+   * draw from p_R without x), and a step commits every chain row that reached
+   * R and was accepted in order. */
+  int copy_k, copy_max_len, copy_match_cap, copy_reserve;
+  float copy_tau;
 } lt_decode_config;
 
 /* Per-generate statistics (section 3.2 Eq. 9 counts, Fig. 5, Table 6, Fig. 6). */
@@ -82,6 +95,9 @@ typedef struct {
   int branches_created;
   int resid_fallback;   /* residuals with zero mass (expected 0) */
   int committed_len;    /* committed length after the call */
+  int copy_chains, copy_rows;  /* copy proposals opened, rows they opened */
+  int copy_cut;         /* copied rows removed by the depth-d1 screen */
+  int n_copy;           /* committed tokens that were copied (included in n_first) */
 } lt_stats;
 
 typedef struct lt_handle lt_handle;
@@ -129,8 +145,8 @@ int lt_prefill(lt_handle* h, const int32_t* h_tokens, int n, int32_t* h_first,
  * Greedy speculative output equals greedy AR output bit for bit.
  */
 int lt_generate(lt_handle* h, int ar_mode, int n, int32_t* h_out, lt_stats* st);
-/* One batched pass.  *n_committed = 1 and *h_tok = the token when this pass
- * committed one, else 0. */
+/* One batched pass.  *n_committed = the tokens this pass committed (0 or 1;
+ * with copy proposals several) and *h_tok = the last of them. */
 int lt_decode_step(lt_handle* h, int ar_mode, int32_t* h_tok, int* n_committed);
 /*
  * Explicit edits of the branch tree between two decode steps (after

@@ -6,6 +6,7 @@ the shared library is missing, the import fails loudly.
 from __future__ import annotations
 
 import ctypes
+import dataclasses
 import os
 
 import torch
@@ -51,13 +52,16 @@ class ModelConfigC(ctypes.Structure):
 class DecodeConfigC(ctypes.Structure):
     _fields_ = [("d1", _i), ("d2", _i), ("temperature", ctypes.c_float),
                 ("top_p", ctypes.c_float), ("seed", ctypes.c_uint64), ("max_branches", _i),
-                ("max_ctx", _i), ("max_new", _i), ("second_mode", _i), ("trace_steps", _i)]
+                ("max_ctx", _i), ("max_new", _i), ("second_mode", _i), ("trace_steps", _i),
+                ("copy_k", _i), ("copy_max_len", _i), ("copy_match_cap", _i),
+                ("copy_reserve", _i), ("copy_tau", ctypes.c_float)]
 
 
 class StatsC(ctypes.Structure):
     _fields_ = [(n, _i) for n in ("steps", "rows_sum", "rows_max", "n_first", "n_second",
                                    "n_fallback", "gate_checks", "gate_opens", "branches_created",
-                                   "resid_fallback", "committed_len")]
+                                   "resid_fallback", "committed_len", "copy_chains",
+                                   "copy_rows", "copy_cut", "n_copy")]
 
     def as_dict(self):
         return {n: getattr(self, n) for n, _ in self._fields_}
@@ -196,24 +200,37 @@ def model_config_c(cfg) -> ModelConfigC:
                         cfg.R, cfg.rms_eps, cfg.rope_theta, cfg.resid_scale)
 
 
+@dataclasses.dataclass
+class CopyConfig:
+    """Context-copy proposals of lt_decode_config (k = 0: off)."""
+    tau: float
+    k: int = 4
+    max_len: int = 16
+    match_cap: int = 64
+    reserve: int = 8
+
+
 class Decoder:
     """One lt_handle: caller-side device memory (weights, workspace) and a
     non-default CUDA stream, owned by this object."""
 
     def __init__(self, cfg, dec, weights=None, max_branches=16, max_ctx=None, trace_steps=0,
-                 second_mode=0, device="cuda", workspace_fill=None):
+                 second_mode=0, device="cuda", workspace_fill=None, copy=None):
         """workspace_fill: a byte value written over the whole workspace before
         lt_create (tests use it to show that no state is read before it is
-        written); None leaves the allocation as it comes."""
+        written); None leaves the allocation as it comes.  copy: context-copy
+        proposals, a CopyConfig (None: off)."""
         import numpy as np
         self.np = np
         self.cfg, self.dec = cfg, dec
         self.device = torch.device(device)
         self.stream = torch.cuda.Stream(device=self.device)
         self.mc = model_config_c(cfg)
+        cp = copy or CopyConfig(tau=0.0, k=0)
         self.dc = DecodeConfigC(dec.d1, dec.d2, dec.temperature, dec.top_p, dec.seed,
                                 max_branches, max_ctx or 4096, dec.max_new, second_mode,
-                                trace_steps)
+                                trace_steps, cp.k, cp.max_len, cp.match_cap, cp.reserve,
+                                cp.tau)
         need = _sz()
         check(lib().lt_workspace_bytes(ctypes.byref(self.mc), ctypes.byref(self.dc),
                                        ctypes.byref(need)), "lt_workspace_bytes")

@@ -23,6 +23,8 @@
 #pragma once
 
 #include "common.cuh"
+#include <climits>
+
 #include "readout.cuh"
 
 namespace lt {
@@ -30,6 +32,7 @@ namespace lt {
 constexpr int CMAX = 64;        // branch-table capacity limit (= max GEMM columns)
 constexpr int WIN = 32;         // chain window: uncommitted positions a branch may span
 constexpr int MAX_SLOT_WORDS = 2048;  // slot bitmap words held in shared memory (65536 slots)
+constexpr int CPMAX = 32;       // longest copy proposal
 
 struct Ctl {
   int L;              // committed length (prompt + generated)
@@ -47,6 +50,7 @@ struct Ctl {
   // statistics (Eq. 9's counts, Fig. 5 rows, Table 6 gate rate)
   int steps, rows_sum, rows_max, n_first, n_second, n_fallback;
   int gate_checks, gate_opens, branches_created, resid_fallback;
+  int copy_chains, copy_rows, copy_cut, n_copy;
 };
 
 struct Dev {
@@ -54,10 +58,18 @@ struct Dev {
   float T, top_p;
   unsigned long long seed;
   int tag_of_depth[33];
+  // context-copy proposals (copy_k = 0: off)
+  int copy_k, copy_max, copy_cap, copy_reserve, copy_slack;
+  float copy_tau;
   Ctl* ctl;
   // branch table
   int *b_alive, *b_uid, *b_parent, *b_slot, *b_pos, *b_tok, *b_depth, *b_x1, *b_x2, *b_gate,
       *b_c1, *b_c2, *b_chain;
+  int *b_copy;   // x1 is a copied token and child1 the next copied row
+  int *b_crow;   // the entry's token was copied
+  // written by k_decide for k_book: screen failures, copy proposals, verify outcomes
+  int *cp_fail, *cp_len, *cp_tok;  // cp_tok [C][CPMAX]
+  int *v_tok, *v_src, *v_fb;
   // rows of the prepared pass
   int *r_tok, *r_pos, *r_slot, *r_depth, *r_ro, *r_blen, *r_boff, *m_alive, *m_new, *m_ro;
   int* lists;      // committed slots
@@ -168,10 +180,77 @@ __device__ __forceinline__ float residual_into(const float* __restrict__ mu,
 // committed position) after its R-th iteration.
 constexpr int BK_RETIRING = -2;
 
+// Block-wide maximum of an int (every thread gets it).
+__device__ __forceinline__ int block_max_int(int v, int* si) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  v = __reduce_max_sync(0xffffffffu, v);
+  __syncthreads();
+  if (lane == 0) si[w] = v;
+  __syncthreads();
+  if (w == 0) {
+    int t = lane < nw ? si[lane] : INT_MIN;
+    t = __reduce_max_sync(0xffffffffu, t);
+    if (lane == 0) si[32] = t;
+  }
+  __syncthreads();
+  return si[32];
+}
+
+// Screen score of token s (CopyLoop card: copied tokens are scored at a
+// shallow depth): softmax of the row's logits z at T = 1, taken at s.
+// a: the row's argmax.
+__device__ __forceinline__ float copy_score(const float* __restrict__ z, int V, int a, int s,
+                                            float* red) {
+  const float zmax = z[a];
+  float acc = 0.f;
+  for (int j = threadIdx.x; j < V; j += blockDim.x) acc += expf(z[j] - zmax);
+  const float Z = block_sum(acc, red);
+  return expf(z[s] - zmax) / Z;
+}
+
+// Copy proposal of entry i (position pos, L committed tokens): the end e of
+// the earlier committed occurrence whose backward match with the prefix's end
+// is longest (>= copy_k, capped at copy_cap; the most recent on ties), and
+// the committed tokens after it (<= copy_max).  Returns the proposal's length
+// (0: none) with its tokens in out[].  tail[]: shared memory, WIN entries.
+__device__ int copy_lookup(const Dev& D, int i, int L, int* tail, int* si, int* out) {
+  const int pos = D.b_pos[i];
+  if (threadIdx.x == 0) {  // the prefix's uncommitted tokens, from the entry up its ancestors
+    int cur = i;
+    for (int guard = 0; cur >= 0 && D.b_pos[cur] >= L && guard <= WIN; ++guard) {
+      tail[D.b_pos[cur] - L] = D.b_tok[cur];
+      const int pu = D.b_parent[cur];
+      int nx = -1;
+      if (pu >= 0)
+        for (int k = 0; k < D.C; ++k)
+          if (D.b_alive[k] && D.b_uid[k] == pu) nx = k;
+      cur = nx;
+    }
+  }
+  __syncthreads();
+  const int* cm = D.committed;
+  auto seq = [&](int t) { return t < L ? cm[t] : tail[t - L]; };
+  int best = -1;  // m * 65536 + e (e < 65536: at most 65536 slots)
+  for (int e = D.copy_k - 1 + (int)threadIdx.x; e <= L - 2; e += blockDim.x) {
+    int m = 0;
+    while (m < D.copy_cap && m <= e && seq(e - m) == seq(pos - m)) ++m;
+    if (m >= D.copy_k) best = max(best, m * 65536 + e);
+  }
+  best = block_max_int(best, si);
+  if (best < 0) return 0;
+  const int e = best & 0xffff;
+  const int n = min(D.copy_max, L - 1 - e);
+  for (int t = threadIdx.x; t < n; t += blockDim.x) out[t] = cm[e + 1 + t];
+  __syncthreads();
+  return n;
+}
+
 __global__ void __launch_bounds__(1024) k_decide(Dev D) {
   __shared__ float sk[33];
   __shared__ int si[33];
   __shared__ float red[33];
+  __shared__ int tail[WIN];
+  __shared__ int prop[CPMAX];
   pdl_wait();
   pdl_trigger();
   Ctl* c = D.ctl;
@@ -183,16 +262,27 @@ __global__ void __launch_bounds__(1024) k_decide(Dev D) {
   const bool ar = c->ar_mode != 0;
   const int V = D.V;
   const bool t0 = threadIdx.x == 0;
+  const bool copied_x1 = !ar && D.b_copy[i];  // x1 is a copied token (child1 exists)
   const bool prop1 = !ar && r == D.d1;
-  const bool prop2 = !ar && D.d2 > 0 && r == D.d2 && D.b_x1[i] >= 0;
-  if (r == D.R && D.r_pos[i] != c->L - 1) {
-    if (t0) set_err(&c->err, DEV_STATE);
-    return;
+  const bool prop2 = !ar && D.d2 > 0 && r == D.d2 && D.b_x1[i] >= 0 && !copied_x1;
+  const float* z = D.logits + (size_t)i * V;
+  const int a = D.ro_arg[i];
+  // at depth d1: screen a copied x1, or propose (and look up a copy proposal)
+  bool draw1 = prop1;
+  if (prop1 && copied_x1) {
+    const bool pass = copy_score(z, V, a, D.b_x1[i], red) >= D.copy_tau;
+    if (t0) D.cp_fail[i] = !pass;
+    draw1 = !pass;
+  }
+  if (prop1 && !copied_x1 && D.copy_k > 0) {
+    int n = copy_lookup(D, i, c->L, tail, si, prop);
+    if (n > 0 && copy_score(z, V, a, prop[0], red) < D.copy_tau) n = 0;
+    if (t0) D.cp_len[i] = n;
+    for (int t = threadIdx.x; t < n; t += blockDim.x) D.cp_tok[(size_t)i * CPMAX + t] = prop[t];
   }
   if (D.greedy) {
     if (!t0) return;
-    const int a = D.ro_arg[i];
-    if (prop1) D.b_x1[i] = a;
+    if (draw1) D.b_x1[i] = a;
     if (prop2) {
       const int g = a != D.b_x1[i];
       D.b_gate[i] = g;
@@ -206,16 +296,16 @@ __global__ void __launch_bounds__(1024) k_decide(Dev D) {
         if (D.b_x1[i] >= 0 && a == D.b_x1[i]) src = 1;
         else if (D.b_gate[i] && a == D.b_x2[i]) src = 2;
       }
-      c->commit_tok = a;
-      c->commit_src = src;
-      c->commit_pending = 1;
+      D.v_tok[i] = a;
+      D.v_src[i] = src;
+      D.v_fb[i] = 0;
     }
     return;
   }
   const float* p = D.P + (size_t)i * V;
   float* q1 = D.q1 + (size_t)i * V;
   float* q2 = D.q2 + (size_t)i * V;
-  if (prop1) {
+  if (draw1) {
     for (int j = threadIdx.x; j < V; j += blockDim.x) q1[j] = p[j];
     const int x1 = block_race(p, V, D.seed, (uint32_t)uid, P_PROP1, sk, si);
     if (t0) D.b_x1[i] = x1;
@@ -251,12 +341,41 @@ __global__ void __launch_bounds__(1024) k_decide(Dev D) {
     }
   }
   if (r != D.R) return;
-  // verification at full depth
+  // verification at full depth (every row at R: a copied chain reaches R
+  // together; the bookkeeping applies the outcomes in chain order)
   int x, src = 0, fb = 0;
+  float* rho_i = D.rho + (size_t)i * V;
+  float* rho2_i = D.rho2 + (size_t)i * V;
   if (ar) {
     x = block_race(p, V, D.seed, (uint32_t)(D.r_pos[i] + 1), P_AR, sk, si);
   } else if (D.b_x1[i] < 0) {
     x = block_race(p, V, D.seed, (uint32_t)uid, P_RES, sk, si);
+  } else if (copied_x1) {
+    // one-hot proposal: accept with probability p(x1), else draw from p without x1
+    const int x1 = D.b_x1[i];
+    const float u1 = uniform01(D.seed, (uint32_t)uid, P_ACC1);
+    if (u1 < p[x1]) {
+      x = x1;
+      src = 1;
+    } else {
+      float zs = 0.f;
+      for (int j = threadIdx.x; j < V; j += blockDim.x) {
+        const float w = j == x1 ? 0.f : p[j];
+        rho_i[j] = w;
+        zs += w;
+      }
+      const float Z = block_sum(zs, red);
+      const float* rho1 = rho_i;
+      if (Z > 0.f) {
+        const float inv = 1.f / Z;
+        for (int j = threadIdx.x; j < V; j += blockDim.x) rho_i[j] *= inv;
+      } else {
+        rho1 = p;  // unreachable: p(x1) = 1 always accepts
+        fb = 1;
+      }
+      __syncthreads();
+      x = block_race(rho1, V, D.seed, (uint32_t)uid, P_RES, sk, si);
+    }
   } else {
     const int x1 = D.b_x1[i];
     const float u1 = uniform01(D.seed, (uint32_t)uid, P_ACC1);
@@ -264,8 +383,8 @@ __global__ void __launch_bounds__(1024) k_decide(Dev D) {
       x = x1;
       src = 1;
     } else {
-      const float* rho1 = D.rho;
-      if (!(residual_into(p, q1, V, D.rho, red) > 0.f)) {
+      const float* rho1 = rho_i;
+      if (!(residual_into(p, q1, V, rho_i, red) > 0.f)) {
         rho1 = p;  // unreachable in exact arithmetic
         fb = 1;
       }
@@ -276,8 +395,8 @@ __global__ void __launch_bounds__(1024) k_decide(Dev D) {
           x = x2;
           src = 2;
         } else {
-          const float* r2 = D.rho2;
-          if (!(residual_into(rho1, q2, V, D.rho2, red) > 0.f)) {
+          const float* r2 = rho2_i;
+          if (!(residual_into(rho1, q2, V, rho2_i, red) > 0.f)) {
             r2 = rho1;
             fb += 1;
           }
@@ -289,10 +408,9 @@ __global__ void __launch_bounds__(1024) k_decide(Dev D) {
     }
   }
   if (t0) {
-    c->commit_tok = x;
-    c->commit_src = src;
-    c->commit_pending = 1;
-    if (fb) atomicAdd(&c->resid_fallback, fb);
+    D.v_tok[i] = x;
+    D.v_src[i] = src;
+    D.v_fb[i] = fb;
   }
 }
 
@@ -320,7 +438,7 @@ __global__ void __launch_bounds__(1024) k_first_token(Dev D, int row, int P_len)
 // ---------------------------------------------------------------------------
 struct BookSmem {
   int alive[CMAX], uid[CMAX], parent[CMAX], slot[CMAX], pos[CMAX], tok[CMAX], depth[CMAX],
-      x1[CMAX], x2[CMAX], gate[CMAX], c1[CMAX], c2[CMAX];
+      x1[CMAX], x2[CMAX], gate[CMAX], c1[CMAX], c2[CMAX], copy[CMAX], crow[CMAX];
   int chain[CMAX * WIN];
   unsigned int bits[MAX_SLOT_WORDS];
   int order[CMAX];
@@ -371,6 +489,7 @@ __device__ int bk_new_entry(BookSmem& b, const Dev& D, Ctl& c, int parent_e, int
   b.x1[e] = b.x2[e] = -1;
   b.gate[e] = 0;
   b.c1[e] = b.c2[e] = -1;
+  b.copy[e] = b.crow[e] = 0;
   if (parent_e >= 0)
     for (int k = 0; k < WIN; ++k) b.chain[e * WIN + k] = b.chain[parent_e * WIN + k];
   b.chain[e * WIN + (pos % WIN)] = s;
@@ -390,6 +509,59 @@ __device__ int bk_find_uid(const BookSmem& b, int C, int uid) {
 // r's slot at r's position in its chain.
 __device__ __forceinline__ bool bk_in_subtree(const BookSmem& b, int k, int r) {
   return k == r || (b.pos[k] > b.pos[r] && b.chain[k * WIN + (b.pos[r] % WIN)] == b.slot[r]);
+}
+
+// Removes entry r's subtree (r included) and frees its slots; returns the count.
+__device__ int bk_prune_subtree(BookSmem& b, int C, int r) {
+  int n = 0;
+  for (int k = 0; k < C; ++k)
+    if (b.alive[k] && k != r && bk_in_subtree(b, k, r)) {
+      b.alive[k] = 0;
+      bk_free_slot(b, b.slot[k]);
+      ++n;
+    }
+  b.alive[r] = 0;
+  bk_free_slot(b, b.slot[r]);
+  return n + 1;
+}
+
+// Copy proposal of entry e at depth d1 (its x1 already drawn): allowed when no
+// copied entry outside e's own ancestors is alive; cut to the free table rows
+// beyond the reserve, to the uncommitted window (room left for the tail's
+// children) and to the token budget.  Opens the chain: child1 of e and each
+// row the child of the previous one, all at depth 0.  Returns whether it did.
+__device__ bool bk_open_copy(BookSmem& b, const Dev& D, Ctl& c, int e) {
+  const int C = D.C;
+  int n = D.cp_len[e];
+  if (n <= 0) return false;
+  int alive = 0;
+  for (int k = 0; k < C; ++k) {
+    if (!b.alive[k]) continue;
+    ++alive;
+    if (b.crow[k] && b.parent[k] != BK_RETIRING && k != e && !bk_in_subtree(b, e, k)) return false;
+  }
+  n = min(n, C - alive - D.copy_reserve);
+  n = min(n, WIN - 2 - (b.pos[e] - (c.L - 1)) - D.copy_slack);
+  n = min(n, c.pos_limit - 1 - b.pos[e]);
+  if (n < 1) return false;
+  const int* tok = D.cp_tok + (size_t)e * CPMAX;
+  c.copy_chains++;
+  c.copy_rows += n;
+  b.x1[e] = tok[0];
+  b.copy[e] = 1;
+  int par = e;
+  for (int j = 0; j < n; ++j) {
+    const int ch = bk_new_entry(b, D, c, par, b.pos[par] + 1, tok[j], 0, false);
+    if (ch < 0) return true;  // error recorded
+    b.crow[ch] = 1;
+    b.c1[par] = b.uid[ch];
+    if (par != e) {
+      b.x1[par] = tok[j];
+      b.copy[par] = 1;
+    }
+    par = ch;
+  }
+  return true;
 }
 
 __device__ void bk_logic(BookSmem& b, const Dev& D, Ctl& c, int mode, int arg) {
@@ -469,38 +641,58 @@ __device__ void bk_logic(BookSmem& b, const Dev& D, Ctl& c, int mode, int arg) {
     if (!c.ar_mode) {
       for (int a = 0; a < n; ++a) {
         const int e = b.order[a];
-        const bool spawn = b.pos[e] + 1 < c.pos_limit;
-        if (!spawn) continue;
+        if (!b.alive[e] || b.parent[e] == BK_RETIRING) continue;  // pruned by a screen above
+        // a child's position stays inside the token budget and the uncommitted window
+        const bool spawn = b.pos[e] + 1 < c.pos_limit && b.pos[e] + 1 - (c.L - 1) < WIN;
         if (b.depth[e] == D.d1 && b.x1[e] >= 0) {
+          if (b.copy[e]) {
+            if (!D.cp_fail[e]) continue;  // the copied token goes on
+            const int ch = bk_find_uid(b, C, b.c1[e]);
+            if (ch >= 0) c.copy_cut += bk_prune_subtree(b, C, ch);
+            b.copy[e] = 0;
+            b.c1[e] = -1;
+          } else if (spawn && D.copy_k > 0 && bk_open_copy(b, D, c, e)) {
+            if (c.err) return;
+            continue;
+          }
+          if (!spawn) continue;
           const int ch = bk_new_entry(b, D, c, e, b.pos[e] + 1, b.x1[e], 0, false);
           if (ch < 0) return;
           b.c1[e] = b.uid[ch];
-        } else if (D.d2 > 0 && b.depth[e] == D.d2 && b.gate[e] && b.x2[e] >= 0) {
+        } else if (spawn && D.d2 > 0 && b.depth[e] == D.d2 && b.gate[e] && b.x2[e] >= 0) {
           const int ch = bk_new_entry(b, D, c, e, b.pos[e] + 1, b.x2[e], 0, false);
           if (ch < 0) return;
           b.c2[e] = b.uid[ch];
         }
       }
     }
-    if (c.commit_pending) {
-      c.commit_pending = 0;
-      const int x = c.commit_tok, src = c.commit_src;
+    // verification outcomes (k_decide) of the root, repeated while the new
+    // root also ran depth R in this step (a copied chain reaches R together)
+    while (!c.finished) {
       int root = -1;
       for (int k = 0; k < C; ++k)
-        if (b.alive[k] && b.pos[k] == c.L - 1) root = k;
-      if (root < 0 || c.L >= D.max_ctx) {
+        if (b.alive[k] && b.pos[k] == c.L - 1 && b.parent[k] != BK_RETIRING) root = k;
+      if (root < 0 || b.depth[root] != D.R) break;
+      if (c.L >= D.max_ctx) {
         set_err(&c.err, DEV_NO_ROOT);
         return;
       }
+      const int x = D.v_tok[root], src = D.v_src[root];
+      if (D.v_fb[root]) c.resid_fallback += D.v_fb[root];
       D.committed[c.L] = x;
       D.log_tok[c.n_commit] = x;
       D.log_src[c.n_commit] = src;
       D.log_step[c.n_commit] = c.steps;
       c.n_commit++;
       c.L++;
-      if (src == 1) c.n_first++;
-      else if (src == 2) c.n_second++;
-      else c.n_fallback++;
+      if (src == 1) {
+        c.n_first++;
+        c.n_copy += b.copy[root];
+      } else if (src == 2) {
+        c.n_second++;
+      } else {
+        c.n_fallback++;
+      }
       const int surv = bk_find_uid(b, C, src == 1 ? b.c1[root] : src == 2 ? b.c2[root] : -1);
       for (int k = 0; k < C; ++k) {
         if (!b.alive[k] || b.parent[k] == BK_RETIRING) continue;
@@ -521,6 +713,11 @@ __device__ void bk_logic(BookSmem& b, const Dev& D, Ctl& c, int mode, int arg) {
       if (c.L >= c.target_len) c.finished = 1;
     }
     if (c.finished) return;
+    for (int k = 0; k < C; ++k)  // every row that ran depth R has been verified
+      if (b.alive[k] && b.parent[k] != BK_RETIRING && b.depth[k] >= D.R) {
+        set_err(&c.err, DEV_STATE);
+        return;
+      }
     for (int k = 0; k < C; ++k)
       if (b.alive[k]) b.depth[k]++;
     c.prepared = 1;
@@ -562,6 +759,8 @@ __global__ void __launch_bounds__(256) k_book(Dev D, int mode, int arg) {
     b.gate[k] = D.b_gate[k];
     b.c1[k] = D.b_c1[k];
     b.c2[k] = D.b_c2[k];
+    b.copy[k] = D.b_copy[k];
+    b.crow[k] = D.b_crow[k];
   }
   for (int k = threadIdx.x; k < C * WIN; k += blockDim.x) b.chain[k] = D.b_chain[k];
   for (int k = threadIdx.x; k < words; k += blockDim.x) b.bits[k] = D.slot_bits[k];
@@ -636,6 +835,8 @@ __global__ void __launch_bounds__(256) k_book(Dev D, int mode, int arg) {
     D.b_gate[k] = b.gate[k];
     D.b_c1[k] = b.c1[k];
     D.b_c2[k] = b.c2[k];
+    D.b_copy[k] = b.copy[k];
+    D.b_crow[k] = b.crow[k];
   }
   for (int k = threadIdx.x; k < C * WIN; k += blockDim.x) D.b_chain[k] = b.chain[k];
   for (int k = threadIdx.x; k < words; k += blockDim.x) D.slot_bits[k] = b.bits[k];

@@ -180,6 +180,11 @@ static int validate(const lt_model_config* m, const lt_decode_config* dc, std::s
   if (dc->max_ctx + C + 8 > (1 << 24)) return bad("max_ctx too large");
   if (dc->temperature < 0.f || !(dc->top_p > 0.f) || dc->top_p > 1.f) return bad("temperature/top_p");
   if (dc->second_mode < 0 || dc->second_mode > 2) return bad("second_mode");
+  if (dc->copy_k < 0 || (dc->copy_k > 0 && (dc->copy_max_len < 1 || dc->copy_max_len > CPMAX ||
+                                            dc->copy_match_cap < dc->copy_k ||
+                                            dc->copy_reserve < 0 || !(dc->copy_tau >= 0.f))))
+    return bad("copy proposals: need copy_k <= copy_match_cap, 1 <= copy_max_len <= 32, copy_reserve >= 0, copy_tau >= 0");
+  if (dc->copy_k > 0 && dc->d1 < 1) return bad("copy proposals need d1 >= 1");
   return LT_OK;
 }
 
@@ -194,6 +199,9 @@ static size_t carve(Handle* H, char* base) {
                  &D.b_x1, &D.b_x2, &D.b_gate, &D.b_c1, &D.b_c2};
   for (int** p : tab) *p = cv.take<int>(C);
   D.b_chain = cv.take<int>((size_t)C * WIN);
+  int** cps[] = {&D.b_copy, &D.b_crow, &D.cp_fail, &D.cp_len, &D.v_tok, &D.v_src, &D.v_fb};
+  for (int** p : cps) *p = cv.take<int>(C);
+  D.cp_tok = cv.take<int>((size_t)C * CPMAX);
   int** rows[] = {&D.r_tok, &D.r_pos, &D.r_slot, &D.r_depth, &D.r_ro, &D.r_blen, &D.r_boff,
                   &D.m_alive, &D.m_new, &D.m_ro};
   for (int** p : rows) *p = cv.take<int>(C);
@@ -260,8 +268,8 @@ static size_t carve(Handle* H, char* base) {
   D.P = cv.take<float>((size_t)C * V);
   D.q1 = cv.take<float>((size_t)C * V);
   D.q2 = cv.take<float>((size_t)C * V);
-  D.rho = cv.take<float>(V);
-  D.rho2 = cv.take<float>(V);
+  D.rho = cv.take<float>((size_t)C * V);  // per row: rows of a copied chain verify in one step
+  D.rho2 = cv.take<float>((size_t)C * V);
   H->rope = cv.take<float2>((size_t)H->max_pos * (m.head_dim / 2));
   H->kv = cv.take<char>((size_t)H->planes * H->S * 2 * d * esz);
   return cv.off + 256;
@@ -307,6 +315,12 @@ static void plan(Handle* H) {
   D.T = dc.temperature;
   D.top_p = dc.top_p;
   D.seed = dc.seed;
+  D.copy_k = dc.copy_k;
+  D.copy_max = dc.copy_max_len;
+  D.copy_cap = dc.copy_match_cap;
+  D.copy_reserve = dc.copy_reserve;
+  D.copy_slack = dc.d1 > 0 ? (m.R + dc.d1 - 1) / dc.d1 : 0;
+  D.copy_tau = dc.copy_tau;
   for (int r = 0; r <= 32; ++r) D.tag_of_depth[r] = -1;
   for (int k = 0; k < n; ++k) D.tag_of_depth[H->tags[k]] = k;
 }
@@ -622,17 +636,22 @@ static cudaError_t decode_step(Handle* H) {
   Ctl* ctl = D.ctl;
   LT_CK(launch(H->use_pdl, k_embed<T>, dim3(C), dim3(EPI_THREADS), H->stream, (const T*)H->embed,
                (const int*)D.r_tok, (const int*)D.m_new, m.d_model, m.vocab, H->h, &ctl->err));
+  // With copy proposals a chain's rows share a depth and attend to each
+  // other's cache rows of the same pass, so every row's K/V is written by the
+  // QKV epilogue kernel before attention runs (the fused attention writes a
+  // row's own K/V inside its own work item).
+  const bool fused = D.copy_k == 0;
   H->prof_cat = 1;
   if (m.n_prelude > 0)
-    LT_CK(run_layers<T>(H, 0, m.n_prelude, 0, D.m_new, H->h, 1.f, &ctl->flag_new, true));
+    LT_CK(run_layers<T>(H, 0, m.n_prelude, 0, D.m_new, H->h, 1.f, &ctl->flag_new, fused));
   H->prof_cat = 0;
   if (H->use_pass)
     LT_CK(run_pass<T>(H));
   else
     LT_CK(run_layers<T>(H, m.n_prelude, m.n_core, 1, D.m_alive, H->h, m.resid_scale,
-                        &ctl->flag_run, true));
+                        &ctl->flag_run, fused));
   H->prof_cat = 1;
-  LT_CK(run_readout<T>(H, &ctl->flag_ro, true));
+  LT_CK(run_readout<T>(H, &ctl->flag_ro, fused));
   LT_CK(launch(H->use_pdl, k_decide, dim3(C), dim3(1024), H->stream, D));
   return launch(H->use_pdl, k_book, dim3(1), dim3(256), H->stream, D, 0, 0);
 }
@@ -717,7 +736,7 @@ extern "C" int lt_create(const lt_model_config* m, const lt_decode_config* dc, v
   H->use_pdl = !(e1 && e1[0] == '1');
   H->use_graph = !(e2 && e2[0] == '1');
   const char* e3 = getenv("LT_PASS");
-  H->use_pass = H->pass_ok && e3 && e3[0] == '1';
+  H->use_pass = H->pass_ok && e3 && e3[0] == '1' && dc->copy_k == 0;  // the pass kernel is fused
   // reducer tables of the five GEMM shapes
   const int gc = sm_count();
   const int d = m->d_model, f = m->ffn, V = m->vocab;
@@ -1041,7 +1060,8 @@ extern "C" int lt_generate(lt_handle* hd, int ar_mode, int n, int32_t* h_out, lt
   if ((rc = ensure_graph(hd))) return rc;
   int remaining = n;
   while (remaining > 0) {
-    // every step commits at most one token: `remaining` steps cannot overshoot
+    // a step commits at least 0 tokens and the device stops at the target, so
+    // `remaining` steps cannot overshoot (copied chains can commit several)
     if ((rc = run_steps(hd, remaining))) return rc;
     if ((rc = read_ctl(hd, &c))) return rc;
     remaining = L0 + n - c.L;
@@ -1065,6 +1085,10 @@ extern "C" int lt_generate(lt_handle* hd, int ar_mode, int n, int32_t* h_out, lt
     st->branches_created = c.branches_created;
     st->resid_fallback = c.resid_fallback;
     st->committed_len = c.L;
+    st->copy_chains = c.copy_chains;
+    st->copy_rows = c.copy_rows;
+    st->copy_cut = c.copy_cut;
+    st->n_copy = c.n_copy;
   }
   H->begun = false;
   return LT_OK;
@@ -1081,21 +1105,17 @@ extern "C" int lt_decode_step(lt_handle* hd, int ar_mode, int32_t* h_tok, int* n
     const int room = H->dc.max_ctx - c.L;
     if ((rc = begin(hd, std::min(H->dc.max_new, room), ar_mode ? 1 : 0))) return rc;
   }
+  if ((rc = read_ctl(hd, &c))) return rc;
+  const int before = c.n_commit;
   if ((rc = ensure_graph(hd))) return rc;
   if ((rc = run_steps(hd, 1))) return rc;
   if ((rc = read_ctl(hd, &c))) return rc;
-  int got = 0;
-  if (c.n_commit > 0 && c.steps > 0) {
-    int step_of_last = 0, tok = 0;
+  const int got = c.n_commit - before;
+  if (got > 0 && h_tok) {
     cudaError_t e;
-    if ((e = cudaMemcpyAsync(&step_of_last, H->D.log_step + c.n_commit - 1, 4, cudaMemcpyDeviceToHost, H->stream)) ||
-        (e = cudaMemcpyAsync(&tok, H->D.log_tok + c.n_commit - 1, 4, cudaMemcpyDeviceToHost, H->stream)) ||
+    if ((e = cudaMemcpyAsync(h_tok, H->D.log_tok + c.n_commit - 1, 4, cudaMemcpyDeviceToHost, H->stream)) ||
         (e = cudaStreamSynchronize(H->stream)))
       return cuda_fail(hd, e, "log readback");
-    if (step_of_last == c.steps) {
-      got = 1;
-      if (h_tok) *h_tok = tok;
-    }
   }
   if (n_committed) *n_committed = got;
   if (c.finished) H->begun = false;

@@ -40,7 +40,8 @@ Context-copy proposals (CopyLoop card, kongchang.com; oracle/copy.py has the
 lookup and the readings), when enabled, change steps 4-6 as follows:
   4a. a branch at depth d1 whose first proposal is a copied token (it has a
       copy child) is screened: if the token's depth-d1 score is below tau the
-      copy child's subtree is pruned and the branch proposes normally;
+      copy child's subtree is pruned (its slots freed at once) and the branch
+      makes an ordinary proposal (no new lookup);
   4b. a branch at depth d1 without a copy child looks up a copy proposal when
       no copy row outside its own ancestors is alive; if the first copied
       token passes the screen, x1 is that token (q1 one-hot) and the proposal
@@ -284,6 +285,7 @@ class SpecDecoder:
                  copy: Optional[CopyConfig] = None):
         assert 1 <= d1 < R and (d2 == 0 or d1 < d2 < R)
         self.copy = copy
+        self.copy_scores: List[float] = []  # every screen score evaluated (tests check margins)
         self.rows, self.R, self.d1, self.d2 = rows, R, d1, d2
         self.T, self.top_p, self.seed = temperature, top_p, seed
         self.second = second
@@ -401,12 +403,19 @@ class SpecDecoder:
             spawn = b.pos + 1 < self.pos_limit and b.pos + 1 - (L - 1) < WIN
             if b.depth == self.d1:
                 if b.copy_child:
-                    if CP.screen_score(b.z, b.x1) >= self.copy.tau:
+                    sc = CP.screen_score(b.z, b.x1)
+                    self.copy_scores.append(sc)
+                    if sc >= self.copy.tau:
                         continue  # the copied token goes on
                     st.copy_cut += len(self._subtree(b.child1))
                     for v in self._subtree(b.child1):
                         self.free.add(self.branches.pop(v).slot)
                     b.child1, b.copy_child = -1, False
+                    b.q1 = b.p  # an ordinary proposal; no new lookup
+                    b.x1 = S.race(b.q1, self.seed, b.uid, S.PROP1)
+                    if spawn:
+                        b.child1 = self._new_branch(b.uid, b.pos + 1, b.x1, b.chain).uid
+                    continue
                 b.q1 = b.p
                 b.x1 = S.race(b.q1, self.seed, b.uid, S.PROP1)
                 if spawn and self.copy is not None and self._copy_allowed(b):
@@ -451,7 +460,11 @@ class SpecDecoder:
         cp = self.copy
         seq = self.prefix_of(b)
         _, _, prop = CP.lookup(seq, L, cp.k, cp.max_len, cp.match_cap)
-        if not prop or CP.screen_score(b.z, prop[0]) < cp.tau:
+        if not prop:
+            return False
+        sc = CP.screen_score(b.z, prop[0])
+        self.copy_scores.append(sc)
+        if sc < cp.tau:
             return False
         m = min(len(prop),
                 cp.table - len(self.branches) - cp.reserve,  # free table rows beyond the reserve
