@@ -177,7 +177,8 @@ WORKLOAD = ("ouro14: Ouro-1.4B-shaped looped LM (bf16, 24 shared layers x R=4, d
 def run_ours(args):
     import torch
     import synthetic as syn
-    from looped_transformer_self_b200.binding import Decoder, lib, ProfileC, InfoC
+    from looped_transformer_self_b200.binding import CopyConfig, Decoder, lib, ProfileC, InfoC
+    from looped_transformer_self_b200 import copyloop
     import ctypes
 
     rank, local, ws = _dist()
@@ -199,6 +200,33 @@ def run_ours(args):
     _, am, _ = g.prefill(prompt, argmax=True)
     tags = sorted({r for r in (dec_g.d1, dec_g.d2, cfg.R) if r > 0})
     agree = float(np.mean(am[:, tags.index(dec_g.d1)] == am[:, tags.index(cfg.R)]))
+
+    # context-copy proposals (the Ouro-2.6B workload): tau calibrated on the
+    # prompt; the LoopSpec-only handle g stays for comparison
+    copy_on = args.copy == "on" or (args.copy == "auto" and args.model == "ouro26")
+    copy_info, g_plain = None, None
+    cc = None
+    if copy_on:
+        # calibration text: another prompt of the same recipe (not the timed
+        # one), 1024 tokens, and 512 tokens the decoder continues it with
+        cal_prompt = syn.prompt_for(args.model, seed=1001 + rank)[:1024]
+        cal = copyloop.calibrate(g, cal_prompt, warm=512)
+        slack = -(-cfg.R // dec_g.d1) + max(cfg.R - dec_g.d2, 0) // dec_g.d1 + 1
+        cc = CopyConfig(tau=cal["tau"], reserve=slack)
+        copy_info = {"calibration": cal, "k": cc.k, "max_len": cc.max_len,
+                     "match_cap": cc.match_cap, "reserve": cc.reserve, "max_branches": 32,
+                     "copied_prompt_fraction": syn.copy_prompt(P, cfg.vocab, 1 + rank)[1]}
+        if cal["admitted"] == 0:
+            # the calibration admits no copy proposal: decode without them
+            copy_info["decision"] = "off (no prompt proposal is more likely accepted than not)"
+            copy_on, cc = False, None
+        else:
+            copy_info["decision"] = "on"
+            g_plain = g
+            g = Decoder(cfg, dec_g, None, max_branches=32, max_ctx=P + 1 + n_new + 8,
+                        trace_steps=0, device=dev, copy=cc)
+            g.weights = g_plain.weights
+            g.bind_weights()
 
     def one_generate(ar=False):
         g.prefill(prompt)
@@ -226,8 +254,35 @@ def run_ours(args):
     # full-depth AR baseline and sampled decoding (same kernels), one run each
     ar_ms, ar_toks, ar_st = one_generate(ar=True)
     spec_equal_ar = ar_toks == toks
+    if g_plain is not None:  # LoopSpec proposals only, same prompt
+        g_plain.prefill(prompt)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(g_plain.stream)
+        plain_toks, plain_st = g_plain.generate(n_new)
+        e1.record(g_plain.stream)
+        e1.synchronize()
+        copy_info.update(loopspec_only_tokens_per_s=n_new / (e0.elapsed_time(e1) / 1e3),
+                         loopspec_only_stats=plain_st,
+                         loopspec_only_equals_ar=plain_toks == ar_toks,
+                         copy_vs_loopspec_only=(e0.elapsed_time(e1)) / times[-1])
+        g_plain.close()
+    if copy_info is not None:  # every copy proposal admitted (tau = 0), for context
+        g_f = Decoder(cfg, dec_g, None, max_branches=32, max_ctx=P + 1 + n_new + 8, device=dev,
+                      copy=CopyConfig(tau=0.0, reserve=copy_info["reserve"]))
+        g_f.weights = g.weights
+        g_f.bind_weights()
+        g_f.prefill(prompt)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(g_f.stream)
+        f_toks, f_st = g_f.generate(n_new)
+        e1.record(g_f.stream)
+        e1.synchronize()
+        copy_info.update(forced_tau0_tokens_per_s=n_new / (e0.elapsed_time(e1) / 1e3),
+                         forced_tau0_stats=f_st, forced_tau0_equals_ar=f_toks == ar_toks)
+        g_f.close()
     g_s = Decoder(cfg, syn.DECODES[f"{args.model}_sample"].replace(max_new=n_new, seed=2 + rank),
-                  None, max_branches=C, max_ctx=P + 1 + n_new + 8, device=dev)
+                  None, max_branches=32 if copy_on else C, max_ctx=P + 1 + n_new + 8, device=dev,
+                  copy=cc if copy_on else None)
     g_s.weights = g.weights
     g_s.bind_weights()
     g_s.prefill(prompt)
@@ -280,7 +335,7 @@ def run_ours(args):
                        "parallelism": f"replicas x{ws}",
                        "l2": "no flush: 2.47 GB of weights per pass exceed the 126 MB L2",
                        "resid_scale": cfg.resid_scale, "agreement_d1_vs_R": agree,
-                       "max_branches": C, "n_new": n_new, "prompt_len": P},
+                       "max_branches": 32 if copy_on else C, "n_new": n_new, "prompt_len": P},
             "speedup_vs_full_depth_ar": (ar_ms / times[-1]),
             "ar_tokens_per_s": n_new / (ar_ms / 1e3),
             "sampled_tokens_per_s": n_new / (sample_ms / 1e3),
@@ -301,6 +356,7 @@ def run_ours(args):
             "e2e": {"value": n_new / e2e_s, "unit": "tokens/s",
                     "h2d_bytes_per_step": 4 * P, "d2h_bytes_per_step": 4 * (n_new + 1),
                     "includes": "lt_prefill + lt_generate wall time, host buffers"},
+            "copy_proposals": copy_info,
             "gpu_launches": info["kernels_per_step"] * n_steps * args.steps,
             "clocks": clk.summary(),
             "profile": prof,
@@ -328,6 +384,8 @@ def main():
     ap.add_argument("--n-new", type=int, default=None,
                     help="decode tokens (default: the model's configured count)")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--copy", default="auto", choices=["auto", "on", "off"],
+                    help="context-copy proposals (auto: on for the Ouro-2.6B workload)")
     args = ap.parse_args()
     if args.impl == "reference":
         run_reference(args)
