@@ -115,17 +115,20 @@ def _barrier(ws):
 # CPU oracle baseline (also the --impl reference arm)
 # ---------------------------------------------------------------------------
 
-def oracle_sample(cfg, dec, prompt, weights, n_prompt=8, n_tokens=4):
+def oracle_sample(cfg, dec, prompt, weights, n_prompt=8, n_tokens=4, copy=None):
     """Oracle decode tokens/s on a bounded sample: the first n_prompt prompt
     tokens, then n_tokens greedy pipelined speculative decode tokens (decode
-    phase timed, like the metric)."""
+    phase timed, like the metric).  copy: the decoder's CopyConfig, if any."""
     from oracle import decode as D
     from oracle.model import LoopedModel
     t0 = time.perf_counter()
     rows = D.OracleRows(LoopedModel(cfg, weights, n_prompt + n_tokens + 16))
+    cp = None if copy is None else D.CopyConfig(tau=copy.tau, k=copy.k, max_len=copy.max_len,
+                                                 match_cap=copy.match_cap, table=32,
+                                                 reserve=copy.reserve)
     sd = D.SpecDecoder(rows, list(prompt[:n_prompt]), cfg.R, dec.d1, dec.d2, n_tokens,
                        dec.temperature, dec.top_p, dec.seed, n_prompt + n_tokens + 16,
-                       keep_trace=False)
+                       keep_trace=False, copy=cp)
     t1 = time.perf_counter()
     sd.run()
     t2 = time.perf_counter()
@@ -322,7 +325,8 @@ def run_ours(args):
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu:
-        cpu = oracle_sample(cfg, dec_g, prompt, weights, n_prompt=8, n_tokens=24)
+        cpu = oracle_sample(cfg, dec_g, prompt, weights, n_prompt=8, n_tokens=24,
+                            copy=cc if copy_on else None)
 
     if rank == 0:
         n_steps = stats["steps"]
