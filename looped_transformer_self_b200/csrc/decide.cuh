@@ -79,6 +79,8 @@ struct Dev {
   int* trace;      // [trace_cap][C][4]
   int* ro_arg;
   float *logits, *P, *q1, *q2, *rho, *rho2;
+  float* cb_val;  // per readout row and logit chunk: the chunk's max logit
+  int* cb_idx;    // and its index
 };
 
 // ---------------------------------------------------------------------------
@@ -104,37 +106,48 @@ __device__ __forceinline__ int block_race(const float* __restrict__ w, int V,
 }
 
 // ---------------------------------------------------------------------------
-// K4: readout processing of LM-head partials (one block of 1024 per readout row)
+// K4: readout processing of LM-head partials.
+// k_logits: logits of every readout row (final RMSNorm factor times the
+// reduced head GEMM partials) and each chunk's argmax, spread over
+// ceil(V / RO_CHUNK) blocks per row so the row's partials stream in parallel;
+// k_readout (one block of 1024 per readout row): the row's argmax from its
+// chunks (lowest index on ties, as one pass over the row would give), then
+// the readout processing (temperature, top-p, normalisation).
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(1024)
-    k_readout(const float* __restrict__ part, const GemmShape s, int C,
-              const int* __restrict__ mask, int V, int greedy, float T, float top_p,
-              float* __restrict__ logits, float* __restrict__ P, int* __restrict__ arg,
-              const float* __restrict__ ssq, int ssq_tiles, int d, float eps) {
+constexpr int RO_CHUNK = 2048;
+constexpr int RO_THREADS = 256;
+
+__host__ __device__ constexpr int ro_chunks(int V) { return (V + RO_CHUNK - 1) / RO_CHUNK; }
+
+__global__ void __launch_bounds__(RO_THREADS)
+    k_logits(const float* __restrict__ part, const GemmShape s, int C,
+             const int* __restrict__ mask, int V, float* __restrict__ logits,
+             float* __restrict__ cb_val, int* __restrict__ cb_idx, const float* __restrict__ ssq,
+             int ssq_tiles, int d, float eps) {
   __shared__ float sk[33];
   __shared__ int si[33];
-  __shared__ DistSmem ds;
   pdl_wait();
   pdl_trigger();
-  const int i = blockIdx.x;
+  const int i = blockIdx.y;
   if (!mask[i]) return;
+  const int nch = ro_chunks(V);
   float* z = logits + (size_t)i * V;
-  float* p = P + (size_t)i * V;
   const float rr = inv_rms_parts(ssq, ssq_tiles, C, i, d, eps);  // final RMSNorm factor
+  const int j0 = blockIdx.x * RO_CHUNK, j1 = min(V, j0 + RO_CHUNK);
   float best = -INFINITY;
   int bi = 0x7fffffff;
   // four elements per round so their partial loads overlap
-  for (int j0 = threadIdx.x; j0 < V; j0 += 4 * blockDim.x) {
+  for (int jb = j0 + threadIdx.x; jb < j1; jb += 4 * RO_THREADS) {
     float v[4];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      const int j = j0 + u * blockDim.x;
-      v[u] = j < V ? rr * sk_reduce(part, s, C, i, j) : 0.f;
+      const int j = jb + u * RO_THREADS;
+      v[u] = j < j1 ? rr * sk_reduce(part, s, C, i, j) : 0.f;
     }
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      const int j = j0 + u * blockDim.x;
-      if (j < V) {
+      const int j = jb + u * RO_THREADS;
+      if (j < j1) {
         z[j] = v[u];
         if (better_max(v[u], j, best, bi)) {
           best = v[u];
@@ -144,9 +157,43 @@ __global__ void __launch_bounds__(1024)
     }
   }
   const int a = block_arg<false>(best, bi, sk, si);
+  if (threadIdx.x == 0) {
+    const bool ok = a >= j0 && a < j1;  // false only when no value compared (NaN)
+    cb_val[(size_t)i * nch + blockIdx.x] = ok ? z[a] : -INFINITY;
+    cb_idx[(size_t)i * nch + blockIdx.x] = ok ? a : 0x7fffffff;
+  }
+}
+
+__global__ void __launch_bounds__(1024)
+    k_readout(const int* __restrict__ mask, int V, int greedy, float T, float top_p,
+              float* __restrict__ logits, float* __restrict__ P, int* __restrict__ arg,
+              const float* __restrict__ cb_val, const int* __restrict__ cb_idx, int* err) {
+  __shared__ float sk[33];
+  __shared__ int si[33];
+  __shared__ DistSmem ds;
+  pdl_wait();
+  pdl_trigger();
+  const int i = blockIdx.x;
+  if (!mask[i]) return;
+  const int nch = ro_chunks(V);
+  float best = -INFINITY;
+  int bi = 0x7fffffff;
+  for (int c = threadIdx.x; c < nch; c += blockDim.x) {
+    const float v = cb_val[(size_t)i * nch + c];
+    const int j = cb_idx[(size_t)i * nch + c];
+    if (better_max(v, j, best, bi)) {
+      best = v;
+      bi = j;
+    }
+  }
+  int a = block_arg<false>(best, bi, sk, si);
+  if (a < 0 || a >= V) {  // every logit was NaN
+    if (threadIdx.x == 0) set_err(err, DEV_BAD_INDEX);
+    a = 0;
+  }
   if (threadIdx.x == 0) arg[i] = a;
   if (greedy) return;
-  readout_dist(z, p, V, a, T, top_p, ds);
+  readout_dist(logits + (size_t)i * V, P + (size_t)i * V, V, a, T, top_p, ds);
 }
 
 // ---------------------------------------------------------------------------

@@ -268,6 +268,8 @@ static size_t carve(Handle* H, char* base) {
   D.P = cv.take<float>((size_t)C * V);
   D.q1 = cv.take<float>((size_t)C * V);
   D.q2 = cv.take<float>((size_t)C * V);
+  D.cb_val = cv.take<float>((size_t)C * ro_chunks(V));
+  D.cb_idx = cv.take<int>((size_t)C * ro_chunks(V));
   D.rho = cv.take<float>((size_t)C * V);  // per row: rows of a copied chain verify in one step
   D.rho2 = cv.take<float>((size_t)C * V);
   H->rope = cv.take<float2>((size_t)H->max_pos * (m.head_dim / 2));
@@ -525,9 +527,12 @@ static cudaError_t run_readout(Handle* H, const int* flag, bool fused) {
                (const float*)src, (const int*)D.m_ro, (const T*)H->final_norm, d, C, (T*)H->Xd,
                H->lo_d, H->ssq));
   LT_CK(gemm<T>(H, H->tm_head, H->tm_head_lo, H->tm_Xd, H->tm_Xd_lo, H->sh_head, flag));
-  return launch(H->use_pdl, k_readout, dim3(C), dim3(1024), H->stream, (const float*)H->part,
-                H->sh_head, C, (const int*)D.m_ro, m.vocab, D.greedy, D.T, D.top_p, D.logits,
-                D.P, D.ro_arg, (const float*)H->ssq, H->ssq_tiles, d, m.rms_eps);
+  LT_CK(launch(H->use_pdl, k_logits, dim3(ro_chunks(m.vocab), C), dim3(RO_THREADS), H->stream,
+               (const float*)H->part, H->sh_head, C, (const int*)D.m_ro, m.vocab, D.logits,
+               D.cb_val, D.cb_idx, (const float*)H->ssq, H->ssq_tiles, d, m.rms_eps));
+  return launch(H->use_pdl, k_readout, dim3(C), dim3(1024), H->stream, (const int*)D.m_ro,
+                m.vocab, D.greedy, D.T, D.top_p, D.logits, D.P, D.ro_arg,
+                (const float*)D.cb_val, (const int*)D.cb_idx, &D.ctl->err);
 }
 
 // Arguments of the persistent pass kernel (after the weights are loaded).
