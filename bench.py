@@ -160,7 +160,8 @@ def run_reference(args):
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 2000.0 / v, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": WORKLOAD, "l2": "weights larger than L2"},
+            "config": {"workload": WORKLOAD if args.model == "ouro14" else args.model,
+                       "l2": "weights larger than L2"},
             "cpu_baseline": dict(last, value=v),
             "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
