@@ -11,7 +11,9 @@ oracle/copy.py) against facts worked out by hand and against invariants:
 * scripted schedules (R = 4, d1 = 1, one proposal): a copied 5-token chain
   commits in one step after its root; a full-depth disagreement inside the
   chain restarts there; a depth-1 disagreement cuts the chain at the screen;
-* greedy speculative decoding with copies equals greedy full-depth decoding.
+* greedy speculative decoding with copies equals greedy full-depth decoding;
+* in sampled decoding the token after a copied proposal follows p_R (a
+  model whose readouts depend only on depth, 4000 seeds, chi-square).
 """
 import numpy as np
 import pytest
@@ -166,3 +168,47 @@ def test_tiny_greedy_with_copies_equals_full_depth():
                        2, 256, copy=cp)
     assert sp.tokens == ar.tokens
     assert sp.stats.copy_chains > 0
+
+
+class _SoftRows:
+    """Readouts whose logits depend only on the depth (a fixed soft p_r)."""
+
+    def __init__(self, z_by_depth):
+        self.z = z_by_depth
+
+    def prelude(self, prefix, pos, slots):
+        return None
+
+    def iterate(self, h, r, prefix, pos, slots):
+        return None
+
+    def readout(self, h, r, prefix, pos, slots, head=True):
+        return self.z[r].copy() if head else None
+
+
+def test_sampled_tokens_after_a_copy_follow_p_R():
+    """Sampled decoding (T = 1) with copies: prompt 1 2 3 4 5 1 2 3; when the
+    first token is 4, the root's lookup copies 5 1 2 3 and the next token is
+    verified with a one-hot proposal.  Over 4000 seeds the token after a
+    copied proposal is distributed as p_R (chi-square p > 0.01), and copies
+    were both accepted and rejected."""
+    V, R = 8, 4
+    rng = np.random.default_rng(9)
+    zR = np.log(np.array([0.04, 0.06, 0.05, 0.05, 0.45, 0.2, 0.1, 0.05]))
+    z = {r: zR + (4 - r) * 0.4 * rng.normal(size=V) for r in range(1, R + 1)}
+    pR = S.process(zR, 1.0, 1.0)
+    prompt = [1, 2, 3, 4, 5, 1, 2, 3]
+    counts = np.zeros(V)
+    copied = accepted = 0
+    for seed in range(4000):
+        cp = D.CopyConfig(tau=0.0, table=32, reserve=4)
+        sd = D.SpecDecoder(_SoftRows(z), prompt, R, 1, 0, 2, 1.0, 1.0, seed, 64, copy=cp)
+        res = sd.run()
+        if res.tokens[0] != 4:
+            continue
+        assert sd.stats.copy_chains >= 1
+        copied += 1
+        accepted += res.tokens[1] == 5
+        counts[res.tokens[1]] += 1
+    assert copied > 1000 and 0 < accepted < copied
+    assert scipy.stats.chisquare(counts, pR * copied).pvalue > 0.01
