@@ -262,6 +262,19 @@ int lt_readout_tv(float* d_za, long long stride_a, float* d_zb, long long stride
                   float T, float top_p, float* d_tv, void* stream);
 
 /*
+ * Self-test of the bounded waits (a test hook; the pages have no counterpart).
+ * Every pipeline wait in the library gives up after ~1 s, records
+ * DEV_TIMEOUT (1) and lets its kernel return, so a lost arrival ends in an
+ * error status instead of a hung GPU.  This call launches one warp that
+ * waits, through the same wait routine, on an mbarrier phase nothing
+ * completes, then a trivial kernel.  h_out (host, 3 ints): [0] the status
+ * the waiting kernel reported (1 = gave up), [1] 1 if the following kernel
+ * ran (the context stayed usable), [2] the wait's duration in ms.
+ * Synchronises `stream`.  Errors: LT_ERR_ARG (null h_out), LT_ERR_CUDA.
+ */
+int lt_selftest_wait(int32_t* h_out, void* stream);
+
+/*
  * Stand-alone weight-streaming GEMM of the shared block (tcgen05 + TMEM + TMA):
  *   d_y[i][n] = sum_k d_x[i][k] * d_w[n][k],  i < ncols, n < n_out.
  * This is the contraction every shared-block layer runs once per decode step

@@ -97,6 +97,7 @@ def _declare(L):
     L.lt_gemm_scratch_bytes.argtypes = [_i, _i, _i, _i, ctypes.POINTER(_sz)]
     L.lt_gemm_rows.argtypes = [_i, _vp, _vp, _vp, _i, _i, _i, _vp, _sz, _vp]
     L.lt_gemm_rows_noalloc.argtypes = [_i, _vp, _vp, _vp, _i, _i, _i, _vp]
+    L.lt_selftest_wait.argtypes = [_ip, _vp]
     L.lt_readout_tv.argtypes = [_vp, ctypes.c_longlong, _vp, ctypes.c_longlong, _i, _i,
                                 ctypes.c_float, ctypes.c_float, _vp, _vp]
     L.lt_workspace_bytes.argtypes = [ctypes.POINTER(ModelConfigC), ctypes.POINTER(DecodeConfigC),
@@ -184,6 +185,15 @@ def readout_tv(za: torch.Tensor, zb: torch.Tensor, temperature: float, top_p: fl
                               float(temperature), float(top_p), _ptr(tv), _stream(stream)),
           "lt_readout_tv")
     return tv
+
+
+def selftest_wait(stream=None) -> dict:
+    """lt_selftest_wait: a bounded wait that nothing releases must give up
+    (status 1), and the next kernel must still run."""
+    import numpy as np
+    out = np.zeros(3, dtype=np.int32)
+    check(lib().lt_selftest_wait(out.ctypes.data_as(_ip), _stream(stream)), "lt_selftest_wait")
+    return {"status": int(out[0]), "context_alive": bool(out[1]), "wait_ms": int(out[2])}
 
 
 # ---------------------------------------------------------------------------
