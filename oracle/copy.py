@@ -21,13 +21,13 @@ which is written separately):
   * screening score of a copied token s at a readout: softmax of the logits at
     T = 1 (no truncation), taken at s -- the model's own depth-d1 probability;
     a copied token goes on only when its score is >= tau;
-  * calibration of tau on the prompt: for every prompt position t whose prefix
-    has a copy proposal, score s_1 with the depth-d1 readout of t and note
-    whether the full-depth readout accepts it (greedy: its argmax is s_1;
-    sampling: with probability p_R(s_1)); tau is the score threshold that
-    maximises the sum over kept proposals of (2 accept - 1), i.e. a proposal is
-    kept when it is more likely accepted than not.  No proposal: tau = 1 (none
-    kept).
+  * calibration of tau on the prompt: for every prompt position t (the last
+    included) whose prefix has a copy proposal, score s_1 with the depth-d1
+    readout of t and note whether the full-depth readout accepts it (greedy:
+    its argmax is s_1; sampling: with probability p_R(s_1)); tau is the score
+    threshold that maximises the sum over kept proposals of (2 accept - 1),
+    i.e. a proposal is kept when it is more likely accepted than not.  No
+    proposal: tau = 1 (none kept).
 """
 from __future__ import annotations
 
@@ -83,8 +83,9 @@ def prompt_calibration(prompt: Sequence[int], z_d1, z_R, k: int, max_len: int, m
     readout logits of prompt position t.  Returns (tau, scores, accepts)."""
     from . import sampling as S
     scores, acc = [], []
-    for t in range(len(prompt) - 1):
-        # the prefix prompt[0..t] with all of it committed
+    for t in range(len(prompt)):
+        # the prefix prompt[0..t] with all of it committed (the last position
+        # too: its full-depth readout exists)
         _, _, prop = lookup(prompt[:t + 1], t + 1, k, max_len, match_cap)
         if not prop:
             continue
