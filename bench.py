@@ -349,6 +349,7 @@ def run_ours(args):
             "gamma_sampled": _gamma(st_s, dec_g.d1, dec_g.d2, cfg.R),
             "decode_stats": stats, "sampled_stats": st_s,
             "step_hbm": {"gbs": step_gbs, "frac_of_measured_hbm": step_gbs / hbm,
+                         "frac_of_8_tbs": step_gbs / 8000.0,
                          "bytes_per_step": step_bytes, "ms_per_step_graphed": graphed_ms,
                          "ms_per_step_profiled": prof["step_ms"] / max(prof["steps"], 1),
                          "peak_source": "measured" if peaks else "fallback"},
