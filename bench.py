@@ -319,10 +319,16 @@ def run_ours(args):
     step_bytes = (prof["gemm_core_bytes"] + prof["gemm_other_bytes"] + prof["kv_bytes"]) / max(prof["steps"], 1)
     graphed_ms = times[-1] / stats["steps"]
     step_gbs = step_bytes / (graphed_ms / 1e3) / 1e9
-    traffic = None
+    # DRAM traffic of the dominant kernel from an ncu capture, reported only
+    # while the GEMM sources are the ones that capture measured
+    traffic, traffic_note = None, "no capture"
     tf = os.path.join(ROOT, "profiles", "gemm_traffic.json")
     if os.path.exists(tf):
-        traffic = json.load(open(tf)).get("traffic_per_launch")
+        cap = json.load(open(tf))
+        if cap.get("source_sha256") == gemm_source_hash():
+            traffic, traffic_note = cap.get("traffic_per_launch"), "capture matches the GEMM sources"
+        else:
+            traffic_note = "GEMM sources changed since the capture"
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu:
@@ -356,6 +362,7 @@ def run_ours(args):
             "roofline": {"kernel": "k_gemm (tcgen05 weight-streaming GEMM)", "bound": "hbm",
                          "achieved": gemm_gbs, "peak": hbm, "unit": "GB/s",
                          "frac": gemm_gbs / hbm, "traffic": traffic,
+                         "traffic_note": traffic_note,
                          "peak_source": "measured" if peaks else "fallback",
                          "launches_profiled": prof["gemm_core_launches"]},
             "cpu_baseline": cpu,
@@ -372,6 +379,16 @@ def run_ours(args):
     if ws > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
+
+
+def gemm_source_hash():
+    """sha256 over the sources that make up k_gemm (a traffic capture records
+    the value it measured)."""
+    import hashlib
+    h = hashlib.sha256()
+    for f in ("gemm.cu", "gemm.cuh", "gemm_epi.cuh", "tc.cuh", "common.cuh"):
+        h.update(open(os.path.join(ROOT, "looped_transformer_self_b200", "csrc", f), "rb").read())
+    return h.hexdigest()
 
 
 def _gamma(st, d1, d2, R):
