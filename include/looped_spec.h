@@ -284,10 +284,14 @@ int lt_selftest_wait(int32_t* h_out, void* stream);
  *   d_w     [n_out][k] row-major (nn.Linear layout), 16-byte aligned, k*elem % 16 == 0.
  *   d_x     [ncols][k] row-major, same alignment; ncols in {8, 16, 32, 64}.
  *   d_y     [ncols][n_out] fp32.
- *   d_scratch  >= lt_gemm_scratch_bytes() bytes of device memory (reduction
- *              tables and fp32 partials); its contents are overwritten.
+ *   d_scratch  >= lt_gemm_scratch_bytes() bytes of device memory (an error
+ *              word, reduction tables and fp32 partials); its contents are
+ *              overwritten.
  * The call synchronises `stream` before returning.  The result for row i does
  * not depend on the other rows' values (the MMA always spans ncols columns).
+ * Errors: LT_ERR_ARG / LT_ERR_SHAPE (arguments), LT_ERR_CAPACITY (scratch too
+ * small), LT_ERR_CUDA (a runtime call failed), LT_ERR_DEVICE_CHECK (a bounded
+ * wait inside the kernel gave up after ~1 s; d_y is then not a valid result).
  */
 int lt_gemm_scratch_bytes(int dtype, int n_out, int k, int ncols, size_t* bytes);
 int lt_gemm_rows(int dtype, const void* d_w, const void* d_x, float* d_y, int n_out, int k,
@@ -304,13 +308,20 @@ int lt_gemm_rows(int dtype, const void* d_w, const void* d_x, float* d_y, int n_
  *     device that loads the library until the process exits; sizes whose
  *     scratch would exceed it return LT_ERR_CAPACITY (e.g. n_out 49152 with
  *     ncols 64);
- *   - the first call on a device resolves the array's device address, so make
- *     that first call before any stream capture;
- *   - every call shares the array: calls that overlap on the GPU (other
- *     streams, other threads) race; serialise them.  Nothing in the array needs
- *     clearing between calls;
- *   - it calls no cudaMalloc / cudaFree and no allocating library routine.
- * Arguments and result as lt_gemm_rows; synchronises `stream` before return.
+ *   - the first call on a device resolves the device addresses of the array
+ *     and of a static error word (cudaGetSymbolAddress), so that first call
+ *     must come before any stream capture; the addresses are kept for the
+ *     life of the process and assume the device's primary context is not
+ *     reset (cudaDeviceReset) in between;
+ *   - every call shares the array and the error word: calls that overlap on
+ *     the GPU (other streams, other threads) race; serialise them.  Each call
+ *     clears the error word before its launch; a completed GEMM writes every
+ *     partial its reduction reads, so nothing else needs clearing;
+ *   - it calls no cudaMalloc / cudaFree and no allocating library routine;
+ *   - every call copies its small reduction tables from the host and reads
+ *     the error word back, synchronising `stream` before it returns.
+ * Arguments, result and errors as lt_gemm_rows (LT_ERR_DEVICE_CHECK when a
+ * bounded wait of the kernel gave up).
  */
 #define LT_NOALLOC_SCRATCH_BYTES (8u << 20)
 int lt_gemm_rows_noalloc(int dtype, const void* d_w, const void* d_x, float* d_y, int n_out,

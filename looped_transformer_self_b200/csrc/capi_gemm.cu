@@ -32,7 +32,7 @@ extern "C" int lt_gemm_scratch_bytes(int dtype, int n_out, int k, int ncols, siz
   if (!bytes || n_out <= 0 || k <= 0) return LT_ERR_ARG;
   GemmShape s;
   gemm_plan(n_out, k, dtype == LT_F32, ncols, sm_count(), &s, nullptr, nullptr);
-  *bytes = align256((size_t)gemm_table_ints(n_out, k, dtype == LT_F32, ncols, sm_count()) *
+  *bytes = 256 /* error word */ + align256((size_t)gemm_table_ints(n_out, k, dtype == LT_F32, ncols, sm_count()) *
                     sizeof(int)) +
            align256(gemm_part_bytes(s, ncols));
   if (dtype == LT_F32) *bytes += 2 * align256((size_t)n_out * k * 4) + 2 * align256((size_t)ncols * k * 4);
@@ -54,13 +54,16 @@ extern "C" int lt_gemm_rows(int dtype, const void* d_w, const void* d_x, float* 
   std::vector<int> tab(gemm_table_ints(n_out, k, f32, ncols, sm_count()));
   gemm_plan(n_out, k, f32, ncols, sm_count(), &s, tab.data(), tab.data() + 2 * s.tiles);
   char* cur = (char*)d_scratch;
+  int* d_err = (int*)cur;  // DEV_TIMEOUT when a bounded wait of the GEMM gave up
+  cur += 256;
   int* d_tab = (int*)cur;
   cur += align256(tab.size() * sizeof(int));
   float* part = (float*)cur;
   cur += align256(gemm_part_bytes(s, ncols));
   cudaStream_t st = (cudaStream_t)stream;
-  if (cudaMemcpyAsync(d_tab, tab.data(), tab.size() * sizeof(int), cudaMemcpyHostToDevice, st) !=
-      cudaSuccess)
+  if (cudaMemsetAsync(d_err, 0, sizeof(int), st) != cudaSuccess ||
+      cudaMemcpyAsync(d_tab, tab.data(), tab.size() * sizeof(int), cudaMemcpyHostToDevice, st) !=
+          cudaSuccess)
     return LT_ERR_CUDA;
   s.tile_c = d_tab;
   s.cta_t0 = d_tab + 2 * s.tiles;
@@ -90,13 +93,17 @@ extern "C" int lt_gemm_rows(int dtype, const void* d_w, const void* d_x, float* 
     twl = tw;
     txl = tx;
   }
-  if (gemm_launch(tw, twl, tx, txl, part, s, ncols, f32 ? 2 : 0, nullptr, nullptr, st, false) !=
+  if (gemm_launch(tw, twl, tx, txl, part, s, ncols, f32 ? 2 : 0, nullptr, d_err, st, false) !=
       cudaSuccess)
     return LT_ERR_CUDA;
   dim3 grid((n_out + 255) / 256, ncols);
   k_reduce_rows<<<grid, 256, 0, st>>>(part, s, ncols, d_y);
   if (cudaGetLastError() != cudaSuccess) return LT_ERR_CUDA;
   // the host copy of the tables must outlive the async copy
-  if (cudaStreamSynchronize(st) != cudaSuccess) return LT_ERR_CUDA;
-  return LT_OK;
+  int h_err = 0;
+  if (cudaMemcpyAsync(&h_err, d_err, sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+      cudaStreamSynchronize(st) != cudaSuccess)
+    return LT_ERR_CUDA;
+  // a bounded wait gave up: d_y holds no valid result
+  return h_err ? LT_ERR_DEVICE_CHECK : LT_OK;
 }

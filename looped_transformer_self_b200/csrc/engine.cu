@@ -120,6 +120,13 @@ static int sm_count() {
   return n > 0 ? n : 148;
 }
 
+constexpr int kMaxDev = 64;
+static int cur_dev() {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  return dev >= 0 && dev < kMaxDev ? dev : 0;
+}
+
 static int* g_launch_counter = nullptr;  // set while the step graph is captured
 
 template <typename... KArgs, typename... Args>
@@ -398,8 +405,9 @@ static cudaError_t attention_items(Handle* H, int gl, const int* tagsrc, int tag
                                    const int* mask, T* Xo, bool fused) {
   const int C = H->C, Hn = H->m.n_heads;
   auto kern = fused ? k_attn<T, HD, true> : k_attn<T, HD, false>;
-  static int per_sm[2] = {0, 0};
-  int& nb = per_sm[fused ? 1 : 0];
+  // occupancy is a property of the device: cached per device ordinal
+  static int per_sm[kMaxDev][2] = {};
+  int& nb = per_sm[cur_dev()][fused ? 1 : 0];
   if (nb == 0 && (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kern, 128, 0) != cudaSuccess ||
                   nb < 1))
     nb = 1;
@@ -416,8 +424,10 @@ static cudaError_t attention(Handle* H, int gl, const int* tagsrc, int tag_off, 
   auto kern = fused ? k_attn2<T, HD, true> : k_attn2<T, HD, false>;
   // one resident wave of ring blocks (items are spread over them)
   const size_t smem = a2_smem_bytes<T, HD>();
-  static int per_sm[2] = {0, 0};
-  int& nb = per_sm[fused ? 1 : 0];
+  // the shared-memory attribute is set per device (function attributes belong
+  // to a context), and the occupancy that follows from it is cached with it
+  static int per_sm[kMaxDev][2] = {};
+  int& nb = per_sm[cur_dev()][fused ? 1 : 0];
   if (nb == 0) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
         cudaSuccess)

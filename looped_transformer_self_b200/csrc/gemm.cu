@@ -597,12 +597,16 @@ static cudaError_t launch_t(const GemmOperand& W, const GemmOperand& Wlo, const 
   const int stages = stages_for(NC, nsplit, s.kc);
   if (stages < 1) return cudaErrorInvalidValue;
   const size_t smem = smem_bytes(NC, stages, nsplit, s.kc);
-  static size_t attr_bytes = 0;
-  if (smem > attr_bytes) {
+  // function attributes belong to a context: remembered per device ordinal
+  static size_t attr_bytes[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  size_t& done = attr_bytes[dev >= 0 && dev < 64 ? dev : 0];
+  if (smem > done) {
     cudaError_t e = cudaFuncSetAttribute(k_gemm<MODE, NC>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    attr_bytes = smem;
+    done = smem;
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(s.grid);

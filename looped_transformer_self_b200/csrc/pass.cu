@@ -584,15 +584,17 @@ static size_t pass_smem_bytes(int ncols, int kc, int stages) {
 template <int NC, int HD>
 static cudaError_t launch_pass(const PassParams& p, cudaStream_t stream) {
   const size_t smem = pass_smem_bytes(NC, p.sh[0].kc, p.stages);
-  static size_t attr_bytes = 0;
-  if (smem > attr_bytes) {
+  int dev = 0, sms = 0;
+  cudaGetDevice(&dev);
+  // function attributes belong to a context: remembered per device ordinal
+  static size_t attr_bytes[64] = {};
+  size_t& done = attr_bytes[dev >= 0 && dev < 64 ? dev : 0];
+  if (smem > done) {
     cudaError_t e = cudaFuncSetAttribute(k_pass<NC, HD>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    attr_bytes = smem;
+    done = smem;
   }
-  int dev = 0, sms = 0;
-  cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(sms);

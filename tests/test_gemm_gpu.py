@@ -67,3 +67,24 @@ def test_gemm_rows_are_independent_and_deterministic():
     xz = torch.zeros_like(x)
     xz[9] = x[0]
     assert torch.equal(gemm_rows(w, xz)[9], y1[0])
+
+
+def test_gemm_returns_ok_status_word():
+    """A normal call clears the scratch's error word, runs, finds the word
+    still 0 after its synchronisation and returns LT_OK (a bounded wait that
+    gave up would make it LT_ERR_DEVICE_CHECK; the give-up path itself is
+    exercised by tests/test_selftest_gpu.py without a fault)."""
+    import ctypes
+    from looped_transformer_self_b200.binding import LT_BF16, lib
+    w = torch.randn(2048, 2048).bfloat16().cuda()
+    x = torch.randn(16, 2048).bfloat16().cuda()
+    y = torch.empty(16, 2048, dtype=torch.float32, device="cuda")
+    need = ctypes.c_size_t()
+    assert lib().lt_gemm_scratch_bytes(LT_BF16, 2048, 2048, 16, ctypes.byref(need)) == 0
+    scratch = torch.full((need.value,), 0xFF, dtype=torch.uint8, device="cuda")  # word != 0 before
+    torch.cuda.synchronize()
+    for _ in range(2):
+        rc = lib().lt_gemm_rows(LT_BF16, w.data_ptr(), x.data_ptr(), y.data_ptr(), 2048, 2048, 16,
+                                scratch.data_ptr(), need.value, torch.cuda.current_stream().cuda_stream)
+        assert rc == 0
+    assert int(scratch[:4].view(torch.int32).item()) == 0

@@ -31,6 +31,19 @@ def test_noalloc_matches_allocating_entry_on_two_calls(n_out, k, ncols):
         assert torch.all((got - ref).abs() <= _bound(w, x, k)), (call, float((got - ref).abs().max()))
 
 
+def test_noalloc_returns_ok_status_on_two_calls():
+    """Each call clears the library's static error word before its launch and
+    reads it back after its synchronisation: a normal call returns LT_OK."""
+    from looped_transformer_self_b200.binding import LT_BF16, lib
+    w = torch.randn(2048, 2048).bfloat16().cuda()
+    x = torch.randn(16, 2048).bfloat16().cuda()
+    y = torch.empty(16, 2048, dtype=torch.float32, device="cuda")
+    for _ in range(2):
+        rc = lib().lt_gemm_rows_noalloc(LT_BF16, w.data_ptr(), x.data_ptr(), y.data_ptr(), 2048,
+                                        2048, 16, torch.cuda.current_stream().cuda_stream)
+        assert rc == 0
+
+
 def test_noalloc_rejects_sizes_beyond_its_scratch():
     from looped_transformer_self_b200.binding import LoopedSpecError, gemm_rows_noalloc
     w = torch.zeros(49152, 2048, dtype=torch.bfloat16, device="cuda")
