@@ -86,7 +86,7 @@ typedef struct {
   float copy_tau;
 } lt_decode_config;
 
-/* Per-generate statistics (section 3.2 Eq. 9 counts, Fig. 5, Table 6, Fig. 6). */
+/* Per-decode statistics (section 3.2 Eq. 9 counts, Fig. 5, Table 6, Fig. 6). */
 typedef struct {
   int steps;            /* batched shared-block passes */
   int rows_sum, rows_max;  /* active branches per pass: sum and peak */
@@ -145,9 +145,29 @@ int lt_prefill(lt_handle* h, const int32_t* h_tokens, int n, int32_t* h_first,
  * Greedy speculative output equals greedy AR output bit for bit.
  */
 int lt_generate(lt_handle* h, int ar_mode, int n, int32_t* h_out, lt_stats* st);
-/* One batched pass.  *n_committed = the tokens this pass committed (0 or 1;
- * with copy proposals several) and *h_tok = the last of them. */
-int lt_decode_step(lt_handle* h, int ar_mode, int32_t* h_tok, int* n_committed);
+/* What one batched pass did (section 3.2 Eq. 9 counts and section 3.4's
+ * mechanism statistics, per step). */
+typedef struct {
+  int step;             /* 1-based index of the pass within the current decode */
+  int rows;             /* active branches the pass advanced */
+  int n_committed;      /* tokens it committed (0 or 1; with copy proposals several) */
+  int n_first, n_second, n_fallback;  /* their sources: first / second proposal, full-depth draw */
+  int n_copy;           /* of n_first: copied tokens */
+  int gate_checks, gate_opens;  /* second-proposal gates evaluated / opened */
+  int branches_created; /* children opened */
+  int committed_len;    /* committed length after the pass */
+  int finished;         /* 1 when the decode reached its token budget */
+} lt_step_info;
+/* One batched pass (the first call after lt_prefill starts a decode of
+ * max_new tokens, or fewer if max_ctx leaves less room).  *n_committed = the
+ * tokens this pass committed and *h_tok = the last of them; info (may be NULL)
+ * receives the pass's statistics.  Synchronises the handle's stream. */
+int lt_decode_step(lt_handle* h, int ar_mode, int32_t* h_tok, int* n_committed,
+                   lt_step_info* info);
+/* Running totals of the current decode (or the last one, once it finished):
+ * the counters of lt_stats since lt_generate or the decode's first
+ * lt_decode_step began.  Errors: LT_ERR_STATE before the first prefill. */
+int lt_get_stats(lt_handle* h, lt_stats* st);
 /*
  * Explicit edits of the branch tree between two decode steps (after
  * lt_decode_step; the next step sees the edited tree).  The pages' own
@@ -260,6 +280,38 @@ void lt_destroy(lt_handle* h);
  */
 int lt_readout_tv(float* d_za, long long stride_a, float* d_zb, long long stride_b, int n, int V,
                   float T, float top_p, float* d_tv, void* stream);
+
+/*
+ * Calibration of the copy screen on a committed text (CopyLoop card,
+ * kongchang.com: copied continuations are scored at a shallow loop depth, and
+ * a light calibration sets the threshold that admits them to the full-depth
+ * verification; the copy_* fields of lt_decode_config use the same lookup and
+ * score).  For each position t of d_tokens[0..n-1]:
+ *   d_tok[t]    the first token the decoder's copy lookup proposes after the
+ *               prefix d_tokens[0..t], all of it committed: the end e of the
+ *               earlier occurrence (k-1 <= e <= t-1) whose backward match with
+ *               the prefix's end is longest (>= k, capped at match_cap; the
+ *               most recent on ties) gives d_tokens[e+1]; -1 when none;
+ *   d_score[t]  its screen score, softmax of d_z1 row t at T = 1, taken at
+ *               that token (-1 when none);
+ *   d_accept[t] the probability that full depth accepts it as a one-hot
+ *               draft: T = 0, 1 if it is the argmax of d_zR row t (lowest index
+ *               on ties), else 0; T > 0, its probability after the readout
+ *               processing of d_zR row t (temperature T, top-p, normalisation);
+ *               0 when none.
+ *   d_z1, d_zR  device fp32 logits, row t at base + t * stride (elements, >= V):
+ *               the depth-d1 and full-depth readouts of position t (e.g. the
+ *               d_logits of lt_prefill); d_zR is OVERWRITTEN with the processed
+ *               distribution when T > 0.
+ *   d_tokens, d_tok (device int32 [n]), d_score, d_accept (device fp32 [n]).
+ * Asynchronous on `stream`; allocates nothing.  Errors: LT_ERR_ARG (null
+ * pointer with n > 0, V <= 0, k < 1, match_cap < k, T < 0, top_p outside
+ * (0, 1], a stride below V), LT_ERR_CUDA (launch).
+ */
+int lt_copy_screen_scores(const int32_t* d_tokens, int n, int k, int match_cap,
+                          const float* d_z1, long long stride1, float* d_zR, long long strideR,
+                          int V, float T, float top_p, int32_t* d_tok, float* d_score,
+                          float* d_accept, void* stream);
 
 /*
  * Self-test of the bounded waits (a test hook; the pages have no counterpart).

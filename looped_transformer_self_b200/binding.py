@@ -67,6 +67,15 @@ class StatsC(ctypes.Structure):
         return {n: getattr(self, n) for n, _ in self._fields_}
 
 
+class StepInfoC(ctypes.Structure):
+    _fields_ = [(n, _i) for n in ("step", "rows", "n_committed", "n_first", "n_second",
+                                   "n_fallback", "n_copy", "gate_checks", "gate_opens",
+                                   "branches_created", "committed_len", "finished")]
+
+    def as_dict(self):
+        return {n: getattr(self, n) for n, _ in self._fields_}
+
+
 class ProfileC(ctypes.Structure):
     _fields_ = [("steps", _i), ("rows", _i), ("step_ms", ctypes.c_double),
                 ("gemm_core_ms", ctypes.c_double), ("gemm_core_bytes", ctypes.c_double),
@@ -107,7 +116,11 @@ def _declare(L):
     L.lt_load_weights.argtypes = [_vp, _vp, _vp, _vp, ctypes.POINTER(_vp)]
     L.lt_prefill.argtypes = [_vp, _ip, _i, _ip, _ip, _vp]
     L.lt_generate.argtypes = [_vp, _i, _i, _ip, ctypes.POINTER(StatsC)]
-    L.lt_decode_step.argtypes = [_vp, _i, _ip, ctypes.POINTER(_i)]
+    L.lt_decode_step.argtypes = [_vp, _i, _ip, ctypes.POINTER(_i), ctypes.POINTER(StepInfoC)]
+    L.lt_get_stats.argtypes = [_vp, ctypes.POINTER(StatsC)]
+    L.lt_copy_screen_scores.argtypes = [_vp, _i, _i, _i, _vp, ctypes.c_longlong, _vp,
+                                        ctypes.c_longlong, _i, ctypes.c_float, ctypes.c_float,
+                                        _vp, _vp, _vp, _vp]
     L.lt_read_log.argtypes = [_vp, _ip, _ip, _ip, _i]
     L.lt_read_trace.argtypes = [_vp, _ip, _i]
     L.lt_read_committed.argtypes = [_vp, _ip, _ip, ctypes.POINTER(_i)]
@@ -185,6 +198,28 @@ def readout_tv(za: torch.Tensor, zb: torch.Tensor, temperature: float, top_p: fl
                               float(temperature), float(top_p), _ptr(tv), _stream(stream)),
           "lt_readout_tv")
     return tv
+
+
+def copy_screen_scores(tokens: torch.Tensor, z1: torch.Tensor, zR: torch.Tensor, k: int,
+                       match_cap: int, temperature: float, top_p: float, stream=None):
+    """lt_copy_screen_scores: per position of the committed text `tokens`
+    (device int32 [n]) the first copied token of the decoder's lookup (-1:
+    none), its depth-d1 screen score (softmax of z1 at T = 1) and its
+    full-depth acceptance probability from zR (fp32 [n][V] views, unit column
+    stride).  zR is overwritten with the processed distributions when
+    temperature > 0.  Returns (tok, score, accept) device tensors."""
+    assert tokens.is_cuda and tokens.dtype == torch.int32 and tokens.dim() == 1
+    assert z1.dtype == zR.dtype == torch.float32 and z1.shape == zR.shape
+    assert z1.stride(1) == 1 and zR.stride(1) == 1 and z1.shape[0] == tokens.shape[0]
+    n, V = z1.shape
+    tok = torch.empty(n, dtype=torch.int32, device=tokens.device)
+    score = torch.empty(n, dtype=torch.float32, device=tokens.device)
+    acc = torch.empty(n, dtype=torch.float32, device=tokens.device)
+    check(lib().lt_copy_screen_scores(_ptr(tokens), n, k, match_cap, _ptr(z1), z1.stride(0),
+                                      _ptr(zR), zR.stride(0), V, float(temperature),
+                                      float(top_p), _ptr(tok), _ptr(score), _ptr(acc),
+                                      _stream(stream)), "lt_copy_screen_scores")
+    return tok, score, acc
 
 
 def selftest_wait(stream=None) -> dict:
@@ -309,12 +344,22 @@ class Decoder:
                     "lt_generate")
         return out[:n].tolist(), st.as_dict()
 
-    def step(self, ar=False):
+    def step(self, ar=False, info=False):
+        """One decode pass: the last token it committed (None if none); with
+        info=True also the pass's lt_step_info as a dict."""
         tok = self.np.zeros(1, dtype=self.np.int32)
         n = _i()
-        self._check(lib().lt_decode_step(self.h, 1 if ar else 0, _i32p(tok), ctypes.byref(n)),
-                    "lt_decode_step")
-        return int(tok[0]) if n.value else None
+        si = StepInfoC()
+        self._check(lib().lt_decode_step(self.h, 1 if ar else 0, _i32p(tok), ctypes.byref(n),
+                                         ctypes.byref(si)), "lt_decode_step")
+        t = int(tok[0]) if n.value else None
+        return (t, si.as_dict()) if info else t
+
+    def stats(self):
+        """lt_get_stats: running totals of the current (or last) decode."""
+        st = StatsC()
+        self._check(lib().lt_get_stats(self.h, ctypes.byref(st)), "lt_get_stats")
+        return st.as_dict()
 
     def kv_pool(self):
         """(torch view of the KV pool [planes, slots, 2, d], plane of core layer 0)."""

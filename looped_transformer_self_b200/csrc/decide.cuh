@@ -246,14 +246,6 @@ __device__ __forceinline__ int block_max_int(int v, int* si) {
 // Screen score of token s (CopyLoop card: copied tokens are scored at a
 // shallow depth): softmax of the row's logits z at T = 1, taken at s.
 // a: the row's argmax.
-__device__ __forceinline__ float copy_score(const float* __restrict__ z, int V, int a, int s,
-                                            float* red) {
-  const float zmax = z[a];
-  float acc = 0.f;
-  for (int j = threadIdx.x; j < V; j += blockDim.x) acc += expf(z[j] - zmax);
-  const float Z = block_sum(acc, red);
-  return expf(z[s] - zmax) / Z;
-}
 
 // Copy proposal of entry i (position pos, L committed tokens): the end e of
 // the earlier committed occurrence whose backward match with the prefix's end

@@ -1017,6 +1017,25 @@ static int read_ctl(lt_handle* hd, Ctl* c) {
   return LT_OK;
 }
 
+// Running totals of the device counters since the current decode began.
+static void fill_stats(const Ctl& c, lt_stats* st) {
+  st->steps = c.steps;
+  st->rows_sum = c.rows_sum;
+  st->rows_max = c.rows_max;
+  st->n_first = c.n_first;
+  st->n_second = c.n_second;
+  st->n_fallback = c.n_fallback;
+  st->gate_checks = c.gate_checks;
+  st->gate_opens = c.gate_opens;
+  st->branches_created = c.branches_created;
+  st->resid_fallback = c.resid_fallback;
+  st->committed_len = c.L;
+  st->copy_chains = c.copy_chains;
+  st->copy_rows = c.copy_rows;
+  st->copy_cut = c.copy_cut;
+  st->n_copy = c.n_copy;
+}
+
 static int ensure_graph(lt_handle* hd) {
   Handle* H = &hd->h;
   if (!H->use_graph || H->graph) return LT_OK;
@@ -1088,28 +1107,24 @@ extern "C" int lt_generate(lt_handle* hd, int ar_mode, int n, int32_t* h_out, lt
         (e = cudaStreamSynchronize(H->stream)))
       return cuda_fail(hd, e, "tokens readback");
   }
-  if (st) {
-    st->steps = c.steps;
-    st->rows_sum = c.rows_sum;
-    st->rows_max = c.rows_max;
-    st->n_first = c.n_first;
-    st->n_second = c.n_second;
-    st->n_fallback = c.n_fallback;
-    st->gate_checks = c.gate_checks;
-    st->gate_opens = c.gate_opens;
-    st->branches_created = c.branches_created;
-    st->resid_fallback = c.resid_fallback;
-    st->committed_len = c.L;
-    st->copy_chains = c.copy_chains;
-    st->copy_rows = c.copy_rows;
-    st->copy_cut = c.copy_cut;
-    st->n_copy = c.n_copy;
-  }
+  if (st) fill_stats(c, st);
   H->begun = false;
   return LT_OK;
 }
 
-extern "C" int lt_decode_step(lt_handle* hd, int ar_mode, int32_t* h_tok, int* n_committed) {
+extern "C" int lt_get_stats(lt_handle* hd, lt_stats* st) {
+  if (!hd || !st) return LT_ERR_ARG;
+  Handle* H = &hd->h;
+  if (!H->prefilled) return fail(hd, LT_ERR_STATE, "prefill first");
+  Ctl c;
+  const int rc = read_ctl(hd, &c);
+  if (rc) return rc;
+  fill_stats(c, st);
+  return LT_OK;
+}
+
+extern "C" int lt_decode_step(lt_handle* hd, int ar_mode, int32_t* h_tok, int* n_committed,
+                              lt_step_info* info) {
   if (!hd) return LT_ERR_ARG;
   Handle* H = &hd->h;
   if (!H->prefilled) return fail(hd, LT_ERR_STATE, "prefill first");
@@ -1121,11 +1136,26 @@ extern "C" int lt_decode_step(lt_handle* hd, int ar_mode, int32_t* h_tok, int* n
     if ((rc = begin(hd, std::min(H->dc.max_new, room), ar_mode ? 1 : 0))) return rc;
   }
   if ((rc = read_ctl(hd, &c))) return rc;
+  const Ctl c0 = c;
   const int before = c.n_commit;
   if ((rc = ensure_graph(hd))) return rc;
   if ((rc = run_steps(hd, 1))) return rc;
   if ((rc = read_ctl(hd, &c))) return rc;
   const int got = c.n_commit - before;
+  if (info) {  // this pass's share of the running counters
+    info->step = c.steps;
+    info->rows = c.rows_sum - c0.rows_sum;
+    info->n_committed = got;
+    info->n_first = c.n_first - c0.n_first;
+    info->n_second = c.n_second - c0.n_second;
+    info->n_fallback = c.n_fallback - c0.n_fallback;
+    info->n_copy = c.n_copy - c0.n_copy;
+    info->gate_checks = c.gate_checks - c0.gate_checks;
+    info->gate_opens = c.gate_opens - c0.gate_opens;
+    info->branches_created = c.branches_created - c0.branches_created;
+    info->committed_len = c.L;
+    info->finished = c.finished;
+  }
   if (got > 0 && h_tok) {
     cudaError_t e;
     if ((e = cudaMemcpyAsync(h_tok, H->D.log_tok + c.n_commit - 1, 4, cudaMemcpyDeviceToHost, H->stream)) ||

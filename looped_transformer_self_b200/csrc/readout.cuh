@@ -170,4 +170,17 @@ __device__ __forceinline__ void readout_dist(const float* z, float* p, int V, in
   }
 }
 
+// Screen score of a copied token s (CopyLoop card: copied continuations are
+// scored at a shallow depth): softmax of the row's logits at T = 1, taken at
+// s.  a: the row's argmax.  One block; `red` holds >= 33 floats.  The decode
+// step's screen and the calibration call both use this.
+__device__ __forceinline__ float copy_score(const float* __restrict__ z, int V, int a, int s,
+                                            float* red) {
+  const float zmax = z[a];
+  float acc = 0.f;
+  for (int j = threadIdx.x; j < V; j += blockDim.x) acc += expf(z[j] - zmax);
+  const float Z = block_sum(acc, red);
+  return expf(z[s] - zmax) / Z;
+}
+
 }  // namespace lt

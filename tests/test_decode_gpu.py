@@ -297,3 +297,44 @@ def test_tree_edits_match_oracle(tiny, fill):
     table = g.read_table()
     live = sorted(int(table[1, k]) for k in range(table.shape[1]) if table[0, k])
     assert live == sorted(sd.branches)
+
+
+def test_step_info_and_running_stats_match_oracle(tiny):
+    """lt_decode_step's lt_step_info, pass by pass, against the oracle's own
+    record of the same greedy decode: rows advanced (the step's trace),
+    tokens committed and their sources (commit steps and sources), gate checks
+    and opens and children created (deltas of the oracle's counters); and
+    lt_get_stats equals the oracle's totals after every step."""
+    from oracle import decode as D
+    from oracle.model import LoopedModel
+    cfg, w, prompt = tiny
+    dec = syn.DECODES["tiny_greedy"].replace(d1=1, d2=2, max_new=20)
+    g = _decoder(cfg, dec, w, max_branches=16)
+    g.prefill(prompt)
+    sd = D.SpecDecoder(D.OracleRows(LoopedModel(cfg, w, 256)), prompt, cfg.R, dec.d1, dec.d2,
+                       dec.max_new, 0.0, 1.0, dec.seed, 256)
+    fields = ("gate_checks", "gate_opens", "branches_created")
+    while not sd.done():
+        before = {f: getattr(sd.stats, f) for f in fields}
+        n_src = len(sd.src)
+        sd.step()
+        tok, info = g.step(info=True)
+        k = sd.stats.steps
+        assert info["step"] == k
+        assert info["rows"] == len(sd.trace[k - 1])
+        new_src = sd.src[n_src:]
+        assert info["n_committed"] == len(new_src)
+        assert (info["n_first"], info["n_second"], info["n_fallback"]) == (
+            new_src.count(1), new_src.count(2), new_src.count(0))
+        if new_src:
+            assert tok == sd.committed[-1]
+        for f in fields:
+            assert info[f] == getattr(sd.stats, f) - before[f], f
+        assert info["committed_len"] == len(sd.committed)
+        assert info["finished"] == int(sd.done())
+        st = g.stats()
+        for f in ("steps", "rows_sum", "rows_max", "n_first", "n_second", "n_fallback",
+                  "gate_checks", "gate_opens", "branches_created"):
+            assert st[f] == getattr(sd.stats, f), f
+    assert sd.stats.n_first > 0 and sd.stats.gate_opens > 0
+    g.close()
