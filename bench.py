@@ -1,17 +1,20 @@
 """Decode benchmark: pipelined self-speculative decoding of a looped LM on B200.
 
-Workload (the pages' single-request decode setting, LoopSpec page section 3.1):
-an Ouro-1.4B-shaped looped LM (bf16, random init with the residual scale tuned
-for depth-1 vs depth-4 top-1 agreement ~0.6; shared stack 24 layers x R = 4,
-d 2048, 16 x 128 heads, SwiGLU 5632, vocab 49152), a 512-token Zipf(1.1)
-prompt, 1024 decoded tokens, proposal readouts at depths 1 and 2.
+Default workload (the pages' single-request decode setting, LoopSpec page
+section 3.1, on the largest configuration that fits one GPU): a Huginn/Raven-
+3.5B-shaped looped LM (bf16, random init with the residual scale tuned for
+depth-8 vs depth-32 top-1 agreement ~0.7; prelude 2 layers, core block 4
+layers looped R = 32, coda 2 layers; d 5280, 55 x 96 heads, SwiGLU 17920,
+vocab 65536), a 256-token Zipf(1.1) prompt, 512 decoded tokens, proposal
+readouts at depths 8 and 16.  `--model ouro14 | ouro26 | tiny` selects the
+other workloads.
 
 One bench step = prefill (untimed: the pages time the decode phase only) +
-one greedy pipelined speculative decode of 1024 tokens through the C ABI,
-timed with CUDA events on the decoder's stream.  value = decoded tokens / s
-summed over ranks (replicas: one independent request per GPU, no collective
-on the data path).  The weights (2.47 GB per shared-block pass) exceed the
-126 MB L2, so no flush is needed between steps.
+one greedy pipelined speculative decode of the workload's tokens through the
+C ABI, timed with CUDA events on the decoder's stream.  value = decoded
+tokens / s summed over ranks (replicas: one independent request per GPU, no
+collective on the data path).  The shared block's weights exceed the 126 MB
+L2, so no flush is needed between steps.
 
 `--impl reference` times the CPU oracle (the plain fp64 implementation the
 GPU path is checked against) on the host cores on a bounded sample of the
@@ -115,63 +118,111 @@ def _barrier(ws):
 # CPU oracle baseline (also the --impl reference arm)
 # ---------------------------------------------------------------------------
 
-def oracle_sample(cfg, dec, prompt, weights, n_prompt=8, n_tokens=4, copy=None):
-    """Oracle decode tokens/s on a bounded sample: the first n_prompt prompt
-    tokens, then n_tokens greedy pipelined speculative decode tokens (decode
-    phase timed, like the metric).  copy: the decoder's CopyConfig, if any."""
-    from oracle import decode as D
-    from oracle.model import LoopedModel
-    t0 = time.perf_counter()
-    rows = D.OracleRows(LoopedModel(cfg, weights, n_prompt + n_tokens + 16))
-    cp = None if copy is None else D.CopyConfig(tau=copy.tau, k=copy.k, max_len=copy.max_len,
-                                                 match_cap=copy.match_cap, table=32,
-                                                 reserve=copy.reserve)
-    sd = D.SpecDecoder(rows, list(prompt[:n_prompt]), cfg.R, dec.d1, dec.d2, n_tokens,
-                       dec.temperature, dec.top_p, dec.seed, n_prompt + n_tokens + 16,
-                       keep_trace=False, copy=cp)
-    t1 = time.perf_counter()
-    sd.run()
-    t2 = time.perf_counter()
-    return {"value": n_tokens / (t2 - t1), "unit": "tokens/s", "cores": os.cpu_count(),
-            "kind": "oracle",
-            "sample": f"{cfg.name}: prompt truncated to {n_prompt} tokens, {n_tokens} greedy "
-                      f"speculative decode tokens (d1={dec.d1}, d2={dec.d2}); prefill "
-                      f"{t1 - t0:.1f}s untimed, decode {t2 - t1:.1f}s timed, fp64 on "
-                      f"{os.cpu_count()} host threads"}
+# bounded oracle samples per workload (prompt tokens kept, decode tokens timed
+# per sample): about 10-30 s of fp64 host work for the CPU baseline; the
+# reference arm times one sample per step
+ORACLE_SAMPLE = {"tiny": (32, 64), "ouro14": (8, 24), "huginn35": (2, 2), "ouro26": (8, 16)}
+REFERENCE_SAMPLE = {"tiny": (32, 16), "ouro14": (8, 4), "huginn35": (2, 1), "ouro26": (8, 4)}
+
+
+class OracleSample:
+    """The CPU oracle on a bounded sample of a workload: the prompt truncated
+    to n_prompt tokens is prefilled once (untimed, as the metric excludes
+    prefill), its caches are kept, and each timed sample restores them and
+    runs the oracle's pipelined speculative decoder for n_tokens tokens."""
+
+    def __init__(self, cfg, dec, prompt, weights, n_prompt, n_tokens, copy=None):
+        from oracle import decode as D
+        from oracle.model import LoopedModel
+        self.D, self.cfg, self.dec = D, cfg, dec
+        self.n_prompt, self.n_tokens = n_prompt, n_tokens
+        self.prompt = list(prompt[:n_prompt])
+        self.n_slots = n_prompt + n_tokens + 24
+        self.cp = None if copy is None else D.CopyConfig(
+            tau=copy.tau, k=copy.k, max_len=copy.max_len, match_cap=copy.match_cap, table=32,
+            reserve=copy.reserve)
+        t0 = time.perf_counter()
+        self.model = LoopedModel(cfg, weights, self.n_slots)
+        self.rows = D.OracleRows(self.model)
+        tags = D.readout_depths(cfg.R, dec.d1, dec.d2)
+        zs = D.prefill(self.rows, self.prompt, cfg.R, tags)
+        self.first = D.first_token(zs[(n_prompt - 1, cfg.R)], n_prompt, dec.temperature,
+                                   dec.top_p, dec.seed)
+        self.snap = {k: (K.copy(), V.copy()) for k, (K, V) in self.model.caches.items()}
+        self.prefill_s = time.perf_counter() - t0
+
+    def run(self):
+        """One timed sample: decode seconds."""
+        for k, (K, V) in self.snap.items():
+            Kc, Vc = self.model.cache(*k)
+            Kc[:] = K
+            Vc[:] = V
+        for k in list(self.model.caches):
+            if k not in self.snap:
+                del self.model.caches[k]
+        D, cfg, dec = self.D, self.cfg, self.dec
+        t1 = time.perf_counter()
+        D.SpecDecoder(self.rows, self.prompt, cfg.R, dec.d1, dec.d2, self.n_tokens,
+                      dec.temperature, dec.top_p, dec.seed, self.n_slots, keep_trace=False,
+                      skip_prefill=True, first=self.first, copy=self.cp).run()
+        return time.perf_counter() - t1
+
+    def describe(self, decode_s):
+        return (f"{self.cfg.name}: prompt truncated to {self.n_prompt} tokens (prefilled once, "
+                f"{self.prefill_s:.1f} s, untimed), {self.n_tokens} greedy pipelined speculative "
+                f"decode tokens per sample (d1={self.dec.d1}, d2={self.dec.d2}), decode "
+                f"{decode_s:.1f} s timed, fp64 on {os.cpu_count()} host threads")
+
+
+def oracle_baseline(cfg, dec, prompt, weights, model, copy=None):
+    n_prompt, n_tokens = ORACLE_SAMPLE[model]
+    o = OracleSample(cfg, dec, prompt, weights, n_prompt, n_tokens, copy)
+    t = o.run()
+    return {"value": n_tokens / t, "unit": "tokens/s", "cores": os.cpu_count(), "kind": "oracle",
+            "sample": o.describe(t)}
 
 
 def run_reference(args):
     import synthetic as syn
-    rank, _, ws = int(os.environ.get("RANK", "0")), 0, int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
     cfg = syn.MODELS[args.model]
     dec = syn.DECODES[f"{args.model}_greedy"]
     prompt = syn.prompt_for(args.model)
-    w = syn.make_weights(cfg)
-    for _ in range(args.warmup if args.warmup < 1 else 0):
-        pass
-    vals, last = [], None
-    for _ in range(max(1, args.steps)):
-        last = oracle_sample(cfg, dec, prompt, w, n_tokens=2)
-        vals.append(last["value"])
-    v = sum(vals) / len(vals)
+    n_prompt, n_tokens = REFERENCE_SAMPLE[args.model]
+    o = OracleSample(cfg, dec, prompt, syn.make_weights(cfg), n_prompt, n_tokens)
+    for _ in range(args.warmup):
+        o.run()
+    times = [o.run() for _ in range(max(1, args.steps))]
+    v = n_tokens * len(times) / sum(times)
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": 2000.0 / v, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": WORKLOAD if args.model == "ouro14" else args.model,
+            "ms_per_step": 1000.0 * sum(times) / len(times), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOADS.get(args.model, args.model),
                        "l2": "weights larger than L2"},
-            "cpu_baseline": dict(last, value=v),
+            "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": os.cpu_count(),
+                             "kind": "oracle", "sample": o.describe(sum(times))},
             "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line))
 
 
 METRIC = "decoded tokens/s at batch 1 (greedy, T=1) + step HBM GB/s vs 8 TB/s"
-WORKLOAD = ("ouro14: Ouro-1.4B-shaped looped LM (bf16, 24 shared layers x R=4, d2048, 16x128, "
-            "ffn5632, V49152), 512-token Zipf(1.1) prompt, 1024 decode tokens, proposals at "
-            "depths 1 and 2, batch 1")
+WORKLOADS = {
+    "huginn35": ("huginn35: Huginn/Raven-3.5B-shaped looped LM (bf16, prelude 2 + core 4 x R=32 "
+                 "+ coda 2 layers, d5280, 55x96, ffn17920, V65536), 256-token Zipf(1.1) prompt, "
+                 "512 decode tokens, proposals at depths 8 and 16, batch 1"),
+    "ouro14": ("ouro14: Ouro-1.4B-shaped looped LM (bf16, 24 shared layers x R=4, d2048, 16x128, "
+               "ffn5632, V49152), 512-token Zipf(1.1) prompt, 1024 decode tokens, proposals at "
+               "depths 1 and 2, batch 1"),
+    "ouro26": ("ouro26: Ouro-2.6B-shaped looped LM (bf16, 48 shared layers x R=4, d2048, 16x128, "
+               "ffn5632, V49152), 4096-token Zipf(1.1) prompt with 40% copied 16-64-token spans, "
+               "2048 decode tokens, proposals at depths 1 and 2, batch 1"),
+    "tiny": ("tiny: looped LM (fp32, prelude 1 + shared 2 x R=4 + coda 1, d128, 4x32, ffn384, "
+             "V512), 32-token uniform prompt, 64 decode tokens, proposals at depths 2 and 3"),
+}
 
 
 # ---------------------------------------------------------------------------
@@ -332,8 +383,8 @@ def run_ours(args):
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu:
-        cpu = oracle_sample(cfg, dec_g, prompt, weights, n_prompt=8, n_tokens=24,
-                            copy=cc if copy_on else None)
+        cpu = oracle_baseline(cfg, dec_g, prompt, weights, args.model,
+                              copy=cc if copy_on else None)
 
     if rank == 0:
         n_steps = stats["steps"]
@@ -342,9 +393,10 @@ def run_ours(args):
             "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": total_ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": WORKLOAD if args.model == "ouro14" else args.model,
+            "config": {"workload": WORKLOADS.get(args.model, args.model),
                        "parallelism": f"replicas x{ws}",
-                       "l2": "no flush: 2.47 GB of weights per pass exceed the 126 MB L2",
+                       "l2": ("no flush: the shared block's weights (%.2f GB per pass) exceed the "
+                              "126 MB L2" % (info["weight_bytes_core"] / 1e9)),
                        "resid_scale": cfg.resid_scale, "agreement_d1_vs_R": agree,
                        "max_branches": 32 if copy_on else C, "n_new": n_new, "prompt_len": P},
             "speedup_vs_full_depth_ar": (ar_ms / times[-1]),
@@ -403,7 +455,8 @@ def main():
     ap.add_argument("--steps", type=int, default=3)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--model", default="ouro14")
+    ap.add_argument("--model", default="huginn35", choices=sorted(WORKLOADS),
+                    help="workload (default: the largest single-GPU configuration)")
     ap.add_argument("--n-new", type=int, default=None,
                     help="decode tokens (default: the model's configured count)")
     ap.add_argument("--no-cpu", action="store_true")

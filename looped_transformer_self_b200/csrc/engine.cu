@@ -827,7 +827,10 @@ extern "C" int lt_create(const lt_model_config* m, const lt_decode_config* dc, v
     delete hd;
     return LT_ERR_SHAPE;
   }
-  if (cudaMemsetAsync(H->attn_cnt, 0, (size_t)H->C * m->n_heads * 4, H->stream) != cudaSuccess) {
+  // the control block (error word, counters) starts zeroed: calls that run
+  // before the first prefill (lt_block_pass) read its error word
+  if (cudaMemsetAsync(H->D.ctl, 0, sizeof(Ctl), H->stream) != cudaSuccess ||
+      cudaMemsetAsync(H->attn_cnt, 0, (size_t)H->C * m->n_heads * 4, H->stream) != cudaSuccess) {
     delete hd;
     return LT_ERR_CUDA;
   }

@@ -60,7 +60,9 @@ def _fill(g, cfg, depth, nslots):
 
 def _pass(cfg, w, depth, lens, lists, offs, nslots, max_ctx, hid0):
     from looped_transformer_self_b200.binding import Decoder
-    g = Decoder(cfg, syn.DecodeConfig(1, 2, 0.0, 1.0, 2, 4), w, max_branches=8, max_ctx=max_ctx)
+    # workspace of NaN / -1 bytes: nothing may be read before it is written
+    g = Decoder(cfg, syn.DecodeConfig(1, 2, 0.0, 1.0, 2, 4), w, max_branches=8, max_ctx=max_ctx,
+                workspace_fill=0xFF)
     kvs = _fill(g, cfg, depth, nslots)
     hid = torch.from_numpy(hid0).cuda()
     g.block_pass(depth, lens, torch.from_numpy(lists).cuda(), offs, hid)
