@@ -21,7 +21,6 @@
 #include "decide.cuh"
 #include "gemm.cuh"
 #include "layers.cuh"
-#include "pass.cuh"
 
 namespace lt {
 
@@ -67,16 +66,6 @@ struct Handle {
   int P = 0;
   cudaGraphExec_t graph = nullptr;
   bool use_pdl = true, use_graph = true;
-  // persistent pass kernel for the shared block of decode steps (bf16)
-  bool pass_ok = false, use_pass = false;
-  float* part_g[4] = {nullptr, nullptr, nullptr, nullptr};  // partials of QKV, O, gate/up, down
-  void* Xm = nullptr;            // gate/up operand rows (the O epilogue's output)
-  GemmOperand tm_Xm;
-  PassLayer* pass_layers = nullptr;
-  unsigned* pass_ctr = nullptr;
-  size_t pass_ctr_n = 0;
-  int* need_qkv = nullptr;
-  PassParams pp = {};
   int kernels_per_step = 0;  // launches counted while capturing the step graph
   bool counting = false;
   // profiling: events around GEMMs and attention of un-graphed steps
@@ -233,20 +222,6 @@ static size_t carve(Handle* H, char* base) {
     part_floats = std::max(part_floats, gemm_part_bytes(*shapes[k], C) / sizeof(float));
   }
   H->part = cv.take<float>(part_floats);
-  if (H->pass_ok) {
-    H->part_g[0] = H->part;
-    for (int k = 1; k < 4; ++k) H->part_g[k] = cv.take<float>(gemm_part_bytes(*shapes[k], C) / sizeof(float));
-    H->Xm = cv.take<char>((size_t)C * d * esz);
-    H->pass_layers = cv.take<PassLayer>(m.n_core);
-    H->need_qkv = cv.take<int>(H->sh_qkv.tiles);
-    PassParams tmp = {};
-    tmp.groups[PG_QKV] = H->sh_qkv.tiles;
-    tmp.groups[PG_O] = H->sh_o.tiles;
-    tmp.groups[PG_GU] = f / 128;
-    tmp.groups[PG_D] = H->sh_d.tiles;
-    H->pass_ctr_n = pass_ctr_layout(&tmp, m.n_core, m.n_heads);
-    H->pass_ctr = cv.take<unsigned>(H->pass_ctr_n);
-  }
   H->h = cv.take<float>((size_t)C * d);
   H->hc = cv.take<float>((size_t)C * d);
   H->q = cv.take<float>((size_t)C * d);
@@ -308,7 +283,6 @@ static void plan(Handle* H) {
   for (int l = 0; l < m.n_core; ++l) H->plane_base.push_back(planes), planes += m.R;
   for (int l = 0; l < m.n_coda; ++l) H->plane_base.push_back(planes), planes += n;
   H->planes = planes;
-  H->pass_ok = !H->f32 && m.n_core > 0 && pass_supported(H->C, m.head_dim);
   Dev& D = H->D;
   D.d = m.d_model;
   D.V = m.vocab;
@@ -545,104 +519,6 @@ static cudaError_t run_readout(Handle* H, const int* flag, bool fused) {
                 (const float*)D.cb_val, (const int*)D.cb_idx, &D.ctl->err);
 }
 
-// Arguments of the persistent pass kernel (after the weights are loaded).
-static cudaError_t setup_pass(Handle* H) {
-  const lt_model_config& m = H->m;
-  Dev& D = H->D;
-  const int n = m.n_core, d = m.d_model, f = m.ffn;
-  std::vector<PassLayer> pl(n);
-  for (int l = 0; l < n; ++l) {
-    const LayerW& L = H->layers[m.n_prelude + l];
-    pl[l].w[PG_QKV] = L.tm_qkv;
-    pl[l].w[PG_O] = L.tm_o;
-    pl[l].w[PG_GU] = L.tm_gu;
-    pl[l].w[PG_D] = L.tm_d;
-    pl[l].g2 = L.g2;
-    pl[l].g_next = l + 1 < n ? H->layers[m.n_prelude + l + 1].g1 : nullptr;
-    pl[l].plane_base = H->plane_base[m.n_prelude + l];
-  }
-  cudaError_t e = cudaMemcpy(H->pass_layers, pl.data(), n * sizeof(PassLayer), cudaMemcpyHostToDevice);
-  if (e != cudaSuccess) return e;
-  PassParams& p = H->pp;
-  p = PassParams{};
-  p.x[PG_QKV] = H->tm_Xd;
-  p.x[PG_O] = H->tm_Xo;
-  p.x[PG_GU] = H->tm_Xm;
-  p.x[PG_D] = H->tm_Xf;
-  p.layers = H->pass_layers;
-  p.n_layers = n;
-  p.stages = pass_stages(H->C, H->sh_qkv.kc);
-  const char* pf = getenv("LT_PASS_L2_AHEAD");
-  p.l2_ahead = pf ? std::max(0, atoi(pf)) : 8;
-  p.sh[PG_QKV] = H->sh_qkv;
-  p.sh[PG_O] = H->sh_o;
-  p.sh[PG_GU] = H->sh_gu;
-  p.sh[PG_D] = H->sh_d;
-  for (int k = 0; k < 4; ++k) p.part[k] = H->part_g[k];
-  p.need[PG_QKV] = H->need_qkv;
-  p.need[PG_O] = H->need_o;
-  p.need[PG_GU] = H->need_gu;
-  p.need[PG_D] = H->need_d;
-  p.ctr = H->pass_ctr;
-  p.groups[PG_QKV] = H->sh_qkv.tiles;
-  p.groups[PG_O] = H->sh_o.tiles;
-  p.groups[PG_GU] = f / 128;
-  p.groups[PG_D] = H->sh_d.tiles;
-  pass_ctr_layout(&p, n, m.n_heads);
-  GemmEpi eo = {}, egu = {}, ed = {};
-  eo.kind = ed.kind = EPI_RESID;
-  eo.need = H->need_o;
-  ed.need = H->need_d;
-  eo.mask = ed.mask = egu.mask = D.m_alive;
-  eo.h = ed.h = H->h;
-  eo.scale = ed.scale = m.resid_scale;
-  eo.X = H->Xm;  // O: h += s * o W_o^T; Xm = g2 (.) h for the gate/up GEMM
-  ed.X = H->Xd;  // down: Xd = (next layer's g1) (.) h for the next QKV GEMM
-  eo.ssq_out = ed.ssq_out = H->ssq;
-  eo.d = ed.d = d;
-  egu.kind = EPI_SWIGLU;
-  egu.need = H->need_gu;
-  egu.ssq_in = H->ssq;
-  egu.ssq_tiles = H->ssq_tiles;
-  egu.eps = m.rms_eps;
-  egu.ffn = f;
-  egu.d = d;
-  egu.X = H->Xf;
-  p.epi[PG_O] = eo;
-  p.epi[PG_GU] = egu;
-  p.epi[PG_D] = ed;
-  p.att = attn_args(H, m.n_prelude, D.r_depth, -1, H->Xo);
-  p.att.part = H->part_g[PG_QKV];
-  p.mask = D.m_alive;
-  p.run_flag = &D.ctl->flag_run;
-  p.err = &D.ctl->err;
-  p.C = H->C;
-  p.H = m.n_heads;
-  p.d = d;
-  p.ffn = f;
-  return cudaSuccess;
-}
-
-// The shared block of a decode pass as one persistent kernel: stage layer 0's
-// operand rows, zero the pass counters, launch.
-template <typename T>
-static cudaError_t run_pass(Handle* H) {
-  Dev& D = H->D;
-  const lt_model_config& m = H->m;
-  const int C = H->C, d = m.d_model;
-  const LayerW& L0 = H->layers[m.n_prelude];
-  LT_CK(launch(H->use_pdl, k_stage_norm<T>, dim3(C), dim3(EPI_THREADS), H->stream,
-               (const float*)H->h, (const int*)D.m_alive, (const T*)L0.g1, d, C, (T*)H->Xd,
-               H->lo_d, H->ssq));
-  LT_CK(cudaMemsetAsync(H->pass_ctr, 0, H->pass_ctr_n * sizeof(unsigned), H->stream));
-  double bytes = 0;
-  for (const GemmShape* s : {&H->sh_qkv, &H->sh_o, &H->sh_gu, &H->sh_d})
-    bytes += 2.0 * ((double)s->n_out * s->k + (double)C * s->k) + 4.0 * C * s->n_out;
-  ProfScope ps(H, 0, bytes * m.n_core, 1);
-  if (H->counting) H->kernels_per_step++;
-  return pass_launch(H->pp, C, m.head_dim, H->stream);
-}
-
 template <typename T>
 static cudaError_t decode_step(Handle* H) {
   Dev& D = H->D;
@@ -660,11 +536,8 @@ static cudaError_t decode_step(Handle* H) {
   if (m.n_prelude > 0)
     LT_CK(run_layers<T>(H, 0, m.n_prelude, 0, D.m_new, H->h, 1.f, &ctl->flag_new, fused));
   H->prof_cat = 0;
-  if (H->use_pass)
-    LT_CK(run_pass<T>(H));
-  else
-    LT_CK(run_layers<T>(H, m.n_prelude, m.n_core, 1, D.m_alive, H->h, m.resid_scale,
-                        &ctl->flag_run, fused));
+  LT_CK(run_layers<T>(H, m.n_prelude, m.n_core, 1, D.m_alive, H->h, m.resid_scale,
+                      &ctl->flag_run, fused));
   H->prof_cat = 1;
   LT_CK(run_readout<T>(H, &ctl->flag_ro, fused));
   LT_CK(launch(H->use_pdl, k_decide, dim3(C), dim3(1024), H->stream, D));
@@ -750,8 +623,6 @@ extern "C" int lt_create(const lt_model_config* m, const lt_decode_config* dc, v
   const char* e2 = getenv("LT_NO_GRAPH");
   H->use_pdl = !(e1 && e1[0] == '1');
   H->use_graph = !(e2 && e2[0] == '1');
-  const char* e3 = getenv("LT_PASS");
-  H->use_pass = H->pass_ok && e3 && e3[0] == '1' && dc->copy_k == 0;  // the pass kernel is fused
   // reducer tables of the five GEMM shapes
   const int gc = sm_count();
   const int d = m->d_model, f = m->ffn, V = m->vocab;
@@ -804,15 +675,6 @@ extern "C" int lt_create(const lt_model_config* m, const lt_decode_config* dc, v
       delete hd;
       return LT_ERR_CUDA;
     }
-    if (H->pass_ok) {
-      std::vector<int> need_qkv(H->sh_qkv.tiles);
-      gemm_group_need(H->sh_qkv, tab.data() + offs[0], 0, need_qkv.data());
-      if (cudaMemcpy(H->need_qkv, need_qkv.data(), need_qkv.size() * 4, cudaMemcpyHostToDevice) ||
-          cudaMemset(H->Xm, 0, (size_t)H->C * d * esz)) {
-        delete hd;
-        return LT_ERR_CUDA;
-      }
-    }
   }
   // activation tensor maps (B operands)
   const size_t esz = H->f32 ? 4 : 2;
@@ -822,8 +684,7 @@ extern "C" int lt_create(const lt_model_config* m, const lt_decode_config* dc, v
       make_operand(&H->tm_Xf, H->Xf, H->f32, H->C, f, H->C, kc) ||
       make_operand(&H->tm_Xd_lo, (char*)H->Xd + H->lo_d * esz, H->f32, H->C, d, H->C, kc) ||
       make_operand(&H->tm_Xo_lo, (char*)H->Xo + H->lo_d * esz, H->f32, H->C, d, H->C, kc) ||
-      make_operand(&H->tm_Xf_lo, (char*)H->Xf + H->lo_f * esz, H->f32, H->C, f, H->C, kc) ||
-      (H->pass_ok && make_operand(&H->tm_Xm, H->Xm, false, H->C, d, H->C, kc))) {
+      make_operand(&H->tm_Xf_lo, (char*)H->Xf + H->lo_f * esz, H->f32, H->C, f, H->C, kc)) {
     delete hd;
     return LT_ERR_SHAPE;
   }
@@ -893,7 +754,6 @@ extern "C" int lt_load_weights(lt_handle* hd, const void* d_embed, const void* d
   if (maps(d_head, m.vocab, d, &H->tm_head, &H->tm_head_lo))
     return fail(hd, LT_ERR_SHAPE, "head tensor map");
   if (cudaStreamSynchronize(H->stream) != cudaSuccess) return fail(hd, LT_ERR_CUDA, "weight split");
-  if (H->pass_ok && setup_pass(H) != cudaSuccess) return fail(hd, LT_ERR_CUDA, "pass tables");
   H->embed = d_embed;
   H->final_norm = d_final_norm;
   H->head = d_head;
