@@ -348,11 +348,16 @@ def run_ours(args):
     e1.synchronize()
     sample_ms = e0.elapsed_time(e1)
 
-    # live roofline of the dominant kernel: CUDA events around every GEMM of
+    # per-step breakdown: CUDA events around every GEMM and attention launch of
     # 64 un-graphed decode steps (on the decoder's stream)
     g.prefill(prompt)
     prof = g.profile(64)
     info = g.info()
+    # live roofline of the dominant kernel in its graphed regime: one pass's
+    # shared-block GEMMs captured alone as a graph (programmatic dependent
+    # launch between them, as in the step), replayed with CUDA events around
+    # the replays on the decoder's stream (resets the decode state)
+    pg = g.profile_gemms(20)
 
     # end to end through the public API: host prompt in, host tokens out
     t0 = time.perf_counter()
@@ -363,7 +368,8 @@ def run_ours(args):
 
     peaks = _peaks()
     hbm = peaks["hbm_gbs"] if peaks else 6650.0
-    gemm_gbs = prof["gemm_core_bytes"] / (prof["gemm_core_ms"] / 1e3) / 1e9
+    gemm_gbs = pg["bytes"] / (pg["ms"] / 1e3) / 1e9
+    gemm_gbs_ungraphed = prof["gemm_core_bytes"] / (prof["gemm_core_ms"] / 1e3) / 1e9
     # algorithmic bytes of an average step (shared-block weights, prelude / coda /
     # LM-head weights on the steps that run them, KV reads and writes), over the
     # graphed step time of the timed decode
@@ -375,11 +381,20 @@ def run_ours(args):
     traffic, traffic_note = None, "no capture"
     tf = os.path.join(ROOT, "profiles", "gemm_traffic.json")
     if os.path.exists(tf):
+        from looped_transformer_self_b200.gemm_traffic import source_hash
         cap = json.load(open(tf))
-        if cap.get("source_sha256") == gemm_source_hash():
-            traffic, traffic_note = cap.get("traffic_per_launch"), "capture matches the GEMM sources"
-        else:
+        if cap.get("source_sha256") != source_hash():
             traffic_note = "GEMM sources changed since the capture"
+        elif cap.get("model") != args.model:
+            traffic_note = f"the capture covers the {cap.get('model')} shapes"
+        else:
+            # the capture's traffic / algorithmic ratio over the four shared-block
+            # shapes, applied to this run's algorithmic bytes per launch
+            ratio = cap["traffic_per_launch"] / cap["algorithmic_per_launch"]
+            traffic = ratio * pg["bytes"] / pg["launches"]
+            traffic_note = ("ncu dram bytes read + written of the four shared-block GEMM shapes "
+                            f"(profiles/gemm_traffic.json, ratio to algorithmic {ratio:.4f}); "
+                            "the GEMM sources match the capture")
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu:
@@ -415,8 +430,14 @@ def run_ours(args):
                          "achieved": gemm_gbs, "peak": hbm, "unit": "GB/s",
                          "frac": gemm_gbs / hbm, "traffic": traffic,
                          "traffic_note": traffic_note,
-                         "peak_source": "measured" if peaks else "fallback",
-                         "launches_profiled": prof["gemm_core_launches"]},
+                         "peak_source": ("measured (burst copy, MEASURED_PEAKS.json)" if peaks
+                                         else "fallback"),
+                         "timing": ("one decode pass's %d shared-block GEMM launches captured "
+                                    "alone as a CUDA graph, 20 replays, CUDA events on the "
+                                    "decoder's stream: %.3f ms per replay" % (pg["launches"], pg["ms"])),
+                         "algorithmic_bytes_per_launch": pg["bytes"] / pg["launches"],
+                         "avg_launch_us": 1e3 * pg["ms"] / pg["launches"],
+                         "ungraphed_gbs": gemm_gbs_ungraphed},
             "cpu_baseline": cpu,
             "e2e": {"value": n_new / e2e_s, "unit": "tokens/s",
                     "h2d_bytes_per_step": 4 * P, "d2h_bytes_per_step": 4 * (n_new + 1),
@@ -431,16 +452,6 @@ def run_ours(args):
     if ws > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
-
-
-def gemm_source_hash():
-    """sha256 over the sources that make up k_gemm (a traffic capture records
-    the value it measured)."""
-    import hashlib
-    h = hashlib.sha256()
-    for f in ("gemm.cu", "gemm.cuh", "gemm_epi.cuh", "tc.cuh", "common.cuh"):
-        h.update(open(os.path.join(ROOT, "looped_transformer_self_b200", "csrc", f), "rb").read())
-    return h.hexdigest()
 
 
 def _gamma(st, d1, d2, R):

@@ -226,6 +226,22 @@ typedef struct {
   double weight_bytes_core; /* one pass of the shared block's GEMM weights */
 } lt_profile;
 int lt_profile_steps(lt_handle* h, int ar_mode, int n_steps, lt_profile* out);
+/*
+ * In-graph timing of the weight-streaming GEMM: the shared-block GEMMs of one
+ * decode pass (per layer QKV, O + residual, gate/up + SwiGLU, down + residual;
+ * LoopSpec page sections 1 and 2.2: the one batched pass of the shared block's
+ * weights per step) are captured alone in a CUDA graph, in the decode step's
+ * order and launch configuration (programmatic dependent launch between them),
+ * over the rows of the handle's last step, and replayed n_iters times with
+ * CUDA events on the handle's stream around the replays.  Attention and the
+ * other kernels of a step are left out, so the GEMMs run back to back.
+ * h_out (host, 3 doubles): [0] ms per replay, [1] algorithmic bytes per replay
+ * (weights, activation rows, fp32 results), [2] GEMM launches per replay.
+ * The epilogues overwrite the hidden states: the decode state is reset
+ * (prefill again).  Synchronises the stream.  Errors: LT_ERR_ARG, LT_ERR_STATE
+ * (weights not loaded), LT_ERR_CUDA, LT_ERR_DEVICE_CHECK.
+ */
+int lt_profile_gemms(lt_handle* h, int n_iters, double* h_out);
 
 /* Static facts of a handle (captures the step graph if not done yet). */
 typedef struct {

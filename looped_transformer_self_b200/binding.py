@@ -132,6 +132,7 @@ def _declare(L):
     L.lt_rollback_branch.argtypes = [_vp, ctypes.c_int32]
     L.lt_commit_branch.argtypes = [_vp, ctypes.c_int32]
     L.lt_profile_steps.argtypes = [_vp, _i, _i, ctypes.POINTER(ProfileC)]
+    L.lt_profile_gemms.argtypes = [_vp, _i, ctypes.POINTER(ctypes.c_double)]
     L.lt_get_info.argtypes = [_vp, ctypes.POINTER(InfoC)]
     L.lt_reset.argtypes = [_vp]
     L.lt_last_error.argtypes = [_vp]
@@ -433,6 +434,13 @@ class Decoder:
         self._check(lib().lt_profile_steps(self.h, 1 if ar else 0, n_steps, ctypes.byref(p)),
                     "lt_profile_steps")
         return p.as_dict()
+
+    def profile_gemms(self, n_iters=20):
+        """lt_profile_gemms: the pass's shared-block GEMMs replayed alone as a
+        graph; resets the decode state."""
+        out = (ctypes.c_double * 3)()
+        self._check(lib().lt_profile_gemms(self.h, n_iters, out), "lt_profile_gemms")
+        return {"ms": out[0], "bytes": out[1], "launches": int(out[2])}
 
     def info(self):
         i = InfoC()

@@ -1194,6 +1194,97 @@ extern "C" int lt_profile_steps(lt_handle* hd, int ar_mode, int n_steps, lt_prof
   return rc;
 }
 
+// The shared-block GEMMs of one decode pass alone (QKV, O + residual,
+// gate/up + SwiGLU, down + residual per layer), in the step's order and launch
+// configuration, over the rows of the last step.
+template <typename T>
+static cudaError_t run_gemms_only(Handle* H) {
+  Dev& D = H->D;
+  const lt_model_config& m = H->m;
+  GemmEpi eo = {}, egu = {}, ed = {};
+  eo.kind = ed.kind = EPI_RESID;
+  eo.counters = H->cnt_o;
+  eo.need = H->need_o;
+  ed.counters = H->cnt_d;
+  ed.need = H->need_d;
+  eo.mask = ed.mask = egu.mask = D.m_alive;
+  eo.h = ed.h = H->h;
+  eo.scale = ed.scale = m.resid_scale;
+  eo.X = ed.X = H->Xd;
+  eo.lo = ed.lo = H->lo_d;
+  eo.ssq_out = ed.ssq_out = H->ssq;
+  eo.d = ed.d = egu.d = m.d_model;
+  egu.kind = EPI_SWIGLU;
+  egu.counters = H->cnt_gu;
+  egu.need = H->need_gu;
+  egu.ssq_in = H->ssq;
+  egu.ssq_tiles = H->ssq_tiles;
+  egu.eps = m.rms_eps;
+  egu.ffn = m.ffn;
+  egu.d = m.d_model;
+  egu.X = H->Xf;
+  egu.lo = H->lo_f;
+  for (int l = 0; l < m.n_core; ++l) {
+    const int gl = m.n_prelude + l;
+    const LayerW& L = H->layers[gl];
+    LT_CK(gemm<T>(H, L.tm_qkv, L.tm_qkv_lo, H->tm_Xd, H->tm_Xd_lo, H->sh_qkv, nullptr));
+    eo.g = L.g2;
+    LT_CK(gemm<T>(H, L.tm_o, L.tm_o_lo, H->tm_Xo, H->tm_Xo_lo, H->sh_o, nullptr, &eo));
+    LT_CK(gemm<T>(H, L.tm_gu, L.tm_gu_lo, H->tm_Xd, H->tm_Xd_lo, H->sh_gu, nullptr, &egu));
+    ed.g = l + 1 < m.n_core ? H->layers[gl + 1].g1 : nullptr;
+    LT_CK(gemm<T>(H, L.tm_d, L.tm_d_lo, H->tm_Xf, H->tm_Xf_lo, H->sh_d, nullptr, &ed));
+  }
+  return cudaSuccess;
+}
+
+extern "C" int lt_profile_gemms(lt_handle* hd, int n_iters, double* h_out) {
+  if (!hd || !h_out || n_iters < 1) return LT_ERR_ARG;
+  Handle* H = &hd->h;
+  if (!H->loaded) return fail(hd, LT_ERR_STATE, "weights not loaded");
+  const lt_model_config& m = H->m;
+  cudaStream_t st = H->stream;
+  double bytes = 0.0;
+  const double esz = H->f32 ? 4.0 : 2.0, split = H->mode == 2 ? 2.0 : 1.0;
+  for (const GemmShape* s : {&H->sh_qkv, &H->sh_o, &H->sh_gu, &H->sh_d})
+    bytes += split * esz * ((double)s->n_out * s->k + (double)H->C * s->k) + 4.0 * H->C * s->n_out;
+  bytes *= m.n_core;
+  cudaGraph_t g = nullptr;
+  cudaGraphExec_t ge = nullptr;
+  cudaError_t e = cudaStreamBeginCapture(st, cudaStreamCaptureModeThreadLocal);
+  if (e) return cuda_fail(hd, e, "capture");
+  cudaError_t e2 = H->f32 ? run_gemms_only<float>(H) : run_gemms_only<__nv_bfloat16>(H);
+  e = cudaStreamEndCapture(st, &g);
+  if (e2 || e || (e = cudaGraphInstantiate(&ge, g, 0))) {
+    if (g) cudaGraphDestroy(g);
+    return cuda_fail(hd, e2 ? e2 : e, "gemm graph");
+  }
+  cudaGraphDestroy(g);
+  cudaEvent_t a, b;
+  cudaEventCreate(&a);
+  cudaEventCreate(&b);
+  int rc = LT_OK;
+  // one untimed replay (first-touch of the graph), then the timed ones
+  if ((e = cudaGraphLaunch(ge, st)) || (e = cudaEventRecord(a, st))) rc = cuda_fail(hd, e, "replay");
+  for (int k = 0; k < n_iters && !rc; ++k)
+    if ((e = cudaGraphLaunch(ge, st))) rc = cuda_fail(hd, e, "replay");
+  float ms = 0.f;
+  if (!rc && ((e = cudaEventRecord(b, st)) || (e = cudaStreamSynchronize(st)) ||
+              (e = cudaEventElapsedTime(&ms, a, b))))
+    rc = cuda_fail(hd, e, "replay timing");
+  cudaEventDestroy(a);
+  cudaEventDestroy(b);
+  cudaGraphExecDestroy(ge);
+  if (rc) return rc;
+  h_out[0] = ms / n_iters;
+  h_out[1] = bytes;
+  h_out[2] = 4.0 * m.n_core;
+  // the GEMMs' epilogues overwrote the hidden states: no decode state survives
+  H->prefilled = false;
+  H->begun = false;
+  Ctl c;
+  return read_ctl(hd, &c);
+}
+
 extern "C" int lt_get_info(lt_handle* hd, lt_info* out) {
   if (!hd || !out) return LT_ERR_ARG;
   Handle* H = &hd->h;

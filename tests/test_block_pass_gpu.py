@@ -81,3 +81,29 @@ def test_block_pass_timed_replays_are_stable():
     ms = g.block_pass(depth, lens, torch.from_numpy(lists).cuda(), offs, hid, iters=5, timed=True)
     assert len(ms) == 5 and all(0 < t < 1000 for t in ms)
     assert torch.isfinite(hid).all()
+
+
+def test_profile_gemms_times_the_pass_gemms_and_resets_state():
+    """lt_profile_gemms replays one pass's shared-block GEMMs as a graph: a
+    positive time, the algorithmic bytes of 4 GEMMs per layer, and a decode
+    state that must be prefilled again."""
+    from looped_transformer_self_b200.binding import Decoder, LoopedSpecError
+    cfg = CFG
+    C = 8
+    g = Decoder(cfg, syn.DecodeConfig(1, 2, 0.0, 1.0, 2, 4), syn.make_weights(cfg), max_branches=C,
+                max_ctx=200)
+    g.prefill(syn.uniform_prompt(20, cfg.vocab, seed=2))
+    r = g.profile_gemms(3)
+    d, f = cfg.d_model, cfg.ffn
+    want = 0.0
+    for n_out, k in ((3 * d, d), (d, d), (2 * f, d), (d, f)):
+        want += 2.0 * (n_out * k + C * k) + 4.0 * C * n_out
+    assert r["launches"] == 4 * cfg.n_core
+    assert abs(r["bytes"] - want * cfg.n_core) < 1.0
+    assert 0.0 < r["ms"] < 100.0
+    with pytest.raises(LoopedSpecError):
+        g.generate(2)
+    g.prefill(syn.uniform_prompt(20, cfg.vocab, seed=2))
+    toks, _ = g.generate(4)
+    assert len(toks) == 4
+    g.close()
