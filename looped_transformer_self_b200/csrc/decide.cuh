@@ -26,6 +26,7 @@
 #include <climits>
 
 #include "readout.cuh"
+#include <cooperative_groups.h>
 
 namespace lt {
 
@@ -194,6 +195,164 @@ __global__ void __launch_bounds__(1024)
   if (threadIdx.x == 0) arg[i] = a;
   if (greedy) return;
   readout_dist(logits + (size_t)i * V, P + (size_t)i * V, V, a, T, top_p, ds);
+}
+
+// Sampled readouts on a thread-block cluster: the same processing as
+// k_readout (argmax from the chunk maxima, then softmax at T, the exact top-p
+// cut and normalisation; LoopSpec page section 2.1), with each readout row
+// spread over the RO_CL CTAs of one cluster instead of one block.  CTA rank r
+// holds the row's slice [r * S, (r + 1) * S), S = ceil(V / RO_CL), in
+// registers (thread t: elements t + k * 1024), so the row is read once.  The
+// softmax sum, the three 1024-bin levels of the radix select over the float
+// bits of p (integer 2^-40 masses) and the kept-mass sum are merged through
+// distributed shared memory after cluster barriers, every CTA adding the
+// partials in rank order: all CTAs take the same decisions, and the result
+// does not depend on scheduling.  Rows without a readout exit as a whole
+// cluster (the mask is read by every CTA), so all CTAs of a cluster meet at
+// the same barriers.
+constexpr int RO_CL = 8;          // CTAs per readout row (the portable cluster size)
+constexpr int RO_CL_MAXK = 16;    // elements per thread held in registers
+constexpr int RO_CL_MAXV = RO_CL * 1024 * RO_CL_MAXK;  // larger vocabularies use k_readout
+
+__global__ void __launch_bounds__(1024)
+    k_readout_cl(const int* __restrict__ mask, int V, float T, float top_p,
+                 const float* __restrict__ logits, float* __restrict__ P,
+                 int* __restrict__ arg, const float* __restrict__ cb_val,
+                 const int* __restrict__ cb_idx, int* err) {
+  namespace cg = cooperative_groups;
+  cg::cluster_group cluster = cg::this_cluster();
+  __shared__ float sk[33];
+  __shared__ int si[33];
+  __shared__ float red[33];
+  __shared__ unsigned long long hist[1024];
+  __shared__ unsigned long long wsum[32];
+  __shared__ float part[2];            // this CTA's softmax sum / kept-mass sum
+  __shared__ int sel[2];
+  __shared__ unsigned long long sel_above;
+  pdl_wait();
+  pdl_trigger();
+  const int i = blockIdx.y;
+  if (!mask[i]) return;  // the whole cluster (same row) returns
+  const unsigned rank = cluster.block_rank();
+  const int tid = threadIdx.x;
+  const int nch = ro_chunks(V);
+  // the row's argmax from its chunk maxima (every CTA; lowest index on ties)
+  float best = -INFINITY;
+  int bi = 0x7fffffff;
+  for (int c = tid; c < nch; c += blockDim.x) {
+    const float v = cb_val[(size_t)i * nch + c];
+    const int j = cb_idx[(size_t)i * nch + c];
+    if (better_max(v, j, best, bi)) {
+      best = v;
+      bi = j;
+    }
+  }
+  int a = block_arg<false>(best, bi, sk, si);
+  if (a < 0 || a >= V) {  // every logit was NaN
+    if (tid == 0 && rank == 0) set_err(err, DEV_BAD_INDEX);
+    a = 0;
+  }
+  if (tid == 0 && rank == 0) arg[i] = a;
+  const float* z = logits + (size_t)i * V;
+  const float zmax = z[a];
+  const float invT = 1.f / T;
+  const int S = (V + RO_CL - 1) / RO_CL;
+  const int lo = (int)rank * S, hi = min(V, lo + S);
+  float p[RO_CL_MAXK];
+  float ssum = 0.f;
+#pragma unroll
+  for (int k = 0; k < RO_CL_MAXK; ++k) {
+    const int j = lo + tid + k * 1024;
+    p[k] = 0.f;
+    if (j < hi) {
+      p[k] = expf((z[j] - zmax) * invT);
+      ssum += p[k];
+    }
+  }
+  // softmax sum: block sums, merged in rank order
+  {
+    const float b = block_sum(ssum, red);
+    if (tid == 0) part[0] = b;
+  }
+  cluster.sync();
+  float Z = 0.f;
+  for (int r = 0; r < RO_CL; ++r) Z += *cluster.map_shared_rank(&part[0], r);
+  const float invZ = 1.f / Z;
+#pragma unroll
+  for (int k = 0; k < RO_CL_MAXK; ++k) p[k] *= invZ;
+  float* out = P + (size_t)i * V;
+  if (!(top_p < 1.f)) {
+#pragma unroll
+    for (int k = 0; k < RO_CL_MAXK; ++k) {
+      const int j = lo + tid + k * 1024;
+      if (j < hi) out[j] = p[k];
+    }
+    cluster.sync();  // no CTA leaves while a peer may still read its part[]
+    return;
+  }
+  const double SCALE = 1099511627776.0;  // 2^40
+  const unsigned long long target = (unsigned long long)((double)top_p * SCALE + 0.5);
+  unsigned long long above = 0ull;
+  uint32_t prefix = 0u;
+  const int shifts[3] = {20, 10, 0};
+  bool all = false;
+  for (int lvl = 0; lvl < 3; ++lvl) {
+    hist[tid] = 0ull;
+    __syncthreads();
+    const int sh = shifts[lvl];
+#pragma unroll
+    for (int k = 0; k < RO_CL_MAXK; ++k) {
+      const int j = lo + tid + k * 1024;
+      if (j < hi) {
+        const uint32_t b = __float_as_uint(p[k]);
+        if (lvl == 0 || (b >> (sh + 10)) == prefix) {
+          const unsigned long long m = (unsigned long long)((double)p[k] * SCALE + 0.5);
+          atomicAdd(&hist[(b >> sh) & 1023u], m);
+        }
+      }
+    }
+    cluster.sync();  // every CTA's histogram of this level is complete
+    const int bin = 1023 - tid;
+    unsigned long long hv = 0ull;
+    for (int r = 0; r < RO_CL; ++r) hv += *cluster.map_shared_rank(&hist[bin], r);
+    cluster.sync();  // peers have read this CTA's histogram before it is reset
+    const unsigned long long cum = suffix_scan_1024(hv, wsum);  // mass of bins >= bin
+    if (tid == 0) sel[0] = -1;
+    __syncthreads();
+    if (above + cum >= target && above + cum - hv < target) {
+      sel[0] = bin;
+      sel_above = above + cum - hv;
+    }
+    __syncthreads();
+    if (sel[0] < 0) {
+      all = true;
+      break;
+    }
+    above = sel_above;
+    prefix = (prefix << 10) | (uint32_t)sel[0];
+    __syncthreads();
+  }
+  const uint32_t theta = all ? 0u : prefix;
+  float ks = 0.f;
+#pragma unroll
+  for (int k = 0; k < RO_CL_MAXK; ++k) {
+    const int j = lo + tid + k * 1024;
+    if (j < hi && __float_as_uint(p[k]) >= theta) ks += p[k];
+  }
+  {
+    const float b = block_sum(ks, red);
+    if (tid == 0) part[1] = b;
+  }
+  cluster.sync();
+  float Z2 = 0.f;
+  for (int r = 0; r < RO_CL; ++r) Z2 += *cluster.map_shared_rank(&part[1], r);
+  const float inv2 = 1.f / Z2;
+#pragma unroll
+  for (int k = 0; k < RO_CL_MAXK; ++k) {
+    const int j = lo + tid + k * 1024;
+    if (j < hi) out[j] = __float_as_uint(p[k]) >= theta ? p[k] * inv2 : 0.f;
+  }
+  cluster.sync();  // no CTA leaves while a peer may still read its part[]
 }
 
 // ---------------------------------------------------------------------------

@@ -514,9 +514,28 @@ static cudaError_t run_readout(Handle* H, const int* flag, bool fused) {
   LT_CK(launch(H->use_pdl, k_logits, dim3(ro_chunks(m.vocab), C), dim3(RO_THREADS), H->stream,
                (const float*)H->part, H->sh_head, C, (const int*)D.m_ro, m.vocab, D.logits,
                D.cb_val, D.cb_idx, (const float*)H->ssq, H->ssq_tiles, d, m.rms_eps));
-  return launch(H->use_pdl, k_readout, dim3(C), dim3(1024), H->stream, (const int*)D.m_ro,
-                m.vocab, D.greedy, D.T, D.top_p, D.logits, D.P, D.ro_arg,
-                (const float*)D.cb_val, (const int*)D.cb_idx, &D.ctl->err);
+  if (D.greedy || m.vocab > RO_CL_MAXV)
+    return launch(H->use_pdl, k_readout, dim3(C), dim3(1024), H->stream, (const int*)D.m_ro,
+                  m.vocab, D.greedy, D.T, D.top_p, D.logits, D.P, D.ro_arg,
+                  (const float*)D.cb_val, (const int*)D.cb_idx, &D.ctl->err);
+  // sampled readouts: one cluster of RO_CL CTAs per row
+  if (g_launch_counter) ++*g_launch_counter;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(RO_CL, C);
+  cfg.blockDim = dim3(1024);
+  cfg.stream = H->stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = RO_CL;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = H->use_pdl ? 2 : 1;
+  return cudaLaunchKernelEx(&cfg, k_readout_cl, (const int*)D.m_ro, m.vocab, D.T, D.top_p,
+                            (const float*)D.logits, D.P, D.ro_arg, (const float*)D.cb_val,
+                            (const int*)D.cb_idx, &D.ctl->err);
 }
 
 template <typename T>

@@ -342,3 +342,36 @@ def test_step_info_and_running_stats_match_oracle(tiny):
             assert st[f] == getattr(sd.stats, f), f
     assert sd.stats.n_first > 0 and sd.stats.gate_opens > 0
     g.close()
+
+
+@pytest.mark.parametrize("V,top_p", [(49152, 0.95), (65539, 0.9), (65536, 1.0)])
+def test_sampled_readout_distributions_match_oracle(V, top_p):
+    """Sampled decoding with large vocabularies (the readout runs on thread-block
+    clusters): every fresh readout row's processed distribution (softmax at T,
+    exact top-p, normalisation; LoopSpec page section 2.1) equals the oracle's
+    processing of the same logits within 2e-6, rows whose top-p cut is within
+    2e-6 of a boundary excepted."""
+    from looped_transformer_self_b200.binding import Decoder
+    from oracle import sampling as S
+    from test_depth_gpu import _ambiguous
+    cfg = syn.ModelConfig("bf16_bigv", "bf16", 256, 2, 128, 512, V, 0, 2, 0, 4,
+                          resid_scale=0.5, head_gain=4.0, seed=3)
+    dec = syn.DecodeConfig(1, 2, 1.0, top_p, 5, 6)
+    # (1, 2, 4) proposals fork up to 12 branches at once
+    g = Decoder(cfg, dec, syn.make_weights(cfg), max_branches=16, max_ctx=64)
+    g.prefill(syn.uniform_prompt(12, V, seed=4))
+    checked = 0
+    for _ in range(6):
+        g.step()
+        lg, pr, am = g.read_readouts()
+        for i in range(lg.shape[0]):
+            z = lg[i].astype(np.float64)
+            if not np.all(np.isfinite(z)) or abs(pr[i].sum() - 1.0) > 1e-3:
+                continue  # no readout in this row yet
+            assert am[i] == int(np.argmax(lg[i]))
+            if _ambiguous(z, 1.0, top_p, 2e-6):
+                continue
+            np.testing.assert_allclose(pr[i], S.process(z, 1.0, top_p), atol=2e-6, rtol=0)
+            checked += 1
+    assert checked >= 6
+    g.close()
