@@ -211,7 +211,7 @@ __global__ void __launch_bounds__(1024)
 // cluster (the mask is read by every CTA), so all CTAs of a cluster meet at
 // the same barriers.
 constexpr int RO_CL = 8;          // CTAs per readout row (the portable cluster size)
-constexpr int RO_CL_MAXK = 16;    // elements per thread held in registers
+constexpr int RO_CL_MAXK = 12;    // elements per thread held in registers (V <= 98304)
 constexpr int RO_CL_MAXV = RO_CL * 1024 * RO_CL_MAXK;  // larger vocabularies use k_readout
 
 __global__ void __launch_bounds__(1024)
@@ -224,7 +224,7 @@ __global__ void __launch_bounds__(1024)
   __shared__ float sk[33];
   __shared__ int si[33];
   __shared__ float red[33];
-  __shared__ unsigned long long hist[1024];
+  __shared__ unsigned long long hist[2][1024];  // radix levels alternate between the two
   __shared__ unsigned long long wsum[32];
   __shared__ float part[2];            // this CTA's softmax sum / kept-mass sum
   __shared__ int sel[2];
@@ -297,7 +297,7 @@ __global__ void __launch_bounds__(1024)
   const int shifts[3] = {20, 10, 0};
   bool all = false;
   for (int lvl = 0; lvl < 3; ++lvl) {
-    hist[tid] = 0ull;
+    hist[lvl & 1][tid] = 0ull;
     __syncthreads();
     const int sh = shifts[lvl];
 #pragma unroll
@@ -307,15 +307,16 @@ __global__ void __launch_bounds__(1024)
         const uint32_t b = __float_as_uint(p[k]);
         if (lvl == 0 || (b >> (sh + 10)) == prefix) {
           const unsigned long long m = (unsigned long long)((double)p[k] * SCALE + 0.5);
-          atomicAdd(&hist[(b >> sh) & 1023u], m);
+          atomicAdd(&hist[lvl & 1][(b >> sh) & 1023u], m);
         }
       }
     }
     cluster.sync();  // every CTA's histogram of this level is complete
     const int bin = 1023 - tid;
     unsigned long long hv = 0ull;
-    for (int r = 0; r < RO_CL; ++r) hv += *cluster.map_shared_rank(&hist[bin], r);
-    cluster.sync();  // peers have read this CTA's histogram before it is reset
+    for (int r = 0; r < RO_CL; ++r) hv += *cluster.map_shared_rank(&hist[lvl & 1][bin], r);
+    // (a histogram buffer is reset two levels later, after the next level's
+    // barrier, which every CTA passes only after these reads)
     const unsigned long long cum = suffix_scan_1024(hv, wsum);  // mass of bins >= bin
     if (tid == 0) sel[0] = -1;
     __syncthreads();
@@ -610,6 +611,243 @@ __global__ void __launch_bounds__(1024) k_decide(Dev D) {
     D.v_src[i] = src;
     D.v_fb[i] = fb;
   }
+}
+
+// The sampled path of k_decide on a thread-block cluster of RO_CL CTAs per
+// readout row (greedy decoding keeps k_decide: it needs only the argmax).  CTA
+// rank r owns the slice [r * S, (r + 1) * S) of every V-long vector of the row
+// (q1, q2, the residuals) and only ever touches that slice, so no CTA reads
+// another's global writes; sums merge in rank order through distributed shared
+// memory, and an exponential race takes each CTA's (key, index) winner and the
+// smallest key over the cluster (lowest index on ties) -- the same token a
+// race over the whole row picks.  A residual's value at one index is recomputed
+// from its definition where a decision needs it.  Every decision comes from
+// cluster-wide values, so all CTAs of a row take the same branches and meet at
+// the same cluster barriers; scalar state is written by rank 0 only.
+__global__ void __launch_bounds__(1024) k_decide_cl(Dev D) {
+  namespace cg = cooperative_groups;
+  cg::cluster_group cluster = cg::this_cluster();
+  __shared__ float sk[33];
+  __shared__ int si[33];
+  __shared__ float red[33];
+  __shared__ int tail[WIN];
+  __shared__ int prop[CPMAX];
+  __shared__ float slot_f[2];  // block partials of cluster reductions (alternating)
+  __shared__ int slot_i[2];
+  pdl_wait();
+  pdl_trigger();
+  Ctl* c = D.ctl;
+  const int i = blockIdx.y;
+  // rows without a readout, and retiring entries, decide nothing (the whole cluster)
+  if (c->finished || !D.m_ro[i] || D.b_parent[i] == BK_RETIRING) return;
+  const int tid = threadIdx.x;
+  const unsigned rank = cluster.block_rank();
+  const bool lead = rank == 0 && tid == 0;
+  const int r = D.r_depth[i];
+  const int uid = D.b_uid[i];
+  const bool ar = c->ar_mode != 0;
+  const int V = D.V;
+  const int S = (V + RO_CL - 1) / RO_CL;
+  const int lo = (int)rank * S, hi = min(V, lo + S);
+  const bool copied_x1 = !ar && D.b_copy[i];
+  const bool prop1 = !ar && r == D.d1;
+  const bool prop2 = !ar && D.d2 > 0 && r == D.d2 && D.b_x1[i] >= 0 && !copied_x1;
+  const float* z = D.logits + (size_t)i * V;
+  const int a = D.ro_arg[i];
+  int nred = 0;  // cluster reductions so far: the slot of the next one
+  // a slot is written again two reductions later, after the barrier of the one
+  // in between, which every CTA passes only after reading it
+  auto csum = [&](float v) -> float {
+    const float b = block_sum(v, red);
+    const int sl = nred++ & 1;
+    if (tid == 0) slot_f[sl] = b;
+    cluster.sync();
+    float t = 0.f;
+    for (int q = 0; q < RO_CL; ++q) t += *cluster.map_shared_rank(&slot_f[sl], q);
+    return t;
+  };
+  auto crace = [&](const float* w, uint32_t stream, uint32_t purpose) -> int {
+    float best = INFINITY;
+    int bi = 0x7fffffff;
+    for (int j = lo + tid; j < hi; j += blockDim.x) {
+      const float wj = w[j];
+      if (wj > 0.f) {
+        const float k = race_key(D.seed, stream, purpose, (uint32_t)j, wj);
+        if (better_min(k, j, best, bi)) {
+          best = k;
+          bi = j;
+        }
+      }
+    }
+    const int loc = block_arg<true>(best, bi, sk, si);
+    const int sl = nred++ & 1;
+    if (tid == 0) {
+      slot_i[sl] = loc;
+      slot_f[sl] = loc < V ? race_key(D.seed, stream, purpose, (uint32_t)loc, w[loc]) : INFINITY;
+    }
+    cluster.sync();
+    float bk = INFINITY;
+    int bj = 0x7fffffff;
+    for (int q = 0; q < RO_CL; ++q) {
+      const float k2 = *cluster.map_shared_rank(&slot_f[sl], q);
+      const int j2 = *cluster.map_shared_rank(&slot_i[sl], q);
+      if (better_min(k2, j2, bk, bj)) {
+        bk = k2;
+        bj = j2;
+      }
+    }
+    return bj;
+  };
+  // softmax of the row's logits at T = 1, at token s (the copy screen's score)
+  auto cscore = [&](int s) -> float {
+    const float zmax = z[a];
+    float acc = 0.f;
+    for (int j = lo + tid; j < hi; j += blockDim.x) acc += expf(z[j] - zmax);
+    const float Z = csum(acc);
+    return expf(z[s] - zmax) / Z;
+  };
+  // out = normalised (mu - nu)_+ over this CTA's slice; returns the cluster-wide mass
+  auto cresidual = [&](const float* mu, const float* nu, float* out) -> float {
+    float zs = 0.f;
+    for (int j = lo + tid; j < hi; j += blockDim.x) {
+      const float w = fmaxf(mu[j] - nu[j], 0.f);
+      out[j] = w;
+      zs += w;
+    }
+    const float Z = csum(zs);
+    if (Z > 0.f) {
+      const float inv = 1.f / Z;
+      for (int j = lo + tid; j < hi; j += blockDim.x) out[j] *= inv;
+    }
+    return Z;
+  };
+  do {
+    // at depth d1: screen a copied x1, or propose (and look up a copy proposal)
+    bool draw1 = prop1;
+    if (prop1 && copied_x1) {
+      const bool pass = cscore(D.b_x1[i]) >= D.copy_tau;
+      if (lead) D.cp_fail[i] = !pass;
+      draw1 = !pass;
+    }
+    if (prop1 && !copied_x1 && D.copy_k > 0) {
+      int n = copy_lookup(D, i, c->L, tail, si, prop);  // the same in every CTA
+      if (n > 0 && cscore(prop[0]) < D.copy_tau) n = 0;
+      if (lead) D.cp_len[i] = n;
+      if (rank == 0)
+        for (int t = tid; t < n; t += blockDim.x) D.cp_tok[(size_t)i * CPMAX + t] = prop[t];
+    }
+    const float* p = D.P + (size_t)i * V;
+    float* q1 = D.q1 + (size_t)i * V;
+    float* q2 = D.q2 + (size_t)i * V;
+    if (draw1) {
+      for (int j = lo + tid; j < hi; j += blockDim.x) q1[j] = p[j];
+      const int x1 = crace(p, (uint32_t)uid, P_PROP1);
+      if (lead) D.b_x1[i] = x1;
+    }
+    if (prop2) {
+      const int x1 = D.b_x1[i];
+      int open = 0;
+      if (D.second_mode == 0) {  // gated residual (Eqs. 5-6)
+        if (p[x1] < q1[x1]) open = cresidual(p, q1, q2) > 0.f;
+      } else if (D.second_mode == 1) {  // residual, no gate (ablation)
+        open = cresidual(p, q1, q2) > 0.f;
+      } else {  // non-residual ablation (section 3.4): p_d2 with x1 removed, renormalised
+        float zs = 0.f;
+        for (int j = lo + tid; j < hi; j += blockDim.x) {
+          const float w = j == x1 ? 0.f : p[j];
+          q2[j] = w;
+          zs += w;
+        }
+        const float Z = csum(zs);
+        if (Z > 0.f) {
+          for (int j = lo + tid; j < hi; j += blockDim.x) q2[j] /= Z;
+          open = 1;
+        }
+      }
+      int x2 = -1;
+      if (open) x2 = crace(q2, (uint32_t)uid, P_PROP2);
+      if (lead) {
+        D.b_gate[i] = open;
+        D.b_x2[i] = x2;
+        atomicAdd(&c->gate_checks, 1);
+        atomicAdd(&c->gate_opens, open);
+      }
+    }
+    if (r != D.R) break;
+    // verification at full depth
+    int x, src = 0, fb = 0;
+    float* rho_i = D.rho + (size_t)i * V;
+    float* rho2_i = D.rho2 + (size_t)i * V;
+    if (ar) {
+      x = crace(p, (uint32_t)(D.r_pos[i] + 1), P_AR);
+    } else if (D.b_x1[i] < 0) {
+      x = crace(p, (uint32_t)uid, P_RES);
+    } else if (copied_x1) {
+      // one-hot proposal: accept with probability p(x1), else draw from p without x1
+      const int x1 = D.b_x1[i];
+      const float u1 = uniform01(D.seed, (uint32_t)uid, P_ACC1);
+      if (u1 < p[x1]) {
+        x = x1;
+        src = 1;
+      } else {
+        float zs = 0.f;
+        for (int j = lo + tid; j < hi; j += blockDim.x) {
+          const float w = j == x1 ? 0.f : p[j];
+          rho_i[j] = w;
+          zs += w;
+        }
+        const float Z = csum(zs);
+        const float* rho1 = rho_i;
+        if (Z > 0.f) {
+          const float inv = 1.f / Z;
+          for (int j = lo + tid; j < hi; j += blockDim.x) rho_i[j] *= inv;
+        } else {
+          rho1 = p;  // unreachable: p(x1) = 1 always accepts
+          fb = 1;
+        }
+        x = crace(rho1, (uint32_t)uid, P_RES);
+      }
+    } else {
+      const int x1 = D.b_x1[i];
+      const float u1 = uniform01(D.seed, (uint32_t)uid, P_ACC1);
+      if (u1 * q1[x1] < p[x1]) {
+        x = x1;
+        src = 1;
+      } else {
+        const float Z1 = cresidual(p, q1, rho_i);
+        const float* rho1 = rho_i;
+        if (!(Z1 > 0.f)) {
+          rho1 = p;  // unreachable in exact arithmetic
+          fb = 1;
+        }
+        const int x2 = D.b_x2[i];
+        if (D.b_gate[i] && x2 >= 0) {
+          // rho1 at x2, from its definition (the owning CTA stores the same value)
+          const float rho1_x2 = Z1 > 0.f ? fmaxf(p[x2] - q1[x2], 0.f) * (1.f / Z1) : p[x2];
+          const float u2 = uniform01(D.seed, (uint32_t)uid, P_ACC2);
+          if (u2 * q2[x2] < rho1_x2) {
+            x = x2;
+            src = 2;
+          } else {
+            const float* r2 = rho2_i;
+            if (!(cresidual(rho1, q2, rho2_i) > 0.f)) {
+              r2 = rho1;
+              fb += 1;
+            }
+            x = crace(r2, (uint32_t)uid, P_RES);
+          }
+        } else {
+          x = crace(rho1, (uint32_t)uid, P_RES);
+        }
+      }
+    }
+    if (lead) {
+      D.v_tok[i] = x;
+      D.v_src[i] = src;
+      D.v_fb[i] = fb;
+    }
+  } while (false);
+  cluster.sync();  // no CTA leaves while a peer may still read its shared memory
 }
 
 // First token after prefill: full-depth readout of the last prompt position,

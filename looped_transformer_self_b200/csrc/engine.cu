@@ -135,6 +135,25 @@ static cudaError_t launch(bool pdl, void (*kern)(KArgs...), dim3 grid, dim3 bloc
   return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
+// A 1024-thread kernel on clusters of RO_CL CTAs along x (one cluster per row).
+template <typename... KArgs, typename... Args>
+static cudaError_t launch_cluster(Handle* H, void (*kern)(KArgs...), dim3 grid, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(1024);
+  cfg.stream = H->stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = RO_CL;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = H->use_pdl ? 2 : 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
 // ---------------------------------------------------------------------------
 // workspace layout
 // ---------------------------------------------------------------------------
@@ -520,22 +539,9 @@ static cudaError_t run_readout(Handle* H, const int* flag, bool fused) {
                   (const float*)D.cb_val, (const int*)D.cb_idx, &D.ctl->err);
   // sampled readouts: one cluster of RO_CL CTAs per row
   if (g_launch_counter) ++*g_launch_counter;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(RO_CL, C);
-  cfg.blockDim = dim3(1024);
-  cfg.stream = H->stream;
-  cudaLaunchAttribute attr[2];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = RO_CL;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[1].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = H->use_pdl ? 2 : 1;
-  return cudaLaunchKernelEx(&cfg, k_readout_cl, (const int*)D.m_ro, m.vocab, D.T, D.top_p,
-                            (const float*)D.logits, D.P, D.ro_arg, (const float*)D.cb_val,
-                            (const int*)D.cb_idx, &D.ctl->err);
+  return launch_cluster(H, k_readout_cl, dim3(RO_CL, C), (const int*)D.m_ro, m.vocab, D.T,
+                        D.top_p, (const float*)D.logits, D.P, D.ro_arg, (const float*)D.cb_val,
+                        (const int*)D.cb_idx, &D.ctl->err);
 }
 
 template <typename T>
@@ -559,7 +565,13 @@ static cudaError_t decode_step(Handle* H) {
                       &ctl->flag_run, fused));
   H->prof_cat = 1;
   LT_CK(run_readout<T>(H, &ctl->flag_ro, fused));
-  LT_CK(launch(H->use_pdl, k_decide, dim3(C), dim3(1024), H->stream, D));
+  if (D.greedy) {
+    LT_CK(launch(H->use_pdl, k_decide, dim3(C), dim3(1024), H->stream, D));
+  } else {
+    // sampled decisions: one cluster of RO_CL CTAs per row
+    if (g_launch_counter) ++*g_launch_counter;
+    LT_CK(launch_cluster(H, k_decide_cl, dim3(RO_CL, C), D));
+  }
   return launch(H->use_pdl, k_book, dim3(1), dim3(256), H->stream, D, 0, 0);
 }
 
