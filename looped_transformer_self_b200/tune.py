@@ -45,7 +45,7 @@ def measure(cfg, dec, prompt, weights_dev, device="cuda"):
     return agree, top1
 
 
-def tune(model: str, target_top1: float = 0.3, iters: int = 10, device="cuda"):
+def tune(model: str, target_top1: float = 0.3, iters: int = 10, device="cuda", tol: float = 0.005):
     cfg = syn.MODELS[model]
     dec = syn.DECODES[f"{model}_greedy"]
     d1, target = syn.AGREEMENT_TARGET[model]
@@ -73,18 +73,26 @@ def tune(model: str, target_top1: float = 0.3, iters: int = 10, device="cuda"):
             hi_g = mid
     gain = round(0.5 * (lo_g + hi_g), 3)
     c = with_gain(gain)
-    # residual scale: agreement decreases as s grows
-    lo_s, hi_s = 0.0, 2.0
-    for _ in range(iters):
-        mid = 0.5 * (lo_s + hi_s)
+    # residual scale: agreement decreases as s grows.  The useful scales span
+    # orders of magnitude (~0.005 for Huginn-3.5B, ~0.014 for Ouro-1.4B), so
+    # the bisection runs on log s; it stops once the agreement is within tol of
+    # the target, and the evaluated scale closest to the target wins.
+    lo_s, hi_s = np.log(1e-4), np.log(2.0)
+    best = None
+    for _ in range(2 * iters):
+        mid = float(np.exp(0.5 * (lo_s + hi_s)))
+        mid = float(f"{mid:.4g}")
         a, t1 = measure(c.replace(resid_scale=mid), dec, prompt, w, device)
         log.append(("scale", gain, mid, a, t1))
+        if best is None or abs(a - target) < abs(best[1] - target):
+            best = (mid, a, t1)
+        if abs(a - target) <= tol:
+            break
         if a > target:
-            lo_s = mid
+            lo_s = np.log(mid)
         else:
-            hi_s = mid
-    s = round(0.5 * (lo_s + hi_s), 4)
-    a, t1 = measure(c.replace(resid_scale=s), dec, prompt, w, device)
+            hi_s = np.log(mid)
+    s, a, t1 = best
     return {"model": model, "head_gain": gain, "resid_scale": s, "agreement": a,
             "median_top1": t1, "target_agreement": target, "log": log}
 

@@ -97,13 +97,15 @@ MODELS: Dict[str, ModelConfig] = {
     "ouro14": ModelConfig("ouro14", "bf16", 2048, 16, 128, 5632, 49152, 0, 24, 0, 4,
                           resid_scale=0.0137, head_gain=4.942),
     # Huginn/Raven-3.5B-shaped: prelude 2, core 4 x R=32, coda 2.
-    # knobs from looped_transformer_self_b200.tune (depth-8 vs depth-32 agreement 0.668)
+    # knobs from looped_transformer_self_b200.tune (depth-8 vs depth-32 agreement 0.699,
+    # median full-depth top-1 probability 0.300)
     "huginn35": ModelConfig("huginn35", "bf16", 5280, 55, 96, 17920, 65536, 2, 4, 2, 32,
-                            resid_scale=0.0049, head_gain=4.93),
+                            resid_scale=0.004627, head_gain=5.11),
     # Ouro-2.6B-shaped: 48 shared layers x R=4.
-    # knobs from looped_transformer_self_b200.tune (depth-1 vs depth-4 agreement 0.574)
+    # knobs from looped_transformer_self_b200.tune (depth-1 vs depth-4 agreement 0.597,
+    # median full-depth top-1 probability 0.299)
     "ouro26": ModelConfig("ouro26", "bf16", 2048, 16, 128, 5632, 49152, 0, 48, 0, 4,
-                          resid_scale=0.0127, head_gain=4.717),
+                          resid_scale=0.01165, head_gain=5.301),
     # Kernel sweep: one Ouro-shaped 24-layer shared block (no readout).
     "sweep": ModelConfig("sweep", "bf16", 2048, 16, 128, 5632, 49152, 0, 24, 0, 4,
                          resid_scale=0.35, head_gain=3.5),
