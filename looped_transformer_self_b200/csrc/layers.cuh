@@ -777,7 +777,10 @@ __global__ void __launch_bounds__(128) k_attn2(const AttnArgs a, const int* __re
     pdl_wait();
     pdl_trigger();
   }
-  issue_upto(A2_NS - 1);
+  // fused: every ring stage is requested before the dependency wait (the
+  // cache rows of earlier positions were written by earlier kernels), so an
+  // item's whole 128-position split is in flight while the QKV GEMM finishes
+  issue_upto(FUSED ? A2_NS : A2_NS - 1);
   if constexpr (FUSED) {
     pdl_wait();
     pdl_trigger();
