@@ -409,11 +409,45 @@ static cudaError_t attention_items(Handle* H, int gl, const int* tagsrc, int tag
                 attn_args(H, gl, tagsrc, tag_off, (void*)Xo), mask);
 }
 
+// Long contexts: one resident wave of ring blocks, each streaming a contiguous
+// range of (head, row, split) units (k_attn3; the same bits as k_attn2).
+template <typename T, int HD>
+static cudaError_t attention_ranges(Handle* H, int gl, const int* tagsrc, int tag_off,
+                                    const int* mask, T* Xo, bool fused) {
+  auto kern = fused ? k_attn3<T, HD, true> : k_attn3<T, HD, false>;
+  const size_t smem = a3_smem_bytes<T, HD>();
+  static int per_sm[kMaxDev][2] = {};
+  int& nb = per_sm[cur_dev()][fused ? 1 : 0];
+  if (nb == 0) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess)
+      return cudaErrorInvalidValue;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kern, 128, smem) != cudaSuccess || nb < 1)
+      nb = 1;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(nb * sm_count());
+  cfg.blockDim = dim3(128);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = H->stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = H->use_pdl ? 1 : 0;
+  if (H->counting) H->kernels_per_step++;
+  return cudaLaunchKernelEx(&cfg, kern, attn_args(H, gl, tagsrc, tag_off, (void*)Xo), mask);
+}
+
 template <typename T, int HD>
 static cudaError_t attention(Handle* H, int gl, const int* tagsrc, int tag_off, const int* mask,
                              T* Xo, bool fused) {
   ProfScope ps(H, 2, 0.0);
-  if (H->dc.max_ctx > ATT_RING_MAX_CTX) return attention_items<T, HD>(H, gl, tagsrc, tag_off, mask, Xo, fused);
+  if (H->dc.max_ctx > ATT_RING_MAX_CTX) {
+    static const char* e = getenv("LT_ATT_LONG");
+    if (e && !strcmp(e, "regs")) return attention_items<T, HD>(H, gl, tagsrc, tag_off, mask, Xo, fused);
+    return attention_ranges<T, HD>(H, gl, tagsrc, tag_off, mask, Xo, fused);
+  }
   auto kern = fused ? k_attn2<T, HD, true> : k_attn2<T, HD, false>;
   // one resident wave of ring blocks (items are spread over them)
   const size_t smem = a2_smem_bytes<T, HD>();

@@ -988,6 +988,419 @@ __global__ void __launch_bounds__(128) k_attn2(const AttnArgs a, const int* __re
   }
 }
 
+// ---- long contexts: each block streams a contiguous range of splits -----------
+// The per-split arithmetic is attn_item's and k_attn2's (per half-warp the same
+// positions in the same order, the same merges), so the results are the same
+// bits.  The work assignment differs.  Units are (head, row, split) triples in
+// head, row, split order; block b of G streams units [b*U/G, (b+1)*U/G) of the
+// U units, so the blocks hold the same number of 128-position splits to within
+// one, however the rows' lengths fall.  Consecutive units of a block mostly
+// belong to one (row, head): the query is formed once per such run, and one
+// ticket per run replaces one per split.  K/V rows come through a shared-memory
+// ring NS chunks deep (cp.async), and each unit's slot list is loaded into
+// registers one unit before its first chunk is requested, so no slot-list round
+// trip sits between two chunks.
+template <typename T, int HD, int NS>
+struct A3Smem {
+  T kv[NS][2][A2_CH][HD];  // K then V rows of one chunk
+  int sl[NS][ATT_CH];      // slot lists of the units in flight
+  int rec[NS][8];          // unit records: row, split, splits, head, count, plane, chunks
+  float qsm[HD];
+  float own_k[HD], own_v[HD];  // (fused) the row's own position
+  float hm[8], hl[8];
+  float hacc[8][HD];
+  int rmask[A2_MAXC], rpos[A2_MAXC], rblen[A2_MAXC], rboff[A2_MAXC], rslot[A2_MAXC],
+      rtag[A2_MAXC];
+  int rsplit0[A2_MAXC + 1];  // prefix sums of the active rows' splits
+  float rr[A2_MAXC];         // (fused) RMSNorm factors
+  int last;
+};
+
+// ring depth: about 96 KB of K/V stages (two blocks per SM for bf16, head 128)
+template <typename T, int HD>
+constexpr int a3_stages() {
+  constexpr int stage = 2 * A2_CH * HD * (int)sizeof(T);
+  constexpr int n = (96 * 1024) / stage;
+  return n < 2 ? 2 : (n > 4 ? 4 : n);
+}
+
+template <typename T, int HD>
+constexpr size_t a3_smem_bytes() {
+  return sizeof(A3Smem<T, HD, a3_stages<T, HD>()>);
+}
+
+__device__ __forceinline__ void cp_async_wait_upto3(int pending) {
+  switch (pending) {
+    case 0: asm volatile("cp.async.wait_group 0;" ::: "memory"); break;
+    case 1: asm volatile("cp.async.wait_group 1;" ::: "memory"); break;
+    case 2: asm volatile("cp.async.wait_group 2;" ::: "memory"); break;
+    default: asm volatile("cp.async.wait_group 3;" ::: "memory"); break;
+  }
+}
+
+template <typename T, int HD, bool FUSED>
+__global__ void __launch_bounds__(128) k_attn3(const AttnArgs a, const int* __restrict__ mask) {
+  constexpr int NS = a3_stages<T, HD>();
+  static_assert(NS >= 2 && NS <= 4, "cp_async_wait_upto3 covers up to three pending chunks");
+  extern __shared__ __align__(16) unsigned char a3raw[];
+  A3Smem<T, HD, NS>& sm = *reinterpret_cast<A3Smem<T, HD, NS>*>(a3raw);
+  constexpr int EPL = HD / 16;
+  constexpr int PPR = HD * (int)sizeof(T) / 16;  // 16-byte pieces per K or V row
+  constexpr int EPP = 16 / (int)sizeof(T);       // elements per piece
+  const int tid = threadIdx.x;
+  const int H = a.H, C = a.C, S = a.S, d = a.d;
+  T* const kv = reinterpret_cast<T*>(a.kv);
+
+  // row metadata: written by kernels that finished before this grid
+  if (tid < C) {
+    const int m = mask[tid];
+    sm.rmask[tid] = m;
+    sm.rpos[tid] = a.r_pos[tid];
+    sm.rblen[tid] = a.r_blen[tid];
+    sm.rboff[tid] = a.r_boff[tid];
+    sm.rslot[tid] = a.r_slot[tid];
+    sm.rtag[tid] = a.tagsrc ? a.tagsrc[tid] : 0;
+    if constexpr (FUSED) sm.rr[tid] = m ? inv_rms_parts(a.ssq, a.ssq_tiles, C, tid, d, a.eps) : 1.f;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int acc = 0;
+    for (int r = 0; r < C; ++r) {
+      sm.rsplit0[r] = acc;
+      acc += sm.rmask[r] ? (sm.rpos[r] + ATT_CH) / ATT_CH : 0;
+    }
+    sm.rsplit0[C] = acc;
+  }
+  __syncthreads();
+  const int TS = sm.rsplit0[C];  // splits of one head
+  const long long U = (long long)H * TS;
+  const int u0 = (int)(U * blockIdx.x / gridDim.x);
+  const int nit = (int)(U * (blockIdx.x + 1) / gridDim.x) - u0;
+  if (nit <= 0) {
+    pdl_wait();
+    pdl_trigger();
+    return;
+  }
+
+  // unit k of this block: head, row, split, first position, position count
+  struct Unit {
+    int h, row, sp, start, cnt;
+  };
+  auto unit = [&](int k) {
+    Unit x;
+    const int u = u0 + k;
+    x.h = u / TS;
+    const int j = u - x.h * TS;
+    int lo = 0, hi = C - 1;  // the last row whose first split is <= j (it has splits)
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (sm.rsplit0[mid] <= j)
+        lo = mid;
+      else
+        hi = mid - 1;
+    }
+    x.row = lo;
+    x.sp = j - sm.rsplit0[lo];
+    x.start = x.sp * ATT_CH;
+    x.cnt = min(ATT_CH, sm.rpos[lo] + 1 - x.start);
+    return x;
+  };
+  // this thread's slot of unit x (position start + tid); the load is not waited on here
+  auto slot_load = [&](Unit x) {
+    if (tid >= x.cnt) return 0;
+    const int jj = x.start + tid;
+    return jj < sm.rblen[x.row] ? a.lists[sm.rboff[x.row] + jj]
+                                : a.chain[x.row * a.W + (jj % a.W)];
+  };
+
+  // issue side: unit ki (record written when ji == 0), its chunk ji, chunk count ci
+  int ki = 0, ji = 0, ci = 0, cc = 0;
+  Unit xi = unit(0);
+  int nslot = slot_load(xi);  // slot of unit ki for this thread
+  auto issue_upto = [&](int upto) {
+    while (ci < upto && ki < nit) {
+      const int q = ki % NS;
+      if (ji == 0) {
+        if (tid < xi.cnt) {
+          int s = nslot;
+          if (s < 0 || s >= S) {
+            set_err(a.err, DEV_BAD_INDEX);
+            s = 0;
+          }
+          sm.sl[q][tid] = s;
+        }
+        if (tid == 0) {
+          int* r = sm.rec[q];
+          r[0] = xi.row;
+          r[1] = xi.sp;
+          r[2] = (sm.rpos[xi.row] + ATT_CH) / ATT_CH;
+          r[3] = xi.h;
+          r[4] = xi.cnt;
+          r[5] = a.plane_base + sm.rtag[xi.row] + a.tag_off;
+          r[6] = (xi.cnt + A2_CH - 1) / A2_CH;
+        }
+        if (ki + 1 < nit) {  // the next unit's slot list starts on its way now
+          xi = unit(ki + 1);
+          nslot = slot_load(xi);
+        }
+        __syncthreads();  // slot list and record visible
+      }
+      // the cp.async copies of chunk ji of unit ki into ring stage ci % NS
+      const int st = ci % NS;
+      const int h = sm.rec[q][3], cnt = sm.rec[q][4], plane = sm.rec[q][5];
+      const int p0 = ji * A2_CH, np = min(A2_CH, cnt - p0);
+      for (int idx = tid; idx < A2_CH * 2 * PPR; idx += 128) {
+        const int p = idx / (2 * PPR), which = (idx / PPR) & 1, pc = idx - (idx / PPR) * PPR;
+        T* dst = &sm.kv[st][which][p][pc * EPP];
+        const bool ok = p < np;
+        const T* src = ok ? kv + kv_off<T>(plane, sm.sl[q][p0 + p], which, S, d) + (size_t)h * HD + pc * EPP
+                          : kv;
+        cp_async16(dst, src, ok);
+      }
+      cp_async_commit();
+      ++ci;
+      if (++ji == sm.rec[q][6]) {
+        ji = 0;
+        ++ki;
+      }
+    }
+  };
+  if constexpr (!FUSED) {  // the rows of a prefill chunk read each other's fresh cache rows
+    pdl_wait();
+    pdl_trigger();
+  }
+  // fused: every ring stage is requested before the dependency wait (the cache
+  // rows of earlier positions were written by earlier kernels)
+  issue_upto(FUSED ? NS : NS - 1);
+  if constexpr (FUSED) {
+    pdl_wait();
+    pdl_trigger();
+  }
+
+  const int hw = tid >> 4, l16 = tid & 15;
+  const float scale = rsqrtf((float)HD);
+  const int half = HD / 2;
+  // the (row, head) run in progress: its splits done here since the last ticket
+  int cur_i = -1, cur_h = -1, cur_ns = 0, npend = 0;
+  // Ticket for the run's npend splits; the block that completes the (row, head)
+  // merges all its splits in split order (deterministic whichever block is last).
+  auto finish_run = [&]() {
+    asm volatile("fence.acq_rel.gpu;" ::: "memory");  // release: the run's partials
+    __syncthreads();
+    if (tid == 0) {
+      const int ticket = atomicAdd(&a.counters[cur_i * H + cur_h], npend);
+      sm.last = ticket + npend == cur_ns;
+      if (sm.last) a.counters[cur_i * H + cur_h] = 0;
+    }
+    __syncthreads();
+    if (sm.last) {
+      asm volatile("fence.acq_rel.gpu;" ::: "memory");  // acquire: the other blocks' partials
+      const int ns = cur_ns;
+      const float* base = a.opart + (size_t)(cur_i * H + cur_h) * a.max_splits * (HD + 2);
+      constexpr int ATT_MB = 16;
+      constexpr int CAP = 4 * HD;  // splits whose (max, sum) fit in hacc
+      float* sM = &sm.hacc[0][0];
+      float* sL = sM + CAP;
+      const int e2 = tid;
+      float av[ATT_MB];
+#pragma unroll
+      for (int kk = 0; kk < ATT_MB; ++kk)
+        av[kk] = (e2 < HD && kk < ns) ? __ldcg(base + (size_t)kk * (HD + 2) + 2 + e2) : 0.f;
+      if (ns <= CAP) {
+        for (int s2 = tid; s2 < ns; s2 += 128) {
+          sM[s2] = __ldcg(base + (size_t)s2 * (HD + 2));
+          sL[s2] = __ldcg(base + (size_t)s2 * (HD + 2) + 1);
+        }
+      }
+      __syncthreads();
+      auto mx_of = [&](int s2) { return ns <= CAP ? sM[s2] : __ldcg(base + (size_t)s2 * (HD + 2)); };
+      auto l_of = [&](int s2) { return ns <= CAP ? sL[s2] : __ldcg(base + (size_t)s2 * (HD + 2) + 1); };
+      float Mx = -INFINITY;
+      for (int s2 = 0; s2 < ns; ++s2) Mx = fmaxf(Mx, mx_of(s2));
+      float Lx = 0.f;
+      for (int s2 = 0; s2 < ns; ++s2) Lx += l_of(s2) * __expf(mx_of(s2) - Mx);
+      if (e2 < HD) {
+        float o = 0.f;
+#pragma unroll
+        for (int kk = 0; kk < ATT_MB; ++kk)
+          if (kk < ns) o += av[kk] * __expf(mx_of(kk) - Mx);
+        for (int s2 = ATT_MB; s2 < ns; ++s2)
+          o += __ldcg(base + (size_t)s2 * (HD + 2) + 2 + e2) * __expf(mx_of(s2) - Mx);
+        store_act<T>(reinterpret_cast<T*>(a.X) + (size_t)cur_i * d + cur_h * HD, e2, o / Lx, a.lo);
+      }
+      __syncthreads();  // hacc is reused
+    }
+    npend = 0;
+  };
+
+  float qv[EPL];
+  for (int k = 0; k < nit; ++k) {
+    const int q = k % NS;
+    const int i = sm.rec[q][0], sp = sm.rec[q][1], ns = sm.rec[q][2], h = sm.rec[q][3];
+    const int cnt = sm.rec[q][4], plane = sm.rec[q][5], nch = sm.rec[q][6];
+    const bool own = sp == ns - 1;  // this unit holds the row's own position
+    const bool newrun = i != cur_i || h != cur_h;
+    if (newrun && npend > 0) finish_run();
+    cur_i = i;
+    cur_h = h;
+    cur_ns = ns;
+    const int n = sm.rpos[i] + 1;
+    if constexpr (FUSED) {
+      if (newrun || own) {
+        // q (RoPE) from the QKV partials at a run's start; in the own unit also
+        // k (RoPE) and v, which go to the row's cache slot and into the ring at
+        // the own position
+        const float rr = sm.rr[i];
+        const int t = tid;
+        const bool is_k = t >= half && t < 2 * half;
+        const int e = t < half ? t : t - half;
+        const bool do_pair = t < 2 * half && (is_k ? own : newrun);
+        float a1 = 0.f, a2 = 0.f, av = 0.f;
+        float2 cs = make_float2(1.f, 0.f);
+        if (do_pair) {
+          const int nA = (is_k ? d : 0) + h * HD + e;
+          const int nB = nA + half;
+          const int4 tiA = __ldg(a.qs_shape.tinfo + (nA >> 7));
+          const int4 tiB = __ldg(a.qs_shape.tinfo + (nB >> 7));
+          cs = a.rope[(size_t)(n - 1) * half + e];
+          a1 = rr * sk_reduce_ti(a.part, a.qs_shape, tiA, C, i, nA);
+          a2 = rr * sk_reduce_ti(a.part, a.qs_shape, tiB, C, i, nB);
+        }
+        if (own && t < HD) {
+          const int nV = 2 * d + h * HD + t;
+          av = rr * sk_reduce_ti(a.part, a.qs_shape, __ldg(a.qs_shape.tinfo + (nV >> 7)), C, i, nV);
+        }
+        if (do_pair) {
+          const float r1 = a1 * cs.x - a2 * cs.y, r2 = a2 * cs.x + a1 * cs.y;
+          if (is_k) {
+            T* krow = kv + kv_off<T>(plane, sm.rslot[i], 0, S, d) + (size_t)h * HD;
+            krow[e] = from_f<T>(r1);
+            krow[e + half] = from_f<T>(r2);
+            sm.own_k[e] = to_f<T>(from_f<T>(r1));
+            sm.own_k[e + half] = to_f<T>(from_f<T>(r2));
+          } else {
+            sm.qsm[e] = r1;
+            sm.qsm[e + half] = r2;
+          }
+        }
+        if (own && t < HD) {
+          T* vrow = kv + kv_off<T>(plane, sm.rslot[i], 1, S, d) + (size_t)h * HD;
+          vrow[t] = from_f<T>(av);
+          sm.own_v[t] = to_f<T>(from_f<T>(av));
+        }
+        __syncthreads();
+        if (newrun) {
+#pragma unroll
+          for (int e2 = 0; e2 < EPL; ++e2) qv[e2] = sm.qsm[l16 * EPL + e2] * scale;
+        }
+      }
+    } else {
+      if (newrun) {
+        load_vec<float, EPL>(a.q + (size_t)i * d + h * HD + l16 * EPL, qv);
+#pragma unroll
+        for (int e2 = 0; e2 < EPL; ++e2) qv[e2] *= scale;
+      }
+    }
+    float m = -INFINITY, l = 0.f, acc[EPL];
+#pragma unroll
+    for (int e2 = 0; e2 < EPL; ++e2) acc[e2] = 0.f;
+    for (int jc = 0; jc < nch; ++jc, ++cc) {
+      issue_upto(cc + NS);               // keep NS - 1 chunks ahead of this one
+      cp_async_wait_upto3(ci - 1 - cc);  // this thread's copies of chunk cc have landed
+      __syncthreads();                   // ... and every thread's
+      const int st = cc % NS;
+      const int p0 = jc * A2_CH;
+      if constexpr (FUSED) {
+        const int pown = (cnt - 1) - p0;  // the own position, if it is in this chunk
+        if (own && pown >= 0 && pown < A2_CH) {
+          if (tid < HD) {
+            sm.kv[st][0][pown][tid] = from_f<T>(sm.own_k[tid]);
+            sm.kv[st][1][pown][tid] = from_f<T>(sm.own_v[tid]);
+          }
+          __syncthreads();
+        }
+      }
+      // positions hw * 8 .. hw * 8 + 7 of the chunk (attn_item's assignment)
+      constexpr int U = 8;
+      const int t0 = p0 + hw * U;
+      float sc[U];
+      RawVec<T, EPL> vx[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int pl = hw * U + u;
+        RawVec<T, EPL> kx;
+        const uint32_t* kp = reinterpret_cast<const uint32_t*>(&sm.kv[st][0][pl][l16 * EPL]);
+        const uint32_t* vp = reinterpret_cast<const uint32_t*>(&sm.kv[st][1][pl][l16 * EPL]);
+#pragma unroll
+        for (int c2 = 0; c2 < RawVec<T, EPL>::WORDS; ++c2) {
+          kx.w[c2] = kp[c2];
+          vx[u].w[c2] = vp[c2];
+        }
+        float dot = 0.f;
+#pragma unroll
+        for (int e2 = 0; e2 < EPL; ++e2) dot += qv[e2] * kx.get(e2);
+        sc[u] = dot;
+      }
+#pragma unroll
+      for (int o = 8; o > 0; o >>= 1)
+#pragma unroll
+        for (int u = 0; u < U; ++u) sc[u] += __shfl_xor_sync(0xffffffffu, sc[u], o);
+      float mloc = -INFINITY;
+#pragma unroll
+      for (int u = 0; u < U; ++u)
+        if (t0 + u < cnt) mloc = fmaxf(mloc, sc[u]);
+      if (mloc != -INFINITY) {
+        const float mnew = fmaxf(m, mloc);
+        const float c = __expf(m - mnew);
+        l *= c;
+#pragma unroll
+        for (int e2 = 0; e2 < EPL; ++e2) acc[e2] *= c;
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          if (t0 + u < cnt) {
+            const float wgt = __expf(sc[u] - mnew);
+            l += wgt;
+#pragma unroll
+            for (int e2 = 0; e2 < EPL; ++e2) acc[e2] += wgt * vx[u].get(e2);
+          }
+        }
+        m = mnew;
+      }
+      __syncthreads();  // ring stage st may be refilled
+    }
+    // merge the half-warps in fixed order, write the split's partial
+    if (l16 == 0) {
+      sm.hm[hw] = m;
+      sm.hl[hw] = l;
+    }
+#pragma unroll
+    for (int e2 = 0; e2 < EPL; ++e2) sm.hacc[hw][l16 * EPL + e2] = acc[e2];
+    __syncthreads();
+    float M = -INFINITY;
+#pragma unroll
+    for (int w2 = 0; w2 < 8; ++w2) M = fmaxf(M, sm.hm[w2]);
+    float* out = a.opart + ((size_t)(i * H + h) * a.max_splits + sp) * (HD + 2);
+    for (int e2 = tid; e2 < HD; e2 += 128) {
+      float v = 0.f;
+#pragma unroll
+      for (int w2 = 0; w2 < 8; ++w2)
+        if (sm.hm[w2] != -INFINITY) v += sm.hacc[w2][e2] * __expf(sm.hm[w2] - M);
+      out[2 + e2] = v;
+    }
+    if (tid == 0) {
+      float L = 0.f;
+#pragma unroll
+      for (int w2 = 0; w2 < 8; ++w2)
+        if (sm.hm[w2] != -INFINITY) L += sm.hl[w2] * __expf(sm.hm[w2] - M);
+      out[0] = M;
+      out[1] = L;
+    }
+    ++npend;
+    __syncthreads();  // hacc, qsm and the unit record are reused
+  }
+  finish_run();
+}
+
 // ---- RoPE table: (cos, sin) of pos * theta^(-2e/hd), computed in double ------------
 static __global__ void k_rope_table(float2* __restrict__ rope, int max_pos, int hd, double theta) {
   const int half = hd / 2;

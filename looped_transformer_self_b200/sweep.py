@@ -8,7 +8,7 @@ CUDA graph and replayed; reported: median pass time, algorithmic bytes
 (shared-block weights + every row's K/V reads and writes) and GB/s against the
 measured HBM copy bandwidth.
 
-Usage: python -m looped_transformer_self_b200.sweep [M ...]
+Usage: python -m looped_transformer_self_b200.sweep [M ...] [--layers N] [--iters K]
 """
 from __future__ import annotations
 
@@ -27,8 +27,10 @@ from .binding import Decoder
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
-def run(Ms=(1, 2, 4, 8, 16, 32, 64), iters=50, device="cuda"):
+def run(Ms=(1, 2, 4, 8, 16, 32, 64), iters=50, device="cuda", layers=None):
     cfg = syn.MODELS["sweep"]
+    if layers:  # fewer shared layers: a small case of the same kernels (profilers)
+        cfg = cfg.replace(n_core=layers)
     d = cfg.d_model
     try:
         hbm = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))["hbm_gbs"]
@@ -75,5 +77,10 @@ def run(Ms=(1, 2, 4, 8, 16, 32, 64), iters=50, device="cuda"):
 
 
 if __name__ == "__main__":
-    Ms = tuple(int(x) for x in sys.argv[1:]) or (1, 2, 4, 8, 16, 32, 64)
-    run(Ms)
+    import argparse
+    ap = argparse.ArgumentParser()
+    ap.add_argument("M", type=int, nargs="*", default=[1, 2, 4, 8, 16, 32, 64])
+    ap.add_argument("--layers", type=int, default=None, help="shared layers (default 24)")
+    ap.add_argument("--iters", type=int, default=50, help="graph replays per M")
+    a = ap.parse_args()
+    run(tuple(a.M), iters=a.iters, layers=a.layers)
