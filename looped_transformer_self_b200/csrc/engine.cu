@@ -386,36 +386,18 @@ static AttnArgs attn_args(Handle* H, int gl, const int* tagsrc, int tag_off, voi
   a.ssq_tiles = H->ssq_tiles;
   a.eps = H->m.rms_eps;
   a.err = &D.ctl->err;
-  const char* pf = getenv("LT_ATT_PREFETCH");
-  a.kv_prefetch = pf ? atoi(pf) : 1;
   return a;
 }
 
-// Long contexts: one block per (head, work item) slot, blocks looping over items
-// (k_attn; the same bits as k_attn2).
-template <typename T, int HD>
-static cudaError_t attention_items(Handle* H, int gl, const int* tagsrc, int tag_off,
-                                   const int* mask, T* Xo, bool fused) {
-  const int C = H->C, Hn = H->m.n_heads;
-  auto kern = fused ? k_attn<T, HD, true> : k_attn<T, HD, false>;
-  // occupancy is a property of the device: cached per device ordinal
-  static int per_sm[kMaxDev][2] = {};
-  int& nb = per_sm[cur_dev()][fused ? 1 : 0];
-  if (nb == 0 && (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kern, 128, 0) != cudaSuccess ||
-                  nb < 1))
-    nb = 1;
-  const int gy = std::max(1, std::min(C * H->max_splits, nb * sm_count() / Hn));
-  return launch(H->use_pdl, kern, dim3(Hn, gy), dim3(128), H->stream,
-                attn_args(H, gl, tagsrc, tag_off, (void*)Xo), mask);
-}
-
-// Long contexts: one resident wave of ring blocks, each streaming a contiguous
-// range of (head, row, split) units (k_attn3; the same bits as k_attn2).
-template <typename T, int HD>
-static cudaError_t attention_ranges(Handle* H, int gl, const int* tagsrc, int tag_off,
-                                    const int* mask, T* Xo, bool fused) {
-  auto kern = fused ? k_attn3<T, HD, true> : k_attn3<T, HD, false>;
-  const size_t smem = a3_smem_bytes<T, HD>();
+// One resident wave of attention blocks, each streaming a contiguous range of
+// (head, row, split) units (k_attn).  The shared-memory attribute is set per
+// device (function attributes belong to a context), and the occupancy that
+// follows from it is cached with it.
+template <typename T, int HD, int NS>
+static cudaError_t attention_ns(Handle* H, int gl, const int* tagsrc, int tag_off, const int* mask,
+                                T* Xo, bool fused) {
+  auto kern = fused ? k_attn<T, HD, NS, true> : k_attn<T, HD, NS, false>;
+  const size_t smem = attn_smem_bytes<T, HD, NS>();
   static int per_sm[kMaxDev][2] = {};
   int& nb = per_sm[cur_dev()][fused ? 1 : 0];
   if (nb == 0) {
@@ -443,37 +425,9 @@ template <typename T, int HD>
 static cudaError_t attention(Handle* H, int gl, const int* tagsrc, int tag_off, const int* mask,
                              T* Xo, bool fused) {
   ProfScope ps(H, 2, 0.0);
-  if (H->dc.max_ctx > ATT_RING_MAX_CTX) {
-    static const char* e = getenv("LT_ATT_LONG");
-    if (e && !strcmp(e, "regs")) return attention_items<T, HD>(H, gl, tagsrc, tag_off, mask, Xo, fused);
-    return attention_ranges<T, HD>(H, gl, tagsrc, tag_off, mask, Xo, fused);
-  }
-  auto kern = fused ? k_attn2<T, HD, true> : k_attn2<T, HD, false>;
-  // one resident wave of ring blocks (items are spread over them)
-  const size_t smem = a2_smem_bytes<T, HD>();
-  // the shared-memory attribute is set per device (function attributes belong
-  // to a context), and the occupancy that follows from it is cached with it
-  static int per_sm[kMaxDev][2] = {};
-  int& nb = per_sm[cur_dev()][fused ? 1 : 0];
-  if (nb == 0) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-        cudaSuccess)
-      return cudaErrorInvalidValue;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kern, 128, smem) != cudaSuccess || nb < 1)
-      nb = 1;
-  }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(nb * sm_count());
-  cfg.blockDim = dim3(128);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = H->stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = H->use_pdl ? 1 : 0;
-  if (H->counting) H->kernels_per_step++;
-  return cudaLaunchKernelEx(&cfg, kern, attn_args(H, gl, tagsrc, tag_off, (void*)Xo), mask);
+  static const char* ns = getenv("LT_ATT_STAGES");  // ring depth override (tuning)
+  if (ns && atoi(ns) == 3) return attention_ns<T, HD, 3>(H, gl, tagsrc, tag_off, mask, Xo, fused);
+  return attention_ns<T, HD, attn_stages<T, HD>()>(H, gl, tagsrc, tag_off, mask, Xo, fused);
 }
 
 // kind: 0 prelude (one cache), 1 shared block (cache of the row's depth), 2 coda

@@ -2,13 +2,13 @@
 
 M = 1, 2, 4, 8, 16, 32, 64 active rows; each row at an independent depth 1..4
 with its own KV length drawn uniformly from 256..8192 (synthetic.sweep_rows),
-its own randomly permuted cache slots, caches and hidden states N(0, 1).  One
+its own randomly permuted (or, --order seq, ascending) cache slots, caches and hidden states N(0, 1).  One
 pass = all 24 shared layers over the M rows (lt_block_pass), captured as a
 CUDA graph and replayed; reported: median pass time, algorithmic bytes
 (shared-block weights + every row's K/V reads and writes) and GB/s against the
 measured HBM copy bandwidth.
 
-Usage: python -m looped_transformer_self_b200.sweep [M ...] [--layers N] [--iters K]
+Usage: python -m looped_transformer_self_b200.sweep [M ...] [--layers N] [--iters K] [--order perm|seq]
 """
 from __future__ import annotations
 
@@ -27,7 +27,7 @@ from .binding import Decoder
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
-def run(Ms=(1, 2, 4, 8, 16, 32, 64), iters=50, device="cuda", layers=None):
+def run(Ms=(1, 2, 4, 8, 16, 32, 64), iters=50, device="cuda", layers=None, order="perm"):
     cfg = syn.MODELS["sweep"]
     if layers:  # fewer shared layers: a small case of the same kernels (profilers)
         cfg = cfg.replace(n_core=layers)
@@ -49,7 +49,8 @@ def run(Ms=(1, 2, 4, 8, 16, 32, 64), iters=50, device="cuda", layers=None):
             start = nxt.get(r, 0)
             nxt[r] = start + l + 1
             offs.append(sum(len(x) for x in lists))
-            lists.append(rng.permutation(np.arange(start, start + l + 1)).astype(np.int32))
+            sl = np.arange(start, start + l + 1)
+            lists.append((rng.permutation(sl) if order == "perm" else sl).astype(np.int32))
         S = max(nxt.values())
         g = Decoder(cfg, syn.DecodeConfig(1, 2, 0.0, 1.0, 2, 1), None, max_branches=C,
                     max_ctx=max(S, 8200), device=device)
@@ -82,5 +83,7 @@ if __name__ == "__main__":
     ap.add_argument("M", type=int, nargs="*", default=[1, 2, 4, 8, 16, 32, 64])
     ap.add_argument("--layers", type=int, default=None, help="shared layers (default 24)")
     ap.add_argument("--iters", type=int, default=50, help="graph replays per M")
+    ap.add_argument("--order", choices=("perm", "seq"), default="perm",
+                    help="slot order of each row's list: permuted (default) or ascending")
     a = ap.parse_args()
-    run(tuple(a.M), iters=a.iters, layers=a.layers)
+    run(tuple(a.M), iters=a.iters, layers=a.layers, order=a.order)
