@@ -214,6 +214,10 @@ __device__ __forceinline__ void cp_async16(void* dst, const void* src, bool vali
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(src), "r"(n)
                : "memory");
 }
+__device__ __forceinline__ void cp_async16_full(void* dst, const void* src) {
+  const uint32_t d = (uint32_t)__cvta_generic_to_shared(dst);
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(src) : "memory");
+}
 __device__ __forceinline__ void cp_async_commit() {
   asm volatile("cp.async.commit_group;" ::: "memory");
 }
@@ -285,6 +289,35 @@ __device__ __forceinline__ float piece_elem(const uint32_t* w, int t) {
     return __uint_as_float((t & 1) ? (w[t >> 1] & 0xFFFF0000u) : (w[t >> 1] << 16));
   else
     return __uint_as_float(w[t]);
+}
+
+// bf16 caches: products of two bf16 halves accumulated in fp32 with one rounding
+// per step (a bf16 product is exact in fp32, so each step equals fmaf of the
+// widened operands); saves the widening instruction per element.
+// c + a.lo * b.lo + a.hi * b.hi, in that order
+__device__ __forceinline__ float fma_bf16_pair(uint32_t a, uint32_t b, float c) {
+  asm("{\n\t.reg .b16 al, ah, bl, bh;\n\t"
+      "mov.b32 {al, ah}, %1;\n\t"
+      "mov.b32 {bl, bh}, %2;\n\t"
+      "fma.rn.f32.bf16 %0, al, bl, %0;\n\t"
+      "fma.rn.f32.bf16 %0, ah, bh, %0;\n\t}"
+      : "+f"(c)
+      : "r"(a), "r"(b));
+  return c;
+}
+// a0 += v.lo * w.lo, a1 += v.hi * w.hi
+__device__ __forceinline__ void fma_bf16_split(uint32_t v, uint32_t w, float& a0, float& a1) {
+  asm("{\n\t.reg .b16 vl, vh, wl, wh;\n\t"
+      "mov.b32 {vl, vh}, %2;\n\t"
+      "mov.b32 {wl, wh}, %3;\n\t"
+      "fma.rn.f32.bf16 %0, vl, wl, %0;\n\t"
+      "fma.rn.f32.bf16 %1, vh, wh, %1;\n\t}"
+      : "+f"(a0), "+f"(a1)
+      : "r"(v), "r"(w));
+}
+__device__ __forceinline__ uint32_t bf16x2_bits(float lo, float hi) {
+  const __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&b);
 }
 
 // ring depth: two stages (one chunk ahead) keep three blocks per SM for bf16,
@@ -436,12 +469,20 @@ __global__ void __launch_bounds__(128) k_attn(const AttnArgs a, const int* __res
         if (pc < PPR) {
           const T* src0 = kv + kv_off<T>(plane, 0, which, S, d) + (size_t)h * HD + pc * EPP16;
           const int* sl = &sm.sl[q][p0];
+          T* dst0 = &sm.kv[st][which][r0 >> 1][pc * EPP16];
+          constexpr int DSTEP = (RSTEP / 2) * HD;  // elements between a thread's rows
+          const size_t sstride = 2 * (size_t)d;
+          if (np == ATT_CHUNK) {  // a full chunk: no predicates
 #pragma unroll 4
-          for (int k = 0; k < NCOPY; ++k) {
-            const int p = (r0 >> 1) + k * (RSTEP / 2);
-            const bool ok = p < np;
-            const T* src = ok ? src0 + (size_t)sl[p] * (2 * (size_t)d) : kv;
-            cp_async16(&sm.kv[st][which][p][pc * EPP16], src, ok);
+            for (int k = 0; k < NCOPY; ++k)
+              cp_async16_full(dst0 + k * DSTEP, src0 + (size_t)sl[(r0 >> 1) + k * (RSTEP / 2)] * sstride);
+          } else {
+#pragma unroll 4
+            for (int k = 0; k < NCOPY; ++k) {
+              const int p = (r0 >> 1) + k * (RSTEP / 2);
+              const bool ok = p < np;
+              cp_async16(dst0 + k * DSTEP, ok ? src0 + (size_t)sl[p] * sstride : kv, ok);
+            }
           }
         }
         cp_async_commit();
@@ -522,7 +563,15 @@ __global__ void __launch_bounds__(128) k_attn(const AttnArgs a, const int* __res
     npend = 0;
   };
 
+  // the query, scaled: fp32 (fp32 caches) or bf16 pairs in the cache's word layout
   float qv[L::EL];
+  uint32_t qb[L::EL / 2];
+  auto pack_q = [&]() {
+    if constexpr (sizeof(T) == 2) {
+#pragma unroll
+      for (int t2 = 0; t2 < L::EL / 2; ++t2) qb[t2] = bf16x2_bits(qv[2 * t2], qv[2 * t2 + 1]);
+    }
+  };
   for (int k = 0; k < nit; ++k) {
     const int q = k % NS;
     const int i = sm.rec[q][0], sp = sm.rec[q][1], ns = sm.rec[q][2], h = sm.rec[q][3];
@@ -584,6 +633,7 @@ __global__ void __launch_bounds__(128) k_attn(const AttnArgs a, const int* __res
 #pragma unroll
             for (int t2 = 0; t2 < L::EPP; ++t2)
               qv[kp * L::EPP + t2] = sm.qsm[(kp * 8 + j) * L::EPP + t2] * scale;
+          pack_q();
         }
       }
     } else {
@@ -593,6 +643,7 @@ __global__ void __launch_bounds__(128) k_attn(const AttnArgs a, const int* __res
         for (int kp = 0; kp < L::NP; ++kp)
 #pragma unroll
           for (int t2 = 0; t2 < L::EPP; ++t2) qv[kp * L::EPP + t2] = qrow[(kp * 8 + j) * L::EPP + t2] * scale;
+        pack_q();
       }
     }
     float m = -INFINITY, l = 0.f, acc[L::EL];
@@ -626,8 +677,13 @@ __global__ void __launch_bounds__(128) k_attn(const AttnArgs a, const int* __res
           uint32_t w[L::PB / 4];
           lds_piece<L::PB>(krow + (kp * 8 + j) * L::EPP, w);
           float pd = 0.f;
+          if constexpr (sizeof(T) == 2) {
 #pragma unroll
-          for (int t2 = 0; t2 < L::EPP; ++t2) pd = fmaf(qv[kp * L::EPP + t2], piece_elem<T>(w, t2), pd);
+            for (int w2 = 0; w2 < L::EPP / 2; ++w2) pd = fma_bf16_pair(w[w2], qb[kp * L::EPP / 2 + w2], pd);
+          } else {
+#pragma unroll
+            for (int t2 = 0; t2 < L::EPP; ++t2) pd = fmaf(qv[kp * L::EPP + t2], piece_elem<T>(w, t2), pd);
+          }
           dot += pd;
         }
         sc[k4] = dot;
@@ -650,13 +706,21 @@ __global__ void __launch_bounds__(128) k_attn(const AttnArgs a, const int* __res
 #pragma unroll
       for (int k4 = 0; k4 < 4; ++k4) {
         const T* vrow = &sm.kv[st][1][g + 16 * k4][0];
+        // bf16 caches: the weight in bf16, as the V operand (bf16 attention's usual P)
+        const uint32_t wb = sizeof(T) == 2 ? bf16x2_bits(wk[k4], wk[k4]) : 0u;
 #pragma unroll
         for (int kp = 0; kp < L::NP; ++kp) {
           uint32_t w[L::PB / 4];
           lds_piece<L::PB>(vrow + (kp * 8 + j) * L::EPP, w);
+          if constexpr (sizeof(T) == 2) {
 #pragma unroll
-          for (int t2 = 0; t2 < L::EPP; ++t2)
-            acc[kp * L::EPP + t2] = fmaf(wk[k4], piece_elem<T>(w, t2), acc[kp * L::EPP + t2]);
+            for (int w2 = 0; w2 < L::EPP / 2; ++w2)
+              fma_bf16_split(w[w2], wb, acc[kp * L::EPP + 2 * w2], acc[kp * L::EPP + 2 * w2 + 1]);
+          } else {
+#pragma unroll
+            for (int t2 = 0; t2 < L::EPP; ++t2)
+              acc[kp * L::EPP + t2] = fmaf(wk[k4], piece_elem<T>(w, t2), acc[kp * L::EPP + t2]);
+          }
         }
       }
       m = mnew;
