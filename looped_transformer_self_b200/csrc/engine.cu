@@ -425,8 +425,6 @@ template <typename T, int HD>
 static cudaError_t attention(Handle* H, int gl, const int* tagsrc, int tag_off, const int* mask,
                              T* Xo, bool fused) {
   ProfScope ps(H, 2, 0.0);
-  static const char* ns = getenv("LT_ATT_STAGES");  // ring depth override (tuning)
-  if (ns && atoi(ns) == 3) return attention_ns<T, HD, 3>(H, gl, tagsrc, tag_off, mask, Xo, fused);
   return attention_ns<T, HD, attn_stages<T, HD>()>(H, gl, tagsrc, tag_off, mask, Xo, fused);
 }
 

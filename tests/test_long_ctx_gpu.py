@@ -111,8 +111,8 @@ def test_rows_are_batch_invariant_bitwise(cfg):
 
 
 def test_tiny_long_prompt_decode_matches_oracle():
-    """Tiny fp32 model, 1200-token prompt, max_ctx 4096 (register-path
-    attention; 10-11 splits per row): prefill logits at sampled positions and
+    """Tiny fp32 model, 1200-token prompt, max_ctx 4096 (10-11 attention
+    splits per row, fp32 cache path): prefill logits at sampled positions and
     every readout depth within 1e-4 of the oracle; greedy speculative decoding
     equals GPU AR and its integer work is bit-exact against the oracle."""
     from oracle import decode as D
