@@ -344,7 +344,7 @@ __device__ __forceinline__ void cp_async_wait(int pending) {
 }
 
 template <typename T, int HD, int NS, bool FUSED>
-__global__ void __launch_bounds__(128) k_attn(const AttnArgs a, const int* __restrict__ mask) {
+__global__ void __launch_bounds__(128, 3) k_attn(const AttnArgs a, const int* __restrict__ mask) {
   static_assert(NS >= 2 && NS <= 4, "cp_async_wait covers up to three pending chunks");
   using L = AttnLane<T, HD>;
   extern __shared__ __align__(16) unsigned char attn_raw[];
@@ -665,24 +665,30 @@ __global__ void __launch_bounds__(128) k_attn(const AttnArgs a, const int* __res
           __syncthreads();
         }
       }
-      // scores of the group's four positions: the lane's partial dot product,
-      // then a butterfly over the group's 8 lanes
+      // the group's four positions: every K and V piece of the lane is loaded
+      // first (independent shared-memory loads in flight together), then the
+      // lane's partial dot products and a butterfly over the group's 8 lanes
+      uint32_t kw[4][L::NP][L::PB / 4], vw[4][L::NP][L::PB / 4];
+#pragma unroll
+      for (int k4 = 0; k4 < 4; ++k4)
+#pragma unroll
+        for (int kp = 0; kp < L::NP; ++kp) {
+          lds_piece<L::PB>(&sm.kv[st][0][g + 16 * k4][(kp * 8 + j) * L::EPP], kw[k4][kp]);
+          lds_piece<L::PB>(&sm.kv[st][1][g + 16 * k4][(kp * 8 + j) * L::EPP], vw[k4][kp]);
+        }
       float sc[4];
 #pragma unroll
       for (int k4 = 0; k4 < 4; ++k4) {
-        const T* krow = &sm.kv[st][0][g + 16 * k4][0];
         float dot = 0.f;
 #pragma unroll
         for (int kp = 0; kp < L::NP; ++kp) {
-          uint32_t w[L::PB / 4];
-          lds_piece<L::PB>(krow + (kp * 8 + j) * L::EPP, w);
           float pd = 0.f;
           if constexpr (sizeof(T) == 2) {
 #pragma unroll
-            for (int w2 = 0; w2 < L::EPP / 2; ++w2) pd = fma_bf16_pair(w[w2], qb[kp * L::EPP / 2 + w2], pd);
+            for (int w2 = 0; w2 < L::EPP / 2; ++w2) pd = fma_bf16_pair(kw[k4][kp][w2], qb[kp * L::EPP / 2 + w2], pd);
           } else {
 #pragma unroll
-            for (int t2 = 0; t2 < L::EPP; ++t2) pd = fmaf(qv[kp * L::EPP + t2], piece_elem<T>(w, t2), pd);
+            for (int t2 = 0; t2 < L::EPP; ++t2) pd = fmaf(qv[kp * L::EPP + t2], piece_elem<T>(kw[k4][kp], t2), pd);
           }
           dot += pd;
         }
@@ -705,21 +711,18 @@ __global__ void __launch_bounds__(128) k_attn(const AttnArgs a, const int* __res
       for (int e2 = 0; e2 < L::EL; ++e2) acc[e2] *= c;
 #pragma unroll
       for (int k4 = 0; k4 < 4; ++k4) {
-        const T* vrow = &sm.kv[st][1][g + 16 * k4][0];
         // bf16 caches: the weight in bf16, as the V operand (bf16 attention's usual P)
         const uint32_t wb = sizeof(T) == 2 ? bf16x2_bits(wk[k4], wk[k4]) : 0u;
 #pragma unroll
         for (int kp = 0; kp < L::NP; ++kp) {
-          uint32_t w[L::PB / 4];
-          lds_piece<L::PB>(vrow + (kp * 8 + j) * L::EPP, w);
           if constexpr (sizeof(T) == 2) {
 #pragma unroll
             for (int w2 = 0; w2 < L::EPP / 2; ++w2)
-              fma_bf16_split(w[w2], wb, acc[kp * L::EPP + 2 * w2], acc[kp * L::EPP + 2 * w2 + 1]);
+              fma_bf16_split(vw[k4][kp][w2], wb, acc[kp * L::EPP + 2 * w2], acc[kp * L::EPP + 2 * w2 + 1]);
           } else {
 #pragma unroll
             for (int t2 = 0; t2 < L::EPP; ++t2)
-              acc[kp * L::EPP + t2] = fmaf(wk[k4], piece_elem<T>(w, t2), acc[kp * L::EPP + t2]);
+              acc[kp * L::EPP + t2] = fmaf(wk[k4], piece_elem<T>(vw[k4][kp], t2), acc[kp * L::EPP + t2]);
           }
         }
       }
