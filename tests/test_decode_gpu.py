@@ -375,3 +375,47 @@ def test_sampled_readout_distributions_match_oracle(V, top_p):
             checked += 1
     assert checked >= 6
     g.close()
+
+
+@pytest.mark.parametrize("V,top_p", [(49152, 0.95), (65539, 0.9)])
+def test_sampled_decode_does_not_read_stale_workspace(V, top_p):
+    """Sampled decoding with the cluster readout over a workspace that starts as
+    zeros and over one that starts as finite garbage (0x3F bytes): the readouts
+    (logits, processed distributions, argmax), the committed tokens and the
+    branch table after every step are identical bit for bit, so no kernel of the
+    sampled step reads device memory before writing it."""
+    from looped_transformer_self_b200.binding import Decoder
+    cfg = syn.ModelConfig("bf16_bigv", "bf16", 256, 2, 128, 512, V, 0, 2, 0, 4,
+                          resid_scale=0.5, head_gain=4.0, seed=3)
+    dec = syn.DecodeConfig(1, 2, 1.0, top_p, 5, 6)
+    w = syn.make_weights(cfg)
+    runs = []
+    for fill in (0, 0x3F):
+        g = Decoder(cfg, dec, w, max_branches=16, max_ctx=64, workspace_fill=fill)
+        g.prefill(syn.uniform_prompt(12, V, seed=4))
+        rec = []
+        for _ in range(6):
+            g.step()
+            lg, pr, am = g.read_readouts()
+            rec.append((lg, pr, am, g.read_table()))
+        toks, _ = g.read_committed()
+        rec.append(np.array(toks))
+        runs.append(rec)
+        g.close()
+    compared = 0
+    for (lg0, pr0, am0, t0), (lg1, pr1, am1, t1) in zip(runs[0][:-1], runs[1][:-1]):
+        # the alive flags of every entry, and every field of the live entries (a
+        # dead entry's other fields keep whatever they held, the initial bytes
+        # for entries never used)
+        np.testing.assert_array_equal(t0[0], t1[0])
+        live = t0[0] != 0
+        np.testing.assert_array_equal(t0[:, live], t1[:, live])
+        # rows that hold a readout (written in this step or an earlier one); a row
+        # never read out keeps the initial bytes, which differ by construction
+        rows = np.abs(pr0.astype(np.float64).sum(axis=1) - 1.0) < 1e-3
+        np.testing.assert_array_equal(lg0[rows], lg1[rows])
+        np.testing.assert_array_equal(pr0[rows], pr1[rows])
+        np.testing.assert_array_equal(am0[rows], am1[rows])
+        compared += int(rows.sum())
+    np.testing.assert_array_equal(runs[0][-1], runs[1][-1])
+    assert compared >= 6
