@@ -179,7 +179,7 @@ __global__ void k_qkv_epi(const float* __restrict__ part, const GemmShape s, int
 constexpr int ATT_CHUNK = 64;  // positions per ring stage (16 groups x 4 positions)
 constexpr int ATT_MAXC = 64;   // rows a pass may hold
 
-// Everything one attention work item reads or writes (device pointers).
+// Everything the attention kernel reads or writes (device pointers).
 struct AttnArgs {
   const float* q;            // [C][d] queries (prefill; FUSED reads the QKV partials)
   void* kv;                  // cache pool (T)
@@ -236,7 +236,10 @@ __device__ __forceinline__ void cp_async_commit() {
 // Compute layout: 16 groups of 8 lanes.  Group g takes positions g, g + 16,
 // g + 32 and g + 48 of a chunk.  Lane j of a group takes pieces j, j + 8, ... of
 // a head's K and V rows (PB bytes each), so one shared-memory load per piece
-// reads contiguous bytes across the group.  A group keeps an online softmax state
+// reads contiguous bytes across the group; a lane loads all of its pieces of a
+// chunk before the math.  bf16 caches: the query and the softmax weights enter
+// the products as bf16 (fma.rn.f32.bf16, exact products, fp32 accumulation);
+// fp32 caches: fp32 throughout.  A group keeps an online softmax state
 // (max, sum, accumulator) over its positions of the split.  Positions past the
 // split's end score -inf, and their zero-filled V rows add nothing.  At the
 // split's end the 16 states merge in group order into the split's partial.  The
