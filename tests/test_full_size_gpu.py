@@ -58,3 +58,46 @@ def test_ouro14_prefill_and_greedy_decode_match_oracle(ouro):
             pos = len(prompt) - 1 + k
             assert _margin(sp.logits[(pos, cfg.R)]) <= 0.05, (k, a, b)
             break
+
+
+WIDE = syn.ModelConfig("bf16_wide", "bf16", 2048, 16, 128, 5632, 8192, 0, 2, 0, 2,
+                       resid_scale=0.0137, head_gain=4.942, seed=11)
+
+
+def test_full_width_layers_multi_split_context_match_oracle():
+    """The Ouro layer shapes (d 2048, 16 x 128 heads, ffn 5632, bf16) with two
+    shared layers at R = 2 and a 400-token prompt, so attention runs 4 splits
+    per row spread over several blocks at the benchmark's widths: prefill
+    readout logits at positions in every split and at both depths within
+    relative L-inf 2e-2 of the oracle; greedy speculative decoding equal to GPU
+    full-depth AR bit for bit, and to the oracle wherever the oracle's top-1 /
+    top-2 margin exceeds 0.05."""
+    from looped_transformer_self_b200.binding import Decoder
+    from oracle import decode as D
+    from oracle.model import LoopedModel
+    cfg = WIDE
+    w = syn.make_weights(cfg)
+    prompt = syn.uniform_prompt(400, cfg.vocab, seed=12)
+    n = 4
+    dec = syn.DecodeConfig(1, 0, 0.0, 1.0, 5, n)
+    g = Decoder(cfg, dec, w, max_branches=16, max_ctx=len(prompt) + 16)
+    first, _, lg = g.prefill(prompt, logits=True)
+    lg = lg.cpu().numpy()
+    sp = D.decode_spec(D.OracleRows(LoopedModel(cfg, w, len(prompt) + 16)), prompt, cfg.R, dec.d1,
+                       dec.d2, n, 0.0, 1.0, dec.seed, len(prompt) + 16, keep_logits=True)
+    for pos in (5, 130, 257, 399):
+        for t, r in enumerate((1, 2)):
+            z = sp.logits[(pos, r)]
+            err = np.max(np.abs(lg[pos, t] - z)) / np.max(np.abs(z))
+            assert err < 2e-2, (pos, r, err)
+    toks, _ = g.generate(n)
+    g.prefill(prompt)
+    ar, _ = g.generate(n, ar=True)
+    assert toks == ar
+    gpu = [first] + toks
+    for k, (a, b) in enumerate(zip(gpu, sp.tokens)):
+        if a != b:
+            pos = len(prompt) - 1 + k
+            assert _margin(sp.logits[(pos, cfg.R)]) <= 0.05, (k, a, b)
+            break
+    g.close()
