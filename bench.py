@@ -229,6 +229,29 @@ WORKLOADS = {
 # our arm
 # ---------------------------------------------------------------------------
 
+def gemm_traffic(model, bytes_per_launch, path=None):
+    """DRAM traffic per launch of the dominant kernel, from the committed ncu
+    capture (profiles/gemm_traffic.json), and a note saying where it came from.
+    Reported only while the GEMM sources hash to the captured ones and the
+    capture covers this model's shapes: the capture's traffic / algorithmic
+    ratio over the four shared-block GEMM shapes, applied to this run's
+    algorithmic bytes per launch.  (None, reason) otherwise."""
+    path = path or os.path.join(ROOT, "profiles", "gemm_traffic.json")
+    if not os.path.exists(path):
+        return None, "no capture"
+    from looped_transformer_self_b200.gemm_traffic import source_hash
+    cap = json.load(open(path))
+    if cap.get("source_sha256") != source_hash():
+        return None, "GEMM sources changed since the capture"
+    if cap.get("model") != model:
+        return None, f"the capture covers the {cap.get('model')} shapes"
+    ratio = cap["traffic_per_launch"] / cap["algorithmic_per_launch"]
+    return ratio * bytes_per_launch, (
+        "ncu dram bytes read + written of the four shared-block GEMM shapes "
+        f"(profiles/gemm_traffic.json, ratio to algorithmic {ratio:.4f}); "
+        "the GEMM sources match the capture")
+
+
 def run_ours(args):
     import torch
     import synthetic as syn
@@ -376,25 +399,7 @@ def run_ours(args):
     step_bytes = (prof["gemm_core_bytes"] + prof["gemm_other_bytes"] + prof["kv_bytes"]) / max(prof["steps"], 1)
     graphed_ms = times[-1] / stats["steps"]
     step_gbs = step_bytes / (graphed_ms / 1e3) / 1e9
-    # DRAM traffic of the dominant kernel from an ncu capture, reported only
-    # while the GEMM sources are the ones that capture measured
-    traffic, traffic_note = None, "no capture"
-    tf = os.path.join(ROOT, "profiles", "gemm_traffic.json")
-    if os.path.exists(tf):
-        from looped_transformer_self_b200.gemm_traffic import source_hash
-        cap = json.load(open(tf))
-        if cap.get("source_sha256") != source_hash():
-            traffic_note = "GEMM sources changed since the capture"
-        elif cap.get("model") != args.model:
-            traffic_note = f"the capture covers the {cap.get('model')} shapes"
-        else:
-            # the capture's traffic / algorithmic ratio over the four shared-block
-            # shapes, applied to this run's algorithmic bytes per launch
-            ratio = cap["traffic_per_launch"] / cap["algorithmic_per_launch"]
-            traffic = ratio * pg["bytes"] / pg["launches"]
-            traffic_note = ("ncu dram bytes read + written of the four shared-block GEMM shapes "
-                            f"(profiles/gemm_traffic.json, ratio to algorithmic {ratio:.4f}); "
-                            "the GEMM sources match the capture")
+    traffic, traffic_note = gemm_traffic(args.model, pg["bytes"] / pg["launches"])
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu:

@@ -55,3 +55,34 @@ def test_summary_of_known_launches(tmp_path):
 def test_algorithmic_bytes_formula():
     # bf16 weights [n_out x k] + bf16 rows [ncols x k] + fp32 result [ncols x n_out]
     assert gt.algorithmic_bytes(128, 64, 16) == 2 * 128 * 64 + 2 * 16 * 64 + 4 * 16 * 128
+
+
+def _bench():
+    import importlib.util
+    import os
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    spec = importlib.util.spec_from_file_location("bench_mod", os.path.join(root, "bench.py"))
+    m = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(m)
+    return m
+
+
+def test_bench_reports_traffic_only_for_a_matching_capture(tmp_path):
+    import json
+    bench = _bench()
+    rec = {"model": "huginn35", "source_sha256": gt.source_hash(),
+           "traffic_per_launch": 1.02e8, "algorithmic_per_launch": 1.0e8}
+    p = tmp_path / "cap.json"
+    p.write_text(json.dumps(rec))
+    t, note = bench.gemm_traffic("huginn35", 2.0e8, str(p))
+    assert abs(t - 2.04e8) < 1.0 and "1.0200" in note
+    t, note = bench.gemm_traffic("ouro14", 2.0e8, str(p))
+    assert t is None and "huginn35" in note
+    p.write_text(json.dumps(dict(rec, source_sha256="0" * 64)))
+    t, note = bench.gemm_traffic("huginn35", 2.0e8, str(p))
+    assert t is None and "changed" in note
+    t, note = bench.gemm_traffic("huginn35", 2.0e8, str(tmp_path / "absent.json"))
+    assert t is None and note == "no capture"
+    # the committed capture matches the committed GEMM sources and the default workload
+    t, note = bench.gemm_traffic("huginn35", 1.0e8)
+    assert t is not None and 0.9e8 < t < 1.2e8, note
